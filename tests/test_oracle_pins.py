@@ -1,0 +1,335 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+* bf16 rounding: torch's own fp32 -> bf16 conversion (round to nearest even).
+* Compression: torch ``avg_pool1d`` (the mean over windows of 32 rows, stride 16 is a
+  special case of it) and a closed form for run-constant keys.
+* Attention: selecting every visible block is dense causal attention, which torch's
+  ``scaled_dot_product_attention`` computes (fp64); any block subset equals SDPA with
+  the matching boolean mask.
+* Selection: hand-derived closed-form cases (tests/golden/select_closed_form.json) and
+  invariants that hold for any input (forced blocks, counts, group sharing, decode =
+  last prefill row, identical heads, planted needle).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from trainable_block_sparse_compress_b200.synthetic import as_u16
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(t):
+    return t.to(torch.bfloat16)
+
+
+def f64(u16):
+    """uint16 bf16 patterns -> float64 torch tensor."""
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).view(torch.bfloat16).double()
+
+
+def rand_inputs(B, L, Hq, Hkv, d=128, seed=0, lq=None, offset=0.5):
+    g = torch.Generator().manual_seed(seed)
+    lq = L if lq is None else lq
+    q = bf16(torch.randn((B, lq, Hq, d), generator=g))
+    nb = (L + 63) // 64
+    off = torch.randn((B, Hkv, nb, d), generator=g) * offset
+    k = bf16(torch.randn((B, Hkv, L, d), generator=g) + off.repeat_interleave(64, 2)[:, :, :L])
+    v = bf16(torch.randn((B, Hkv, L, d), generator=g))
+    return q, k, v
+
+
+# ------------------------------------------------------------------ bf16 rounding
+
+def test_bf16_rounding_matches_torch():
+    g = torch.Generator().manual_seed(1)
+    x = torch.cat([
+        torch.randn(20000, generator=g, dtype=torch.float32) * 10,
+        torch.randn(2000, generator=g, dtype=torch.float32) * 1e-39,  # subnormals
+        torch.tensor([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 3.4e38, -3.4e38, 0.0, -0.0]),
+    ])
+    want = x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.bf16_round(x.double().numpy())
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- compression
+
+P1 = oracle.Params(batch=2, num_q_heads=4, num_kv_heads=2, topk=6)
+
+
+def test_compress_exact_means_match_avg_pool():
+    # integer keys in [-4, 4]: every window mean is a multiple of 1/32 with |mean| <= 4,
+    # which bf16 holds exactly, so the rounded mean must equal avg_pool1d exactly.
+    g = torch.Generator().manual_seed(2)
+    B, H, L, d = 2, 2, 301, 128
+    k = torch.randint(-4, 5, (B, H, L, d), generator=g).to(torch.bfloat16)
+    kc = oracle.compress(P1, as_u16(k))
+    ref = F.avg_pool1d(k.double().permute(0, 1, 3, 2).reshape(-1, 1, L), 32, 16)
+    ref = ref.reshape(B, H, d, -1).permute(0, 1, 3, 2)
+    assert kc.shape == (B, H, (L - 32) // 16 + 1, d)
+    assert torch.equal(f64(kc), ref)
+
+
+def test_compress_random_within_one_ulp_of_avg_pool():
+    k = bf16(torch.randn((1, 2, 1000, 128), generator=torch.Generator().manual_seed(3)))
+    kc = oracle.compress(oracle.Params(batch=1, num_q_heads=2, num_kv_heads=2), as_u16(k))
+    ref = F.avg_pool1d(k.double().permute(0, 1, 3, 2).reshape(-1, 1, 1000), 32, 16)
+    ref = ref.reshape(1, 2, 128, -1).permute(0, 1, 3, 2)
+    # the oracle rounds the exact mean once; compare with the exact mean: error <= half ulp
+    err = (f64(kc) - ref).abs()
+    ulp = torch.tensor(2.0).pow(torch.floor(torch.log2(ref.abs().clamp_min(1e-30))) - 7)
+    assert bool((err <= ulp / 2 + 1e-300).all())
+
+
+def test_compress_closed_form_run_constant_keys():
+    # rows [16r, 16r+16) hold the constant c_r, so kernel i = (c_i + c_{i+1}) / 2 exactly
+    B, H, L, d = 1, 1, 16 * 12, 128
+    c = np.array([1, -3, 2.5, 0, 7, -1.25, 6, 6, -8, 0.5, 3, -2], dtype=np.float64)
+    k = torch.from_numpy(np.repeat(c, 16)).view(1, 1, L, 1).expand(B, H, L, d).to(torch.bfloat16)
+    kc = f64(oracle.compress(oracle.Params(1, 1, 1), as_u16(k.contiguous())))
+    want = (c[:-1] + c[1:]) / 2
+    assert kc.shape[2] == 11
+    for i in range(11):
+        assert torch.all(kc[0, 0, i] == want[i]), i
+
+
+def test_compress_respects_per_sequence_lengths():
+    B, H, L, d = 3, 1, 200, 128
+    k = bf16(torch.randn((B, H, L, d), generator=torch.Generator().manual_seed(4)))
+    lens = np.array([200, 31, 64], dtype=np.int32)
+    kc = oracle.compress(oracle.Params(B, 1, 1), as_u16(k), lens=lens)
+    full = oracle.compress(oracle.Params(B, 1, 1), as_u16(k))
+    assert np.array_equal(kc[0], full[0])
+    assert np.all(kc[1] == 0)  # 31 tokens: no complete kernel
+    assert np.array_equal(kc[2, :, :3], full[2, :, :3]) and np.all(kc[2, :, 3:] == 0)
+
+
+# ------------------------------------------------------------------ attention
+
+def sdpa(q, k, v, mask, scale):
+    """q [Hq, d]; k, v [Hkv, n, d]; mask [n] bool -> o [Hq, d], lse [Hq] (float64)."""
+    Hq, Hkv = q.shape[0], k.shape[0]
+    G = Hq // Hkv
+    kk = k.repeat_interleave(G, 0)
+    vv = v.repeat_interleave(G, 0)
+    o = F.scaled_dot_product_attention(q[:, None, :], kk, vv, attn_mask=mask[None, None, :], scale=scale)
+    logits = (q[:, None, :] * kk).sum(-1) * scale
+    lse = torch.logsumexp(logits.masked_fill(~mask[None, :], -math.inf), -1)
+    return o[:, 0, :], lse
+
+
+def test_attn_all_blocks_is_dense_causal_attention():
+    B, L, Hq, Hkv = 1, 300, 4, 2
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=5)
+    p = oracle.Params(B, Hq, Hkv, topk=8)  # nblk = 5 <= topk
+    idx = np.full((B, Hkv, L, 8), -1, np.int32)
+    for t in range(L):
+        idx[:, :, t, : t // 64 + 1] = np.arange(t // 64 + 1)
+    o, lse = oracle.attn(p, as_u16(q), as_u16(k), as_u16(v), idx)
+    G = Hq // Hkv
+    qq = q.double().permute(0, 2, 1, 3)  # [B, Hq, L, d]
+    kk = k.double().repeat_interleave(G, 1)
+    vv = v.double().repeat_interleave(G, 1)
+    ref = F.scaled_dot_product_attention(qq, kk, vv, is_causal=True, scale=1 / math.sqrt(128))
+    assert np.allclose(o, ref.permute(0, 2, 1, 3).numpy(), atol=1e-12, rtol=1e-10)
+    logits = qq @ kk.transpose(-1, -2) / math.sqrt(128)
+    causal = torch.ones(L, L, dtype=torch.bool).tril()
+    ref_lse = torch.logsumexp(logits.masked_fill(~causal, -math.inf), -1)
+    assert np.allclose(lse, ref_lse.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [6, 7])
+def test_attn_block_subset_equals_masked_sdpa(seed):
+    B, L, Hq, Hkv, topk = 2, 640, 6, 2, 5
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=seed)
+    rng = np.random.default_rng(seed)
+    rows = np.array([0, 63, 64, 100, 200, 350, 511, 575, 639], dtype=np.int64)
+    idx = np.full((B, Hkv, len(rows), topk), -1, np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for r, t in enumerate(rows):
+                cur = t // 64
+                sel = rng.choice(cur + 1, size=min(topk, cur + 1), replace=False)
+                idx[b, g, r, : len(sel)] = np.sort(sel)
+    p = oracle.Params(B, Hq, Hkv, topk=topk)
+    o, lse = oracle.attn(p, as_u16(q), as_u16(k), as_u16(v), idx, rows=rows)
+    G = Hq // Hkv
+    for b in range(B):
+        for r, t in enumerate(rows):
+            for h in range(Hq):
+                g = h // G
+                sel = set(int(j) for j in idx[b, g, r] if j >= 0)
+                keys = torch.arange(L)
+                mask = torch.tensor([(int(u) // 64 in sel) for u in keys]) & (keys <= t)
+                ro, rl = sdpa(q[b, t, h:h + 1].double(), k[b, g:g + 1].double(), v[b, g:g + 1].double(),
+                              mask, 1 / math.sqrt(128))
+                assert np.allclose(o[b, r, h], ro[0].numpy(), atol=1e-12), (b, t, h)
+                assert abs(lse[b, h, r] - rl[0].item()) < 1e-12
+
+
+def test_attn_decode_positions_follow_lengths():
+    # a decode query sits at lens[b]-1; with every block selected it is plain attention
+    # over the first lens[b] keys
+    B, Lmax, Hq, Hkv = 3, 400, 4, 1
+    g = torch.Generator().manual_seed(8)
+    q = bf16(torch.randn((B, 1, Hq, 128), generator=g))
+    k = bf16(torch.randn((B, Hkv, Lmax, 128), generator=g))
+    v = bf16(torch.randn((B, Hkv, Lmax, 128), generator=g))
+    lens = np.array([400, 65, 1], dtype=np.int32)
+    idx = np.full((B, Hkv, 1, 8), -1, np.int32)
+    for b in range(B):
+        nb = (lens[b] + 63) // 64
+        idx[b, :, 0, :nb] = np.arange(nb)
+    o, lse = oracle.attn(oracle.Params(B, Hq, Hkv, topk=8), as_u16(q), as_u16(k), as_u16(v), idx, lens=lens)
+    for b in range(B):
+        n = int(lens[b])
+        mask = torch.zeros(Lmax, dtype=torch.bool)
+        mask[:n] = True
+        ro, rl = sdpa(q[b, 0].double(), k[b].double(), v[b].double(), mask, 1 / math.sqrt(128))
+        assert np.allclose(o[b, 0], ro.numpy(), atol=1e-12)
+        assert np.allclose(lse[b, :, 0], rl.numpy(), atol=1e-12)
+
+
+def test_attn_rejects_future_blocks():
+    q, k, v = rand_inputs(1, 128, 1, 1, seed=9)
+    idx = np.array([[[[0, 1]]]], np.int32)  # row 10 lies in block 0: block 1 is in its future
+    with pytest.raises(ValueError):
+        oracle.attn(oracle.Params(1, 1, 1, topk=2), as_u16(q), as_u16(k), as_u16(v), idx, rows=[10])
+
+
+# ------------------------------------------------------------------ selection
+
+def golden_inputs(case):
+    L, Hq = case["seq_len"], case["num_q_heads"]
+    k = torch.zeros((1, 1, L, 128))
+    for comp, key in ((0, "u"), (1, "w")):
+        for j, val in case[key].items():
+            k[0, 0, int(j) * 64:(int(j) + 1) * 64, comp] = val
+    q = torch.zeros((1, L, Hq, 128))
+    if not case.get("zero_query"):
+        for h in range(Hq):
+            q[0, :, h, h] = 8.0
+    return bf16(q), bf16(k)
+
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "select_closed_form.json")))["cases"],
+                         ids=lambda c: c["name"])
+def test_select_closed_form_cases(case):
+    q, k = golden_inputs(case)
+    p = oracle.Params(1, case["num_q_heads"], case["num_kv_heads"], topk=case["topk"],
+                      n_init=case["n_init"], n_local=case["n_local"], softmax_scale=0.125)
+    kc = oracle.compress(p, as_u16(k))
+    idx = oracle.select(p, as_u16(q), kc, rows=[case["query_pos"]])
+    assert idx[0, 0, 0].tolist() == case["expected"]
+
+
+def check_selection_invariants(idx, rows, p, n):
+    for t_i, t in enumerate(rows):
+        cur = t // p.block_size
+        row = idx[..., t_i, :]
+        for sel in row.reshape(-1, p.topk):
+            valid = sel[sel >= 0]
+            assert np.all(sel[len(valid):] == -1), "padding must trail"
+            assert np.all(np.diff(valid) > 0), "ascending, no duplicates"
+            assert valid.max() <= cur
+            forced = set(range(min(p.n_init, cur + 1))) | set(range(max(cur - p.n_local + 1, 0), cur + 1))
+            assert forced <= set(valid.tolist())
+            expect = min(p.topk, cur + 1) if t >= 31 else len(forced)
+            assert len(valid) == expect
+
+
+def test_select_invariants_random():
+    B, L, Hq, Hkv = 2, 1000, 8, 2
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=10)
+    p = oracle.Params(B, Hq, Hkv, topk=6)
+    kc = oracle.compress(p, as_u16(k))
+    rows = np.arange(0, L, 7)
+    idx, scores = oracle.select(p, as_u16(q), kc, rows=rows, want_scores=True)
+    check_selection_invariants(idx, rows, p, L)
+    # taken blocks score at least as high as any eligible block left out
+    for b in range(B):
+        for g in range(Hkv):
+            for r, t in enumerate(rows):
+                cur = t // 64
+                sel = set(idx[b, g, r][idx[b, g, r] >= 0].tolist())
+                forced = {0, cur, cur - 1}
+                free = [j for j in sel if j not in forced]
+                rest = [scores[b, g, r, j] for j in range(cur + 1) if j not in sel and scores[b, g, r, j] >= 0]
+                if free and rest:
+                    assert min(scores[b, g, r, j] for j in free) >= max(rest)
+
+
+def test_select_short_rows_keep_only_forced_blocks():
+    q, k, v = rand_inputs(1, 96, 2, 1, seed=11)
+    p = oracle.Params(1, 2, 1, topk=4)
+    kc = oracle.compress(p, as_u16(k))
+    idx = oracle.select(p, as_u16(q), kc, rows=[0, 30, 31, 64, 95])
+    assert idx[0, 0, 0].tolist() == [0, -1, -1, -1]
+    assert idx[0, 0, 1].tolist() == [0, -1, -1, -1]
+    assert idx[0, 0, 2].tolist() == [0, -1, -1, -1]
+    assert idx[0, 0, 3].tolist() == [0, 1, -1, -1]
+
+
+def test_select_identical_heads_scale_scores():
+    B, L = 1, 700
+    q, k, v = rand_inputs(B, L, 1, 1, seed=12)
+    p1 = oracle.Params(B, 1, 1, topk=5)
+    p4 = oracle.Params(B, 4, 1, topk=5)
+    kc = oracle.compress(p1, as_u16(k))
+    rows = np.arange(100, L, 37)
+    i1, s1 = oracle.select(p1, as_u16(q), kc, rows=rows, want_scores=True)
+    i4, s4 = oracle.select(p4, as_u16(q.repeat(1, 1, 4, 1)), kc, rows=rows, want_scores=True)
+    assert np.array_equal(i1, i4)
+    el = s1 >= 0
+    assert np.allclose(s4[el], 4 * s1[el], rtol=1e-13)
+
+
+def test_select_gqa_head_to_group_map():
+    # heads 0,1 -> kv-head 0; heads 2,3 -> kv-head 1 (contiguous groups)
+    L = 600
+    qa, ka, _ = rand_inputs(1, L, 2, 1, seed=13)
+    qb, kb, _ = rand_inputs(1, L, 2, 1, seed=14)
+    p2 = oracle.Params(1, 2, 1, topk=5)
+    p4 = oracle.Params(1, 4, 2, topk=5)
+    rows = np.arange(200, L, 50)
+    ia = oracle.select(p2, as_u16(qa), oracle.compress(p2, as_u16(ka)), rows=rows)
+    ib = oracle.select(p2, as_u16(qb), oracle.compress(p2, as_u16(kb)), rows=rows)
+    q = torch.cat([qa, qb], dim=2)
+    k = torch.cat([ka, kb], dim=1)
+    i4 = oracle.select(p4, as_u16(q), oracle.compress(p4, as_u16(k)), rows=rows)
+    assert np.array_equal(i4[:, 0], ia[:, 0]) and np.array_equal(i4[:, 1], ib[:, 0])
+    assert not np.array_equal(ia, ib)
+
+
+def test_select_decode_equals_last_prefill_row():
+    B, L, Hq, Hkv = 2, 900, 4, 2
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=15)
+    p = oracle.Params(B, Hq, Hkv, topk=6)
+    kc = oracle.compress(p, as_u16(k))
+    lens = np.array([900, 517], dtype=np.int32)
+    qd = torch.stack([q[0, 899], q[1, 516]])[:, None]  # [B, 1, Hq, d]
+    kcd = oracle.compress(p, as_u16(k), lens=lens)
+    idx_d = oracle.select(p, as_u16(qd), kcd, lens=lens, Lmax=L)
+    idx_p = oracle.select(p, as_u16(q), kc, rows=[899, 516])
+    assert np.array_equal(idx_d[0, :, 0], idx_p[0, :, 0])
+    assert np.array_equal(idx_d[1, :, 0], idx_p[1, :, 1])
+
+
+def test_select_planted_needle_is_found():
+    # make one far block's keys point along the group's mean query: it must be selected
+    B, L, Hq, Hkv = 1, 2048, 8, 1
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=16)
+    t, needle = 2000, 11
+    qbar = q[0, t].float().mean(0)
+    k = k.clone()
+    k[0, 0, needle * 64:(needle + 1) * 64] = bf16(qbar / qbar.norm() * 6.0)
+    p = oracle.Params(B, Hq, Hkv, topk=8)
+    idx = oracle.select(p, as_u16(q), oracle.compress(p, as_u16(k)), rows=[t])
+    assert needle in idx[0, 0, 0].tolist()
