@@ -1,0 +1,188 @@
+/*
+ * infllmv2.h -- C ABI of the B200 (sm_100a) InfLLM v2 block-sparse attention library.
+ *
+ * InfLLM v2 splits the KV cache into fixed-size blocks, represents every block by
+ * "semantic kernels" (compressed keys), lets every query token pick its most relevant
+ * blocks (one set shared by all query heads of a GQA group) and runs exact attention
+ * over the picked blocks only.  Sources:
+ *   "MiniCPM4：端设备上的超高效大型语言模型" (MiniCPM4 summary page), s2.1.1 (block units,
+ *   per-token top blocks), s2.1.2 (relevance via semantic kernels, group-shared
+ *   selection), s2.1.3 (attention only with the most relevant blocks);
+ *   "OpenBMB publishes Minicpm4 ..." news page, "Technical innovations in MinicPM4"
+ *   (semantic kernels, dynamic block selection for prefill and decode).
+ * The block/kernel sizes, the pooling rules and the forced blocks come from the
+ * workload definition (block 64, kernel 32 stride 16, mean-pooled kernels,
+ * kernel-to-block max-pool, group-sum, top-k including 1 initial + 2 local blocks).
+ *
+ * Conventions for every entry point
+ *  - Tensors are device pointers, row-major with the innermost index last, and must
+ *    be 16-byte aligned.  bf16 means IEEE bfloat16 bit patterns (uint16_t storage).
+ *  - The caller allocates and owns every buffer.  The library allocates nothing,
+ *    keeps no per-call state, and may be called concurrently on distinct streams.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Host-side argument checks run before anything is launched: on a
+ *    negative status nothing was launched and no output was touched.
+ *  - A kernel that waits on the GPU never waits without a bound: if an internal wait
+ *    exceeds its limit the kernel stops early and sets a device error word, which
+ *    infllmv2_device_error() reads (outputs of that call are then undefined).
+ *  - Query positions: prefill queries are tokens 0..L-1 of a fresh sequence; a decode
+ *    query is the last token of its sequence, at position lens[b]-1, and its own key
+ *    and value are already in the cache.
+ *  - GQA: q-head h uses kv-head h / (num_q_heads / num_kv_heads).
+ */
+#ifndef INFLLMV2_H_
+#define INFLLMV2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define INFLLMV2_API __attribute__((visibility("default")))
+#else
+#define INFLLMV2_API
+#endif
+
+/* Same type as cudaStream_t, without requiring the CUDA headers. */
+typedef struct CUstream_st* infllmv2_stream_t;
+
+/* Status codes (return value of every entry point). */
+enum {
+  INFLLMV2_OK = 0,
+  INFLLMV2_ERR_INVALID_ARG = -1,   /* null / misaligned pointer, bad size or count */
+  INFLLMV2_ERR_UNSUPPORTED = -2,   /* valid but not implemented (e.g. head_dim != 128) */
+  INFLLMV2_ERR_WORKSPACE = -3,     /* workspace missing or smaller than required */
+  INFLLMV2_ERR_CUDA = -4           /* a CUDA runtime call or kernel launch failed */
+};
+
+/* Device error word bits (infllmv2_device_error). */
+enum {
+  INFLLMV2_DEVERR_WAIT_TIMEOUT = 1 /* an internal wait ran out of its time limit */
+};
+
+enum { INFLLMV2_MODE_PREFILL = 0, INFLLMV2_MODE_DECODE = 1 };
+
+/* Operations for infllmv2_workspace_size. */
+enum {
+  INFLLMV2_OP_COMPRESS = 0,
+  INFLLMV2_OP_SELECT_PREFILL = 1,
+  INFLLMV2_OP_SELECT_DECODE = 2,
+  INFLLMV2_OP_ATTN_PREFILL = 3,
+  INFLLMV2_OP_ATTN_DECODE = 4
+};
+
+/* Problem description shared by all calls.
+ *   batch          B >= 1
+ *   num_q_heads    Hq, a multiple of num_kv_heads; Hq / Hkv must be 1, 2, 4, 8 or 16
+ *   num_kv_heads   Hkv >= 1
+ *   head_dim       d; only 128 is implemented
+ *   block_size     KV block length in tokens; only 64 is implemented
+ *   kernel_size    semantic-kernel length; only 32 is implemented
+ *   kernel_stride  distance between kernel starts; only 16 is implemented
+ *   topk           blocks per (query token, kv-head), forced ones included; 1..256
+ *   n_init         initial blocks always selected (blocks 0..n_init-1), >= 0
+ *   n_local        local blocks always selected (the query's block and the
+ *                  n_local-1 blocks before it), >= 0; n_init + n_local <= topk
+ *   softmax_scale  scale of q.k in scoring and attention; <= 0 means 1/sqrt(d)      */
+typedef struct {
+  int32_t batch, num_q_heads, num_kv_heads, head_dim;
+  int32_t block_size, kernel_size, kernel_stride;
+  int32_t topk, n_init, n_local;
+  float softmax_scale;
+} infllmv2_params;
+
+/* Largest sequence length (prefill L or decode Lmax) the kernels accept. */
+#define INFLLMV2_MAX_SEQ_LEN 262144
+
+/* Number of semantic kernels in n tokens: (n - kernel_size) / kernel_stride + 1 when
+ * n >= kernel_size, else 0. */
+INFLLMV2_API int64_t infllmv2_num_kernels(const infllmv2_params* p, int64_t n);
+
+/* Key compression into semantic kernels ([S] s2.1.2; "semantic kernels" of the news
+ * page).  Kernel i of (b, g) is the mean of key rows [16 i, 16 i + 32), computed exactly
+ * (fp64 sums) and rounded once to bf16 (nearest even).
+ *   k     bf16 [B, Hkv, Lmax, d]   (input)
+ *   lens  int32 [B] device, or NULL: sequence b holds lens[b] <= Lmax tokens; with
+ *         NULL every sequence holds Lmax tokens.  Kernels past NK(lens[b]) are not
+ *         written.
+ *   kc    bf16 [B, Hkv, NK(Lmax), d]   (output; may be NULL when NK(Lmax) == 0)
+ * Returns INVALID_ARG for null/misaligned pointers or Lmax outside
+ * [1, INFLLMV2_MAX_SEQ_LEN]. */
+INFLLMV2_API int infllmv2_compress_keys(const infllmv2_params* p, const void* k, const int32_t* lens,
+                           int32_t Lmax, void* kc, infllmv2_stream_t stream);
+
+/* Group-shared top-k block selection ([S] s2.1.1, s2.1.2).  For every (b, kv-head g,
+ * query token at position t):
+ *   x_h(i) = scale * q_h . Kc_i  for the group's heads h and the kernels i whose last
+ *            token is <= t;
+ *   lse_h  = log sum_i exp(x_h(i));
+ *   m_h(j) = max of x_h(i) over the visible kernels overlapping block j (kernels
+ *            4j-1 .. 4j+3);
+ *   S(j)   = sum over the group's heads of exp(m_h(j) - lse_h).
+ * Forced blocks (0..n_init-1 and cur-n_local+1..cur, cur = t / 64) are always taken;
+ * the other topk - |forced| slots go to the eligible blocks with the highest S, lower
+ * block index first on equal S.  Each row of block_idx is written ascending and
+ * padded with -1.
+ *   mode       INFLLMV2_MODE_PREFILL: q bf16 [B, L, Hq, d], lens must be NULL,
+ *              L_or_Lmax = L, kc from infllmv2_compress_keys over L tokens,
+ *              block_idx int32 [B, Hkv, L, topk].
+ *              INFLLMV2_MODE_DECODE: q bf16 [B, Hq, d], lens int32 [B] device
+ *              (1 <= lens[b] <= Lmax), L_or_Lmax = Lmax, kc [B, Hkv, NK(Lmax), d],
+ *              block_idx int32 [B, Hkv, 1, topk].
+ *   ws, ws_bytes  device workspace of at least infllmv2_workspace_size(p,
+ *              INFLLMV2_OP_SELECT_PREFILL or _DECODE, L_or_Lmax) bytes (may be NULL
+ *              when that size is 0).  Contents on entry do not matter. */
+INFLLMV2_API int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, const void* kc,
+                           const int32_t* lens, int32_t L_or_Lmax, int32_t* block_idx,
+                           void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+/* Sparse attention for prefill ([S] s2.1.3).  For every (b, token t, q-head h):
+ *   O = softmax(scale * q . K_J^T) V_J over the keys J of the selected blocks of
+ *   (b, h / G, t), cut at position t (causal inside the query's own block).
+ *   q          bf16 [B, L, Hq, d];  k, v  bf16 [B, Hkv, L, d]
+ *   block_idx  int32 [B, Hkv, L, topk], ascending or not, unique entries, -1 = unused;
+ *              entries outside [0, t / 64] are skipped.
+ *   o          bf16 [B, L, Hq, d] (output)
+ *   lse        fp32 [B, Hq, L] natural-log normaliser (output), or NULL. */
+INFLLMV2_API int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const void* k,
+                                 const void* v, const int32_t* block_idx, int32_t L, void* o,
+                                 float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+/* Sparse attention for one decode token per sequence ([S] s2.1.3, prefill *and*
+ * decode per s2.1 of the same page).  Split over the selected blocks across CTAs,
+ * then merged with the partial log-sum-exps.
+ *   q          bf16 [B, Hq, d];  k_cache, v_cache bf16 [B, Hkv, Lmax, d]
+ *   lens       int32 [B] device, 1 <= lens[b] <= Lmax; the query sits at lens[b]-1
+ *   block_idx  int32 [B, Hkv, 1, topk] (as for prefill)
+ *   o          bf16 [B, Hq, d];  lse fp32 [B, Hq] or NULL
+ *   ws         at least infllmv2_workspace_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax) bytes */
+INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* lens, int32_t Lmax,
+                                const int32_t* block_idx, void* o, float* lse, void* ws,
+                                size_t ws_bytes, infllmv2_stream_t stream);
+
+/* Workspace bytes needed by `op` (INFLLMV2_OP_*) for sequence length L_or_Lmax, or 0
+ * when the op needs none; (size_t)-1 for invalid parameters. */
+INFLLMV2_API size_t infllmv2_workspace_size(const infllmv2_params* p, int op, int32_t L_or_Lmax);
+
+/* Validates a parameter block; returns INFLLMV2_OK or the status a call would get. */
+INFLLMV2_API int infllmv2_check_params(const infllmv2_params* p);
+
+/* Static text for a status code. */
+INFLLMV2_API const char* infllmv2_status_string(int status);
+
+/* Reads (and, if clear != 0, resets) the device error word of the current device.
+ * Synchronises the device.  Returns the INFLLMV2_DEVERR_* bits, or a negative status. */
+INFLLMV2_API int infllmv2_device_error(int clear);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+INFLLMV2_API int infllmv2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFLLMV2_H_ */

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments before touching the GPU (no kernel is launched here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from trainable_block_sparse_compress_b200 import _lib, build
+from trainable_block_sparse_compress_b200.ops import Params
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "infllmv2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"INFLLMV2_API\s+[\w\s\*]+?\b(infllmv2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_symbols()
+    for n in ("infllmv2_compress_keys", "infllmv2_select_blocks", "infllmv2_sparse_attn_prefill",
+              "infllmv2_sparse_attn_decode", "infllmv2_workspace_size", "infllmv2_status_string"):
+        assert n in names
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT\s+(\w+)", out.stdout))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing but the API leaks out of the library
+    assert {s for s in exported if s.startswith("infllmv2_")} == set(declared_symbols())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.infllmv2_version() >= 100
+    assert lib.infllmv2_status_string(0) == b"ok"
+    assert b"workspace" in lib.infllmv2_status_string(-3)
+    assert lib.infllmv2_status_string(12345) == b"unknown status"
+
+
+def cp(**kw):
+    base = dict(batch=1, num_q_heads=32, num_kv_heads=2, topk=96)
+    base.update(kw)
+    return ctypes.byref(Params(**base).c())
+
+
+def test_param_validation(lib):
+    f = lib.infllmv2_check_params
+    assert f(cp()) == _lib.OK
+    assert f(None) == _lib.ERR_INVALID_ARG
+    assert f(cp(num_q_heads=31)) == _lib.ERR_INVALID_ARG  # not a multiple of Hkv
+    assert f(cp(topk=2)) == _lib.ERR_INVALID_ARG  # n_init + n_local > topk
+    assert f(cp(n_init=-1)) == _lib.ERR_INVALID_ARG
+    assert f(cp(batch=0)) == _lib.ERR_INVALID_ARG
+    assert f(cp(head_dim=64)) == _lib.ERR_UNSUPPORTED
+    assert f(cp(block_size=128)) == _lib.ERR_UNSUPPORTED
+    assert f(cp(kernel_size=64)) == _lib.ERR_UNSUPPORTED
+    assert f(cp(num_q_heads=64, num_kv_heads=2)) == _lib.ERR_UNSUPPORTED  # G = 32
+    assert f(cp(num_q_heads=6, num_kv_heads=2)) == _lib.ERR_UNSUPPORTED  # G = 3
+    assert f(cp(topk=257)) == _lib.ERR_UNSUPPORTED
+    assert f(cp(num_q_heads=8, num_kv_heads=1, topk=16)) == _lib.OK
+
+
+def test_num_kernels(lib):
+    for n, want in ((0, 0), (31, 0), (32, 1), (47, 1), (48, 2), (2048, 127), (131072, 8191)):
+        assert lib.infllmv2_num_kernels(cp(), n) == want
+
+
+def test_workspace_sizes(lib):
+    ws = lib.infllmv2_workspace_size
+    assert ws(cp(), _lib.OP_COMPRESS, 4096) == 0
+    assert ws(cp(), _lib.OP_SELECT_PREFILL, 4096) == 0
+    assert ws(cp(), _lib.OP_ATTN_PREFILL, 4096) == 0
+    assert ws(cp(batch=32), _lib.OP_SELECT_DECODE, 131072) > 0
+    assert ws(cp(batch=32), _lib.OP_ATTN_DECODE, 131072) > 0
+    assert ws(cp(), 99, 4096) == ctypes.c_size_t(-1).value
+    assert ws(cp(), _lib.OP_COMPRESS, 0) == ctypes.c_size_t(-1).value
+    assert ws(cp(), _lib.OP_COMPRESS, _lib.MAX_SEQ_LEN + 1) == ctypes.c_size_t(-1).value
+
+
+def test_calls_reject_bad_arguments_before_launch(lib):
+    # every failure below is detected on the host; nothing reaches the GPU
+    good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    assert lib.infllmv2_compress_keys(cp(), None, None, 128, good, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_compress_keys(cp(), good, None, 128, None, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_compress_keys(cp(), good + 2, None, 128, good, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_compress_keys(cp(), good, None, 0, good, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_compress_keys(cp(head_dim=64), good, None, 128, good, None) == _lib.ERR_UNSUPPORTED
+    assert lib.infllmv2_select_blocks(cp(), 0, None, good, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_select_blocks(cp(), 0, good, good, good, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_select_blocks(cp(), 7, good, good, None, 16, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_sparse_attn_prefill(cp(), good, good, None, good, 128, good, None, None, 0,
+                                            None) == _lib.ERR_INVALID_ARG
+    assert lib.infllmv2_sparse_attn_prefill(cp(), good, good, good, good, 128, good, good + 1, None, 0,
+                                            None) == _lib.ERR_INVALID_ARG
+    # decode needs a workspace of the advertised size
+    need = lib.infllmv2_workspace_size(cp(batch=4), _lib.OP_ATTN_DECODE, 1024)
+    assert lib.infllmv2_sparse_attn_decode(cp(batch=4), good, good, good, good, 1024, good, good, None, None, 0,
+                                           None) == _lib.ERR_WORKSPACE
+    assert lib.infllmv2_sparse_attn_decode(cp(batch=4), good, good, good, good, 1024, good, good, None, good,
+                                           need - 1, None) == _lib.ERR_WORKSPACE
+    need_s = lib.infllmv2_workspace_size(cp(batch=4), _lib.OP_SELECT_DECODE, 1024)
+    assert lib.infllmv2_select_blocks(cp(batch=4), 1, good, good, good, 1024, good, good, need_s - 16,
+                                      None) == _lib.ERR_WORKSPACE

@@ -1,0 +1,288 @@
+"""Parity of the CUDA library (called through its C ABI) with the CPU oracle.
+
+Each step is first checked in isolation on inputs the oracle produced (the GPU selection
+is fed the oracle's kernels, the GPU attention the oracle's block lists), then the whole
+path runs on the five benchmark workloads and is compared on sampled rows.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import (bf16_to_f64, bf16_ulp_diff, compare_attention, compare_selection, u16)
+from trainable_block_sparse_compress_b200 import build, ops
+from trainable_block_sparse_compress_b200.synthetic import WORKLOADS, Workload, as_u16, make_inputs
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_library():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    assert ops.device_error(clear=True) == 0
+    yield
+    assert ops.device_error(clear=True) == 0, "a kernel hit its wait time limit"
+
+
+def oparams(p: ops.Params) -> oracle.Params:
+    return oracle.Params(p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.block_size, p.kernel_size,
+                         p.kernel_stride, p.topk, p.n_init, p.n_local, p.softmax_scale)
+
+
+def inputs(B, L, Hq, Hkv, seed, mode="prefill", lens=None):
+    wl = Workload("t", mode, B, L, Hq, Hkv, 16)
+    x = make_inputs(wl, seed)
+    if lens is not None:
+        x.lens = torch.tensor(lens, dtype=torch.int32)
+    return x
+
+
+# ------------------------------------------------------------------ compression
+
+@pytest.mark.parametrize("B,H,L,lens", [(2, 2, 4500, None), (3, 1, 1000, [1000, 31, 517]), (1, 2, 32, None),
+                                        (1, 1, 31, None), (2, 2, 5000, [48, 4999])])
+def test_compress_matches_oracle(B, H, L, lens):
+    x = inputs(B, L, H, H, seed=100 + L, mode="decode" if lens else "prefill", lens=lens)
+    p = ops.Params(B, H, H, topk=16)
+    lens_t = None if lens is None else x.lens.cuda()
+    kc_g = u16(ops.compress_keys(p, x.k.cuda(), lens=lens_t))
+    kc_o = oracle.compress(oparams(p), as_u16(x.k), lens=None if lens is None else np.array(lens, np.int32))
+    nks = [oracle.num_kernels(oparams(p), n) for n in (lens or [L] * B)]
+    # the mean is exact on both sides and rounded once: bit-exact
+    for b in range(B):
+        a, o = kc_g[b, :, :nks[b]], kc_o[b, :, :nks[b]]
+        assert np.array_equal(a, o), f"{int((a != o).sum())} kernel values differ, max {bf16_ulp_diff(a, o).max()} ulp"
+
+
+def test_compress_closed_form_exact():
+    c = np.array([1, -3, 2.5, 0, 7, -1.25, 6, 6, -8, 0.5, 3, -2] * 30, dtype=np.float32)
+    L = 16 * len(c)
+    k = torch.from_numpy(np.repeat(c, 16)).view(1, 1, L, 1).expand(1, 1, L, 128).contiguous().to(torch.bfloat16)
+    p = ops.Params(1, 1, 1, topk=16)
+    kc = bf16_to_f64(u16(ops.compress_keys(p, k.cuda())))
+    want = (c[:-1].astype(np.float64) + c[1:]) / 2
+    assert np.array_equal(kc[0, 0], np.repeat(want[:, None], 128, 1))
+
+
+# -------------------------------------------------------------------- selection
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "select_closed_form.json")))["cases"],
+                         ids=lambda c: c["name"])
+def test_select_closed_form_cases(case):
+    L, Hq = case["seq_len"], case["num_q_heads"]
+    k = torch.zeros((1, 1, L, 128))
+    for comp, key in ((0, "u"), (1, "w")):
+        for j, val in case[key].items():
+            k[0, 0, int(j) * 64:(int(j) + 1) * 64, comp] = val
+    q = torch.zeros((1, L, Hq, 128))
+    if not case.get("zero_query"):
+        for h in range(Hq):
+            q[0, :, h, h] = 8.0
+    p = ops.Params(1, Hq, 1, topk=case["topk"], n_init=case["n_init"], n_local=case["n_local"],
+                   softmax_scale=0.125)
+    kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda())
+    idx = ops.select_blocks_prefill(p, q.to(torch.bfloat16).cuda(), kc).cpu().numpy()
+    assert idx[0, 0, case["query_pos"]].tolist() == case["expected"]
+
+
+SELECT_CASES = [
+    # B, L, Hq, Hkv, topk, n_init, n_local
+    (1, 4500, 32, 2, 16, 1, 2),   # 5 kernel tiles, ragged tail (4500 % 64 = 20, % 8 = 4)
+    (2, 1000, 8, 1, 6, 1, 2),     # G = 8, two sequences
+    (1, 777, 2, 2, 5, 2, 1),      # G = 1, two initial blocks, one local block
+    (1, 2000, 16, 1, 256, 1, 2),  # topk larger than the number of blocks
+    (1, 20, 16, 1, 4, 1, 2),      # no complete kernel: forced blocks only
+    (1, 1100, 4, 1, 3, 0, 0),     # nothing forced
+]
+
+
+def prefill_rows(L):
+    if L <= 1200:
+        return np.arange(L)
+    return np.unique(np.concatenate([np.arange(200), np.arange(200, L - 200, 13), np.arange(L - 200, L)]))
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,topk,ni,nl", SELECT_CASES)
+def test_select_prefill_matches_oracle(B, L, Hq, Hkv, topk, ni, nl):
+    x = inputs(B, L, Hq, Hkv, seed=200 + L)
+    p = ops.Params(B, Hq, Hkv, topk=topk, n_init=ni, n_local=nl)
+    op = oparams(p)
+    kc_o = oracle.compress(op, as_u16(x.k))
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_prefill(p, x.q.cuda(), kc_t).cpu().numpy()
+    rows = prefill_rows(L)
+    idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
+    compare_selection(idx_g[:, :, rows], idx_o, sc, np.tile(rows, (B, 1)), p)
+
+
+@pytest.mark.parametrize("lens,Lmax,Hq,Hkv,topk", [([3000, 1, 31, 1500, 2049], 3000, 32, 2, 16),
+                                                  ([70, 64, 65, 128], 128, 8, 1, 3),
+                                                  ([9000, 8193], 9000, 4, 4, 100)])
+def test_select_decode_matches_oracle(lens, Lmax, Hq, Hkv, topk):
+    B = len(lens)
+    x = inputs(B, Lmax, Hq, Hkv, seed=300 + Lmax, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_decode(p, x.q.cuda(), kc_t, x.lens.cuda(), Lmax).cpu().numpy()
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    compare_selection(idx_g, idx_o, sc, (lens_np - 1)[:, None], p)
+
+
+# -------------------------------------------------------------------- attention
+
+ATTN_CASES = [(1, 4500, 32, 2, 16), (2, 1000, 8, 1, 6), (1, 777, 2, 2, 5), (1, 700, 16, 1, 16), (1, 64, 16, 1, 4)]
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,topk", ATTN_CASES)
+def test_attn_prefill_matches_oracle(B, L, Hq, Hkv, topk):
+    x = inputs(B, L, Hq, Hkv, seed=400 + L)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    kc_o = oracle.compress(op, as_u16(x.k))
+    idx_all = oracle.select(op, as_u16(x.q), kc_o)  # every row, so the GPU sees the oracle's lists
+    o_g, lse_g = ops.sparse_attn_prefill(p, x.q.cuda(), x.k.cuda(), x.v.cuda(),
+                                         torch.from_numpy(idx_all).cuda())
+    rows = prefill_rows(L)[::3]
+    o_o, lse_o = oracle.attn(op, as_u16(x.q), as_u16(x.k), as_u16(x.v), idx_all[:, :, rows], rows=rows)
+    o_g = o_g.float().cpu().numpy()[:, rows]
+    lse_g = lse_g.cpu().numpy()[:, :, rows]
+    compare_attention(o_g, o_o, lse_g, lse_o)
+
+
+@pytest.mark.parametrize("lens,Lmax,Hq,Hkv,topk", [([3000, 1, 31, 1500, 2049], 3000, 32, 2, 16),
+                                                  ([9000, 8193, 64], 9000, 16, 1, 96)])
+def test_attn_decode_matches_oracle(lens, Lmax, Hq, Hkv, topk):
+    B = len(lens)
+    x = inputs(B, Lmax, Hq, Hkv, seed=500 + Lmax, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    idx_o = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax)
+    o_g, lse_g = ops.sparse_attn_decode(p, x.q.cuda(), x.k.cuda(), x.v.cuda(), x.lens.cuda(),
+                                        torch.from_numpy(idx_o).cuda())
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
+
+
+def test_attn_decode_many_items_per_cta_is_deterministic():
+    # more work items than CTAs, ragged lengths: repeated runs must agree bit for bit
+    # and match the oracle
+    rng = np.random.default_rng(7)
+    B, Lmax, Hq, Hkv, topk = 24, 20000, 32, 2, 96
+    lens = rng.integers(1, Lmax + 1, size=B).tolist()
+    x = inputs(B, Lmax, Hq, Hkv, seed=700, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    idx_o = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax)
+    q, k, v, ln, idx = x.q.cuda(), x.k.cuda(), x.v.cuda(), x.lens.cuda(), torch.from_numpy(idx_o).cuda()
+    o_ref, lse_ref = ops.sparse_attn_decode(p, q, k, v, ln, idx)
+    for _ in range(5):
+        o_g, lse_g = ops.sparse_attn_decode(p, q, k, v, ln, idx)
+        assert torch.equal(o_g, o_ref) and torch.equal(lse_g, lse_ref)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
+    compare_attention(o_ref.float().cpu().numpy(), o_o[:, 0], lse_ref.cpu().numpy(), lse_o[:, :, 0])
+
+
+def test_attn_prefill_is_deterministic():
+    B, L, Hq, Hkv, topk = 1, 6000, 32, 2, 24
+    x = inputs(B, L, Hq, Hkv, seed=701)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    q, k, v = x.q.cuda(), x.k.cuda(), x.v.cuda()
+    kc = ops.compress_keys(p, k)
+    idx = ops.select_blocks_prefill(p, q, kc)
+    o_ref, lse_ref = ops.sparse_attn_prefill(p, q, k, v, idx)
+    idx_ref = idx.clone()
+    for _ in range(3):
+        assert torch.equal(ops.select_blocks_prefill(p, q, kc), idx_ref)
+        o_g, lse_g = ops.sparse_attn_prefill(p, q, k, v, idx)
+        assert torch.equal(o_g, o_ref) and torch.equal(lse_g, lse_ref)
+
+
+def test_attn_decode_ignores_garbage_past_the_length():
+    # cache rows at or past lens[b] hold NaN: they must not reach the output
+    lens, Lmax = [100, 64, 65], 192
+    B, Hq, Hkv = 3, 16, 1
+    x = inputs(B, Lmax, Hq, Hkv, seed=600, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=4)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    idx_o = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax)
+    k, v = x.k.clone(), x.v.clone()
+    for b, n in enumerate(lens):
+        k[b, :, n:] = float("nan")
+        v[b, :, n:] = float("nan")
+    o_g, _ = ops.sparse_attn_decode(p, x.q.cuda(), k.cuda(), v.cuda(), x.lens.cuda(), torch.from_numpy(idx_o).cuda())
+    o_o, _ = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
+    assert torch.isfinite(o_g).all()
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0])
+
+
+# ---------------------------------------------------------- whole path, workloads
+
+def sample_rows(L):
+    if L <= 4096:
+        return np.arange(L)
+    stride = max(1, L // 1024)
+    return np.unique(np.concatenate([np.arange(128), np.arange(128, L - 128, stride), np.arange(L - 128, L)]))
+
+
+@pytest.mark.parametrize("name", ["prefill_2k", "prefill_32k", "prefill_128k"])
+def test_prefill_workload_end_to_end(name):
+    wl = WORKLOADS[name]
+    x = make_inputs(wl, seed=0)
+    p = ops.Params.from_workload(wl)
+    op = oparams(p)
+    q, k, v = x.q.cuda(), x.k.cuda(), x.v.cuda()
+    o_g, lse_g, idx_g, kc_g = ops.prefill(p, q, k, v)
+    torch.cuda.synchronize()
+    kc_o = oracle.compress(op, as_u16(x.k))
+    assert np.array_equal(u16(kc_g), kc_o)
+    rows = sample_rows(wl.seq_len)
+    rows_t = torch.from_numpy(rows).cuda()
+    idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
+    idx_gr = idx_g[:, :, rows_t].cpu().numpy()
+    same, n_tie = compare_selection(idx_gr, idx_o, sc, np.tile(rows, (wl.batch, 1)), p)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q), as_u16(x.k), as_u16(x.v), idx_o, rows=rows)
+    o_gr = o_g[:, rows_t].float().cpu().numpy()  # [B, R, Hq, d]
+    lse_gr = lse_g[:, :, rows_t].cpu().numpy()   # [B, Hq, R]
+    G = p.group
+    row_ok = np.repeat(same, G, axis=1)  # [B, Hq, R]
+    compare_attention(o_gr, o_o, mask=np.transpose(row_ok, (0, 2, 1)))
+    dl = np.abs(lse_gr - lse_o)[row_ok]
+    assert float(dl.max()) <= 1e-3
+
+
+@pytest.mark.parametrize("name", ["decode_32k", "decode_ragged_128k"])
+def test_decode_workload_end_to_end(name):
+    wl = WORKLOADS[name]
+    x = make_inputs(wl, seed=0)
+    p = ops.Params.from_workload(wl)
+    op = oparams(p)
+    lens_np = x.lens.numpy()
+    k, v, lens = x.k.cuda(), x.v.cuda(), x.lens.cuda()
+    kc_g = ops.compress_keys(p, k, lens=lens)
+    o_g, lse_g, idx_g = ops.decode(p, x.q.cuda(), k, v, kc_g, lens, wl.seq_len)
+    torch.cuda.synchronize()
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    kcg = u16(kc_g)
+    for b in range(wl.batch):
+        nk = oracle.num_kernels(op, int(lens_np[b]))
+        assert np.array_equal(kcg[b, :, :nk], kc_o[b, :, :nk]), b
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=wl.seq_len, want_scores=True)
+    same, _ = compare_selection(idx_g.cpu().numpy(), idx_o, sc, (lens_np - 1)[:, None], p)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
+    row_ok = np.repeat(same[:, :, 0], p.group, axis=1)  # [B, Hq]
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], mask=row_ok)
+    assert float(np.abs(lse_g.cpu().numpy() - lse_o[:, :, 0])[row_ok].max()) <= 1e-3

@@ -1,0 +1,380 @@
+// infllmv2.cu -- C ABI of the InfLLM v2 block-sparse attention library (sm_100a).
+//
+// Host side of every entry point declared in include/infllmv2.h: argument checks
+// before any launch, TMA tensor-map encoding (driver entry point fetched through the
+// runtime, so the library needs no -lcuda), workspace carving and kernel launches on
+// the caller's stream.  All device code lives in the included .cuh files.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/infllmv2.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "compress.cuh"
+#include "select_decode.cuh"
+#include "select_prefill.cuh"
+#include "topk.cuh"
+
+using namespace infllmv2;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_params(const infllmv2_params* p) {
+  if (p == nullptr) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->num_kv_heads < 1 || p->num_q_heads < 1 || p->head_dim < 1) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->block_size < 1 || p->kernel_size < 1 || p->kernel_stride < 1) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->topk < 1 || p->n_init < 0 || p->n_local < 0) return INFLLMV2_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->n_init) + p->n_local > p->topk) return INFLLMV2_ERR_INVALID_ARG;
+  if (!(p->softmax_scale <= 0.f || std::isfinite(p->softmax_scale))) return INFLLMV2_ERR_INVALID_ARG;
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (p->head_dim != kHeadDim || p->block_size != kBlock || p->kernel_size != kKernel ||
+      p->kernel_stride != kStride)
+    return INFLLMV2_ERR_UNSUPPORTED;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return INFLLMV2_ERR_UNSUPPORTED;
+  if (p->topk > kMaxTopk) return INFLLMV2_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->batch) * p->num_q_heads > (1LL << 24)) return INFLLMV2_ERR_UNSUPPORTED;
+  return INFLLMV2_OK;
+}
+
+int check_len(int32_t L) { return (L >= 1 && L <= INFLLMV2_MAX_SEQ_LEN) ? INFLLMV2_OK : INFLLMV2_ERR_INVALID_ARG; }
+
+int64_t num_kernels(int64_t n) { return n >= kKernel ? (n - kKernel) / kStride + 1 : 0; }
+int64_t num_blocks(int64_t n) { return (n + kBlock - 1) / kBlock; }
+int round32(int64_t x) { return static_cast<int>((x + 31) / 32 * 32); }
+
+float scale_log2(const infllmv2_params* p) {
+  const float s = p->softmax_scale > 0.f ? p->softmax_scale : 1.f / std::sqrt(static_cast<float>(p->head_dim));
+  return s * 1.4426950408889634f;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D view [rows, 128] of a bf16 tensor, box {64 columns, box_rows}, 128-byte swizzle,
+// zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+  if (!get_encoder()) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+int set_smem(const void* fn, size_t bytes) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+                 cudaSuccess
+             ? INFLLMV2_OK
+             : INFLLMV2_ERR_CUDA;
+}
+
+// Decode attention split: selected blocks per split and number of splits per (b, g).
+void decode_split(const infllmv2_params* p, int* n_splits, int* per_split) {
+  const long long bgs = static_cast<long long>(p->batch) * p->num_kv_heads;
+  const int sms = num_sms();
+  int s = static_cast<int>((4LL * sms + bgs - 1) / bgs);
+  s = std::max(1, std::min(s, (p->topk + 7) / 8));
+  *per_split = (p->topk + s - 1) / s;
+  *n_splits = (p->topk + *per_split - 1) / *per_split;
+}
+
+size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
+  if (check_params(p) != INFLLMV2_OK || check_len(L) != INFLLMV2_OK) return static_cast<size_t>(-1);
+  switch (op) {
+    case INFLLMV2_OP_COMPRESS:
+    case INFLLMV2_OP_SELECT_PREFILL:
+    case INFLLMV2_OP_ATTN_PREFILL:
+      return 0;
+    case INFLLMV2_OP_SELECT_DECODE: {
+      const int nch = static_cast<int>((num_kernels(L) + kDecChunk - 1) / kDecChunk);
+      return sel_decode_ws_bytes(p->batch, p->num_kv_heads, std::max(nch, 1));
+    }
+    case INFLLMV2_OP_ATTN_DECODE: {
+      int ns, per;
+      decode_split(p, &ns, &per);
+      const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * ns * kGroupRows;
+      const size_t a = rows * kHeadDim * sizeof(float);
+      return a + rows * sizeof(float);
+    }
+    default:
+      return static_cast<size_t>(-1);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t infllmv2_num_kernels(const infllmv2_params* p, int64_t n) {
+  if (p == nullptr || p->kernel_size < 1 || p->kernel_stride < 1 || n < p->kernel_size) return 0;
+  return (n - p->kernel_size) / p->kernel_stride + 1;
+}
+
+int infllmv2_check_params(const infllmv2_params* p) { return check_params(p); }
+
+int infllmv2_version(void) { return kVersion; }
+
+const char* infllmv2_status_string(int status) {
+  switch (status) {
+    case INFLLMV2_OK:
+      return "ok";
+    case INFLLMV2_ERR_INVALID_ARG:
+      return "invalid argument";
+    case INFLLMV2_ERR_UNSUPPORTED:
+      return "unsupported configuration";
+    case INFLLMV2_ERR_WORKSPACE:
+      return "workspace missing or too small";
+    case INFLLMV2_ERR_CUDA:
+      return "CUDA error";
+    default:
+      return "unknown status";
+  }
+}
+
+size_t infllmv2_workspace_size(const infllmv2_params* p, int op, int32_t L_or_Lmax) {
+  return ws_size(p, op, L_or_Lmax);
+}
+
+int infllmv2_device_error(int clear) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  if (clear) {
+    unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof z) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  }
+  return static_cast<int>(v);
+}
+
+int infllmv2_compress_keys(const infllmv2_params* p, const void* k, const int32_t* lens, int32_t Lmax, void* kc,
+                           infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(Lmax)) != INFLLMV2_OK) return st;
+  if (k == nullptr || !aligned16(k)) return INFLLMV2_ERR_INVALID_ARG;
+  if (lens != nullptr && (reinterpret_cast<uintptr_t>(lens) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+  const int nk = static_cast<int>(num_kernels(Lmax));
+  if (nk == 0) return INFLLMV2_OK;  // kc has no rows (and may be NULL)
+  if (kc == nullptr || !aligned16(kc)) return INFLLMV2_ERR_INVALID_ARG;
+  const int halfwarps = (nk + kCompressKPH - 1) / kCompressKPH;
+  dim3 grid((halfwarps + 7) / 8, p->num_kv_heads, p->batch);
+  compress_kernel<<<grid, kCompressThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(k), lens, Lmax, nk, p->num_kv_heads, static_cast<__nv_bfloat16*>(kc));
+  return launch_status();
+}
+
+int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, const void* kc,
+                           const int32_t* lens, int32_t L, int32_t* block_idx, void* ws, size_t ws_bytes,
+                           infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(L)) != INFLLMV2_OK) return st;
+  if (q == nullptr || block_idx == nullptr || !aligned16(q) || !aligned16(block_idx)) return INFLLMV2_ERR_INVALID_ARG;
+  const int64_t nk = num_kernels(L);
+  if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
+  if (mode == INFLLMV2_MODE_PREFILL) {
+    if (lens != nullptr) return INFLLMV2_ERR_INVALID_ARG;
+  } else if (mode == INFLLMV2_MODE_DECODE) {
+    if (lens == nullptr || (reinterpret_cast<uintptr_t>(lens) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+    const size_t need = ws_size(p, INFLLMV2_OP_SELECT_DECODE, L);
+    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return INFLLMV2_ERR_WORKSPACE;
+  } else {
+    return INFLLMV2_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int G = p->num_q_heads / p->num_kv_heads;
+  const int nblk_cap = round32(num_blocks(L));
+  CUtensorMap tm_kc;
+  std::memset(&tm_kc, 0, sizeof tm_kc);
+  // a map over a 1-row dummy extent is never dereferenced when there are no kernels
+  if (nk > 0 && !make_map(&tm_kc, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kKcTile))
+    return INFLLMV2_ERR_CUDA;
+
+  if (mode == INFLLMV2_MODE_PREFILL) {
+    if (nk == 0) {
+      // no complete kernel: every row keeps only its forced blocks; reuse the kernel
+      // path with an empty score loop (TA = TB = 0 never touches the map)
+      if (!make_map(&tm_kc, q, kKcTile, kKcTile)) return INFLLMV2_ERR_CUDA;
+    }
+    SelPrefillParams a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.idx = block_idx;
+    a.B = p->batch;
+    a.L = L;
+    a.Hq = p->num_q_heads;
+    a.Hkv = p->num_kv_heads;
+    a.G = G;
+    a.NKmax = static_cast<int>(nk);
+    a.topk = p->topk;
+    a.n_init = p->n_init;
+    a.n_local = p->n_local;
+    a.nblk_cap = nblk_cap;
+    a.scale_log2 = scale_log2(p);
+    a.tiles_per_bg = (L + kSelWarps - 1) / kSelWarps;
+    const size_t smem = sel_prefill_smem_bytes(nblk_cap);
+    if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_kernel), smem)) != INFLLMV2_OK) return st;
+    const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
+    if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+    select_prefill_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(tm_kc, a);
+    return launch_status();
+  }
+  SelDecodeParams a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.lens = lens;
+  a.idx = block_idx;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = G;
+  a.Lmax = L;
+  a.NKmax = static_cast<int>(nk);
+  a.topk = p->topk;
+  a.n_init = p->n_init;
+  a.n_local = p->n_local;
+  a.n_chunks = std::max(1, static_cast<int>((nk + kDecChunk - 1) / kDecChunk));
+  a.scale_log2 = scale_log2(p);
+  const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * a.n_chunks;
+  a.ws_lse = static_cast<float2*>(ws);
+  const size_t lse_bytes = (rows * kGroupRows * sizeof(float2) + 255) & ~static_cast<size_t>(255);
+  a.ws_bm = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + lse_bytes);
+  if (nk > 0) {
+    const size_t smem = sel_decode_score_smem_bytes();
+    if ((st = set_smem(reinterpret_cast<const void*>(select_decode_score_kernel), smem)) != INFLLMV2_OK) return st;
+    dim3 grid(a.n_chunks, p->num_kv_heads, p->batch);
+    select_decode_score_kernel<<<grid, kDecScoreThreads, smem, s>>>(tm_kc, a);
+    if ((st = launch_status()) != INFLLMV2_OK) return st;
+  }
+  const size_t smem2 = static_cast<size_t>(nblk_cap) * 4 + kGroupRows * 4 + 256 * 4;
+  if ((st = set_smem(reinterpret_cast<const void*>(select_decode_topk_kernel), smem2)) != INFLLMV2_OK) return st;
+  select_decode_topk_kernel<<<dim3(p->num_kv_heads, p->batch), kDecTopkThreads, smem2, s>>>(a, nblk_cap);
+  return launch_status();
+}
+
+static int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
+                       uint64_t kv_rows, AttnParams& a, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
+      !make_map(&tv, v, kv_rows, kBlock))
+    return INFLLMV2_ERR_CUDA;
+  const size_t smem = attn_smem_bytes();
+  int st = set_smem(reinterpret_cast<const void*>(attn_kernel), smem);
+  if (st != INFLLMV2_OK) return st;
+  const long long grid = std::min<long long>(a.num_items, num_sms());
+  if (grid <= 0) return INFLLMV2_OK;
+  attn_kernel<<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
+int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const void* k, const void* v,
+                                 const int32_t* block_idx, int32_t L, void* o, float* lse, void* ws,
+                                 size_t ws_bytes, infllmv2_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(L)) != INFLLMV2_OK) return st;
+  if (!q || !k || !v || !block_idx || !o) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_idx) || !aligned16(o))
+    return INFLLMV2_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+  AttnParams a;
+  a.idx = block_idx;
+  a.lens = nullptr;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = p->num_q_heads / p->num_kv_heads;
+  a.Lq = L;
+  a.Lmax = L;
+  a.topk = p->topk;
+  a.n_splits = 1;
+  a.blocks_per_split = p->topk;
+  a.scale_log2 = scale_log2(p);
+  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * L;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.part_o = nullptr;
+  a.part_lse = nullptr;
+  return launch_attn(p, q, static_cast<uint64_t>(p->batch) * L * p->num_q_heads, k, v,
+                     static_cast<uint64_t>(p->batch) * p->num_kv_heads * L, a,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* lens, int32_t Lmax, const int32_t* block_idx, void* o, float* lse,
+                                void* ws, size_t ws_bytes, infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(Lmax)) != INFLLMV2_OK) return st;
+  if (!q || !k_cache || !v_cache || !lens || !block_idx || !o) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(block_idx) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lens) & 3u))
+    return INFLLMV2_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+  const size_t need = ws_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return INFLLMV2_ERR_WORKSPACE;
+  int ns, per;
+  decode_split(p, &ns, &per);
+  AttnParams a;
+  a.idx = block_idx;
+  a.lens = lens;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = p->num_q_heads / p->num_kv_heads;
+  a.Lq = 1;
+  a.Lmax = Lmax;
+  a.topk = p->topk;
+  a.n_splits = ns;
+  a.blocks_per_split = per;
+  a.scale_log2 = scale_log2(p);
+  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * ns;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * ns * kGroupRows;
+  a.part_o = static_cast<float*>(ws);
+  a.part_lse = a.part_o + rows * kHeadDim;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = launch_attn(p, q, static_cast<uint64_t>(p->batch) * p->num_q_heads, k_cache, v_cache,
+                   static_cast<uint64_t>(p->batch) * p->num_kv_heads * Lmax, a, s);
+  if (st != INFLLMV2_OK) return st;
+  attn_merge_kernel<<<static_cast<unsigned>(static_cast<long long>(p->batch) * p->num_kv_heads), 128, 0, s>>>(
+      a.part_o, a.part_lse, ns, p->num_q_heads, p->num_kv_heads, a.G, static_cast<__nv_bfloat16*>(o), lse);
+  return launch_status();
+}
+
+}  // extern "C"
