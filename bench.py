@@ -1,0 +1,469 @@
+"""Benchmark of the InfLLM v2 block-sparse attention path on B200.
+
+A step is one whole prefill of a 128K-token sequence (compress keys -> select blocks ->
+sparse attention) on seeded synthetic inputs already resident in HBM.  The line also
+reports one decode step (select -> sparse attention over a filled cache) of 32 ragged
+sequences of 64K-128K tokens, the same prefill end to end through host buffers, the
+per-kernel rooflines and the CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own independent
+sequence: weak scaling, no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from trainable_block_sparse_compress_b200 import build as lib_build  # noqa: E402
+from trainable_block_sparse_compress_b200 import ops  # noqa: E402
+from trainable_block_sparse_compress_b200.synthetic import WORKLOADS, as_u16, make_inputs  # noqa: E402
+
+METRIC = "128K prefill tokens/s + decode µs/step on 1 B200; % of TC/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(name: str) -> str:
+    with open(os.path.join(ROOT, "trainable_block_sparse_compress_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def dram_traffic(kernel: str, source: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel, {})
+    if e.get("source_sha") != source_sha(source) or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def prefill_flops(p: ops.Params, L: int):
+    """Algorithmic FLOPs of one prefill: (selection, attention on selected blocks)."""
+    t = np.arange(L, dtype=np.int64)
+    nk_vis = np.where(t >= 31, (t - 31) // 16 + 1, 0)
+    sel = 2 * 2 * p.head_dim * p.num_q_heads * p.batch * int(nk_vis.sum())  # 2 passes x 2 flop/MAC
+    cur = t // 64
+    nsel = np.minimum(p.topk, cur + 1)
+    keys = 64 * (nsel - 1) + (t - 64 * cur + 1)
+    attn = 4 * p.head_dim * p.num_q_heads * p.batch * int(keys.sum())  # QK^T and PV
+    gather = 2 * 2 * p.head_dim * 64 * p.num_kv_heads * p.batch * int(nsel.sum())  # K+V bytes
+    return sel, attn, gather
+
+
+def decode_bytes(p: ops.Params, lens: np.ndarray):
+    """Algorithmic bytes of one decode step: (selection: Kc + Q, attention: K/V keys + Q + O)."""
+    lens = lens.astype(np.int64)
+    nk = np.where(lens >= 32, (lens - 32) // 16 + 1, 0)
+    qbytes = p.batch * p.num_q_heads * p.head_dim * 2
+    sel = int(nk.sum()) * p.num_kv_heads * p.head_dim * 2 + qbytes
+    cur = (lens - 1) // 64
+    nsel = np.minimum(p.topk, cur + 1)
+    keys = 64 * (nsel - 1) + (lens - 1 - 64 * cur + 1)
+    attn = int(keys.sum()) * p.num_kv_heads * p.head_dim * 2 * 2 + 2 * qbytes
+    return sel, attn
+
+
+# ----------------------------------------------------------------- our path
+
+def run_ours(args, rank, world, device):
+    pk, peak_src = peaks()
+    wl = WORKLOADS[args.workload]
+    p = ops.Params.from_workload(wl)
+    L = wl.seq_len
+    x = make_inputs(wl, seed=args.seed + rank)
+    q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
+    nk = ops.num_kernels(p, L)
+    kc = torch.empty((p.batch, p.num_kv_heads, nk, p.head_dim), dtype=torch.bfloat16, device=device)
+    idx = torch.empty((p.batch, p.num_kv_heads, L, p.topk), dtype=torch.int32, device=device)
+    o = torch.empty_like(q)
+    lse = torch.empty((p.batch, p.num_q_heads, L), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ops.compress_keys(p, k, out=kc)
+        ops.select_blocks_prefill(p, q, kc, out=idx)
+        ops.sparse_attn_prefill(p, q, k, v, idx, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-kernel device times (events on the launching stream), separate pass
+    names = ["compress", "select", "attn"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        ops.compress_keys(p, k, out=kc)
+        ev[s][1].record(stream)
+        ops.select_blocks_prefill(p, q, kc, out=idx)
+        ev[s][2].record(stream)
+        ops.sparse_attn_prefill(p, q, k, v, idx, out=o, lse=lse)
+        ev[s][3].record(stream)
+    torch.cuda.synchronize()
+    kern_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
+               for i, n in enumerate(names)}
+
+    # the timed region: exactly K steps, barrier + synchronize on both sides
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    ms_t = torch.tensor([ms], device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    ms_per_step = ms / args.steps
+    tokens_per_step = p.batch * L
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+
+    sel_flops, attn_flops, gather_bytes = prefill_flops(p, L)
+    comp_bytes = p.batch * p.num_kv_heads * (L + nk) * p.head_dim * 2
+    tc_peak = pk["bf16_tflops_sustained"]
+    kern = {
+        "compress": {"ms": kern_ms["compress"], "bound": "hbm", "algorithmic_bytes": comp_bytes,
+                     "achieved": comp_bytes / kern_ms["compress"] / 1e6, "unit": "GB/s", "peak": pk["hbm_gbs"]},
+        "select": {"ms": kern_ms["select"], "bound": "tensor", "algorithmic_flops": sel_flops,
+                   "achieved": sel_flops / kern_ms["select"] / 1e9, "unit": "TFLOP/s", "peak": tc_peak},
+        "attn": {"ms": kern_ms["attn"], "bound": "tensor", "algorithmic_flops": attn_flops,
+                 "achieved": attn_flops / kern_ms["attn"] / 1e9, "unit": "TFLOP/s", "peak": tc_peak,
+                 "gather_bytes": gather_bytes, "gather_GBps": gather_bytes / kern_ms["attn"] / 1e6},
+    }
+    for kv in kern.values():
+        kv["frac"] = kv["achieved"] / kv["peak"]
+    top = max(kern, key=lambda n: kern[n]["ms"])
+    src = {"compress": "compress.cuh", "select": "select_prefill.cuh", "attn": "attn.cuh"}[top]
+    kname = {"compress": "compress_kernel", "select": "select_prefill_kernel", "attn": "attn_kernel"}[top]
+    roof = {"kernel": kname, "bound": kern[top]["bound"], "achieved": kern[top]["achieved"],
+            "peak": kern[top]["peak"], "unit": kern[top]["unit"], "frac": kern[top]["frac"],
+            "traffic": dram_traffic(kname, src, args.workload),
+            "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kern[top]['bound'] == 'tensor' else 'hbm_gbs'})"}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": p.batch, "seq_len": L, "num_q_heads": p.num_q_heads,
+                   "num_kv_heads": p.num_kv_heads, "head_dim": p.head_dim, "block": p.block_size,
+                   "kernel": p.kernel_size, "stride": p.kernel_stride, "topk": p.topk, "n_init": p.n_init,
+                   "n_local": p.n_local, "seed": args.seed, "parallelism": f"dp{world} (independent sequences)",
+                   "l2": "inputs larger than L2: each step reads Q (1 GiB) and writes O (1 GiB)"},
+        "roofline": roof,
+        "kernels": kern,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    del kc, idx, o, lse
+
+    if rank == 0 and not args.no_e2e:
+        result["e2e"] = run_e2e(args, p, x, device)
+    del q, k, v
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        result["decode"] = run_decode(args, rank, world, device, pk, peak_src)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args, wl, x)
+    return result
+
+
+def run_e2e(args, p, x, device):
+    """Same prefill through the public calls with host buffers: pinned host Q, K, V are
+    copied in, and O is copied back, inside the timed region."""
+    qh, kh, vh = x.q.pin_memory(), x.k.pin_memory(), x.v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    qd, kd, vd = torch.empty_like(qh, device=device), torch.empty_like(kh, device=device), torch.empty_like(
+        vh, device=device)
+    L = x.q.shape[1]
+    kc = torch.empty((p.batch, p.num_kv_heads, ops.num_kernels(p, L), p.head_dim), dtype=torch.bfloat16,
+                     device=device)
+    idx = torch.empty((p.batch, p.num_kv_heads, L, p.topk), dtype=torch.int32, device=device)
+    od = torch.empty_like(qd)
+
+    def step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        ops.compress_keys(p, kd, out=kc)
+        ops.select_blocks_prefill(p, qd, kc, out=idx)
+        ops.sparse_attn_prefill(p, qd, kd, vd, idx, out=od, want_lse=False)
+        oh.copy_(od, non_blocking=True)
+
+    n = max(2, min(args.steps, 5))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(n):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+    return {"value": p.batch * L / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def run_decode(args, rank, world, device, pk, peak_src):
+    """One decode step (select -> attention) over filled ragged caches, L2 flushed before
+    every step (outside the timed events)."""
+    wl = WORKLOADS[args.decode_workload]
+    p = ops.Params.from_workload(wl)
+    x = make_inputs(wl, seed=args.seed + 1000 + rank)
+    Lmax = wl.seq_len
+    q, k, v, lens = x.q.to(device), x.k.to(device), x.v.to(device), x.lens.to(device)
+    kc = ops.compress_keys(p, k, lens=lens)  # cache maintenance, not timed
+    idx = torch.empty((p.batch, p.num_kv_heads, 1, p.topk), dtype=torch.int32, device=device)
+    o = torch.empty_like(q)
+    lse = torch.empty((p.batch, p.num_q_heads), dtype=torch.float32, device=device)
+    ws_s = torch.empty(ops.workspace_size(p, 2, Lmax), dtype=torch.uint8, device=device)
+    ws_a = torch.empty(ops.workspace_size(p, 4, Lmax), dtype=torch.uint8, device=device)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ops.select_blocks_decode(p, q, kc, lens, Lmax, out=idx, ws=ws_s)
+        ops.sparse_attn_decode(p, q, k, v, lens, idx, out=o, lse=lse, ws=ws_a)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    n = max(args.steps, 20)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    for s in range(n):
+        flush.zero_()
+        ev[s][0].record(stream)
+        ops.select_blocks_decode(p, q, kc, lens, Lmax, out=idx, ws=ws_s)
+        ev[s][1].record(stream)
+        ops.sparse_attn_decode(p, q, k, v, lens, idx, out=o, lse=lse, ws=ws_a)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    sel_us = [ev[s][0].elapsed_time(ev[s][1]) * 1e3 for s in range(n)]
+    att_us = [ev[s][1].elapsed_time(ev[s][2]) * 1e3 for s in range(n)]
+    step_us = [a + b for a, b in zip(sel_us, att_us)]
+    us = statistics.median(step_us)
+    us_t = torch.tensor([us], device=device)
+    if world > 1:
+        torch.distributed.all_reduce(us_t, op=torch.distributed.ReduceOp.MAX)
+    us = float(us_t.item())
+    sel_b, att_b = decode_bytes(p, x.lens.numpy())
+    hbm = pk["hbm_gbs"]
+    sel_med, att_med = statistics.median(sel_us), statistics.median(att_us)
+    return {
+        "workload": args.decode_workload, "value": us, "unit": "us/step", "higher_is_better": False,
+        "batch": p.batch, "mean_len": float(x.lens.float().mean()), "steps": n,
+        "l2": "flushed before every step (2x L2 write, outside the timed events)",
+        "roofline": {"bound": "hbm", "achieved": (sel_b + att_b) / us / 1e3, "peak": hbm, "unit": "GB/s",
+                     "frac": (sel_b + att_b) / us / 1e3 / hbm, "algorithmic_bytes": sel_b + att_b,
+                     "peak_source": f"{peak_src} (hbm_gbs)"},
+        "kernels": {
+            "select": {"us": sel_med, "algorithmic_bytes": sel_b, "achieved_GBps": sel_b / sel_med / 1e3},
+            "attn": {"us": att_med, "algorithmic_bytes": att_b, "achieved_GBps": att_b / att_med / 1e3},
+        },
+        "gpu_launches_per_step": 4,
+    }
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_rows_time(wl, x, rows):
+    import oracle
+    op = oracle.Params(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, wl.kernel_size,
+                       wl.kernel_stride, wl.topk, wl.n_init, wl.n_local)
+    q, k, v = as_u16(x.q), as_u16(x.k), as_u16(x.v)
+    t0 = time.perf_counter()
+    kc = oracle.compress(op, k)
+    idx = oracle.select(op, q, kc, rows=rows)
+    oracle.attn(op, q, k, v, idx, rows=rows)
+    return time.perf_counter() - t0
+
+
+def sample_rows(L, n):
+    # evenly strided over the sequence, so the mean cost per row matches the full prefill
+    return np.unique(np.linspace(0, L - 1, n).astype(np.int64))
+
+
+def cpu_baseline(args, wl, x, target_s=12.0):
+    import oracle
+    L = wl.seq_len
+    rows = sample_rows(L, 64)
+    dt = oracle_rows_time(wl, x, rows)
+    n = int(min(L, max(64, len(rows) * target_s / max(dt, 1e-3))))
+    rows = sample_rows(L, n)
+    dt = oracle_rows_time(wl, x, rows)
+    return {"value": wl.batch * len(rows) / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{len(rows)} query rows evenly strided over the {L}-token prefill (all heads), "
+                      f"plus key compression of the whole sequence; tokens/s = rows / time"}
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on bounded samples of the same workload."""
+    import oracle
+    oracle.build()
+    wl = WORKLOADS[args.workload]
+    x = make_inputs(wl, seed=args.seed)
+    L = wl.seq_len
+    rows = sample_rows(L, args.reference_rows)
+    for _ in range(args.warmup):
+        oracle_rows_time(wl, x, rows[:8])
+    times = [oracle_rows_time(wl, x, rows) for _ in range(args.steps)]
+    dt = sum(times)
+    value = wl.batch * len(rows) * args.steps / dt
+    cores = oracle.num_threads()
+    sample = (f"{len(rows)} query rows evenly strided over the {L}-token prefill per step (all heads), "
+              f"plus key compression of the whole sequence")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch": wl.batch, "seq_len": L, "num_q_heads": wl.num_q_heads,
+                       "num_kv_heads": wl.num_kv_heads, "topk": wl.topk, "seed": args.seed},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_128k")
+    ap.add_argument("--decode-workload", default="decode_ragged_128k")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-rows", type=int, default=96)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    lib_build.build()
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+        err = ops.device_error(clear=True)
+        res["device_error"] = err
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
