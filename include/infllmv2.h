@@ -164,6 +164,31 @@ INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const voi
                                 const int32_t* block_idx, void* o, float* lse, void* ws,
                                 size_t ws_bytes, infllmv2_stream_t stream);
 
+/* Decode sparse attention that allocates nothing and takes no workspace.  The paper has
+ * no counterpart to this entry point: it exists for callers that cannot allocate device
+ * memory at call time -- e.g. an engine plugin whose execute step must not allocate, or
+ * a service that reserves its whole memory budget at start-up and forbids later
+ * cudaMalloc.  Same arguments and results as infllmv2_sparse_attn_decode without
+ * ws/ws_bytes; the split partials live in a fixed 8 MiB array inside the library
+ * (INFLLMV2_NOALLOC_SCRATCH_BYTES), which every GPU that loads the library holds until
+ * the process exits.
+ *  - Returns INFLLMV2_ERR_WORKSPACE, without launching anything, when the problem needs
+ *    more scratch than that (the need is infllmv2_workspace_size(p,
+ *    INFLLMV2_OP_ATTN_DECODE, Lmax); e.g. B * Hkv = 64 sequence-heads fit easily).
+ *  - The first call on a device looks up the array's device address (one
+ *    cudaGetSymbolAddress, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device uses the same array, and nothing in it needs to start at
+ *    zero (each call overwrites the parts it reads).  Two calls whose kernels overlap on
+ *    the GPU (e.g. on two streams) race on the array and give undefined results: order
+ *    them on one stream or with events. */
+#define INFLLMV2_NOALLOC_SCRATCH_BYTES (8u << 20)
+INFLLMV2_API int infllmv2_sparse_attn_decode_noalloc(const infllmv2_params* p, const void* q,
+                                                     const void* k_cache, const void* v_cache,
+                                                     const int32_t* lens, int32_t Lmax,
+                                                     const int32_t* block_idx, void* o, float* lse,
+                                                     infllmv2_stream_t stream);
+
 /* Workspace bytes needed by `op` (INFLLMV2_OP_*) for sequence length L_or_Lmax, or 0
  * when the op needs none; (size_t)-1 for invalid parameters. */
 INFLLMV2_API size_t infllmv2_workspace_size(const infllmv2_params* p, int op, int32_t L_or_Lmax);

@@ -28,6 +28,7 @@ OP_ATTN_PREFILL = 3
 OP_ATTN_DECODE = 4
 
 MAX_SEQ_LEN = 262144
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 # every symbol the header declares, with (restype, argtypes)
 _vp = ctypes.c_void_p
@@ -60,6 +61,7 @@ SIGNATURES = {
     "infllmv2_select_blocks": (_int, [_P, _int, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_prefill": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "infllmv2_sparse_attn_decode_noalloc": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "infllmv2_workspace_size": (_sz, [_P, _int, _i32]),
     "infllmv2_check_params": (_int, [_P]),
     "infllmv2_status_string": (ctypes.c_char_p, [_int]),

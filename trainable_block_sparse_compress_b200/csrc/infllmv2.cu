@@ -378,3 +378,45 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ decode attention without allocation
+// The split partials of infllmv2_sparse_attn_decode_noalloc live in this file-scope
+// device array instead of a caller workspace.  Host code only ever sees the symbol's
+// host-side stand-in, so the device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[INFLLMV2_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return INFLLMV2_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return INFLLMV2_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return INFLLMV2_OK;
+}
+}  // namespace
+
+extern "C" int infllmv2_sparse_attn_decode_noalloc(const infllmv2_params* p, const void* q, const void* k_cache,
+                                                   const void* v_cache, const int32_t* lens, int32_t Lmax,
+                                                   const int32_t* block_idx, void* o, float* lse,
+                                                   infllmv2_stream_t stream) {
+  const int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  const size_t need = ws_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax);
+  if (need == static_cast<size_t>(-1)) return INFLLMV2_ERR_INVALID_ARG;
+  if (need > INFLLMV2_NOALLOC_SCRATCH_BYTES) return INFLLMV2_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int sst = noalloc_scratch(&scratch);
+  if (sst != INFLLMV2_OK) return sst;
+  return infllmv2_sparse_attn_decode(p, q, k_cache, v_cache, lens, Lmax, block_idx, o, lse, scratch,
+                                     INFLLMV2_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -185,6 +185,28 @@ def sparse_attn_decode(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cach
     return out, lse
 
 
+def sparse_attn_decode_noalloc(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               lens: torch.Tensor, block_idx: torch.Tensor, out: torch.Tensor,
+                               lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Decode attention for callers that cannot allocate device memory at call time: the
+    caller passes preallocated outputs and the library uses its own fixed scratch array
+    (no workspace).  Calls that overlap on the GPU race on that array."""
+    Lmax = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (p.batch, p.num_q_heads, p.head_dim))
+    _need(k_cache, "k_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(v_cache, "v_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(lens, "lens", torch.int32, (p.batch,))
+    _need(block_idx, "block_idx", torch.int32, (p.batch, p.num_kv_heads, 1, p.topk))
+    _need(out, "o", torch.bfloat16, tuple(q.shape))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (p.batch, p.num_q_heads))
+    st = _lib.load().infllmv2_sparse_attn_decode_noalloc(ctypes.byref(p.c()), _ptr(q), _ptr(k_cache),
+                                                         _ptr(v_cache), _ptr(lens), Lmax, _ptr(block_idx),
+                                                         _ptr(out), _ptr(lse), _stream())
+    _lib.check("infllmv2_sparse_attn_decode_noalloc", st)
+    return out, lse
+
+
 def device_error(clear: bool = True) -> int:
     v = int(_lib.load().infllmv2_device_error(1 if clear else 0))
     if v < 0:
