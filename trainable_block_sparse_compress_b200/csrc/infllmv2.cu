@@ -16,6 +16,7 @@
 #include "compress.cuh"
 #include "select_decode.cuh"
 #include "select_prefill.cuh"
+#include "select_prefill_tc.cuh"
 #include "topk.cuh"
 
 using namespace infllmv2;
@@ -85,6 +86,23 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+// 3-D view [tokens, heads, 128] of the prefill queries, box {64 columns, 16 heads, 8
+// tokens}: the 128 (token, head) rows of one selection tile.
+bool make_q_map_3d(CUtensorMap* m, const void* q, uint64_t tokens, uint64_t heads) {
+  if (!get_encoder()) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, static_cast<cuuint64_t>(heads * kHeadDim * 2)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kGroupRows), static_cast<cuuint32_t>(kTcTokens)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA; }
 
@@ -245,6 +263,20 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
     a.nblk_cap = nblk_cap;
     a.scale_log2 = scale_log2(p);
     a.tiles_per_bg = (L + kSelWarps - 1) / kSelWarps;
+    if (G == kGroupRows && nk > 0 && sel_tc_smem_bytes(nblk_cap) <= kMaxSmem) {
+      // tensor-core path: 8 tokens x 16 heads per 128-row UMMA tile
+      static_assert(kTcTokens == kSelWarps, "both prefill selection kernels tile 8 tokens");
+      CUtensorMap tm_q3, tm_kc128;
+      if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * L, p->num_q_heads)) return INFLLMV2_ERR_CUDA;
+      if (!make_map(&tm_kc128, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kTcN))
+        return INFLLMV2_ERR_CUDA;
+      const size_t smem = sel_tc_smem_bytes(nblk_cap);
+      if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_tc_kernel), smem)) != INFLLMV2_OK) return st;
+      const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
+      if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+      select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kc128, a);
+      return launch_status();
+    }
     const size_t smem = sel_prefill_smem_bytes(nblk_cap);
     if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_kernel), smem)) != INFLLMV2_OK) return st;
     const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
