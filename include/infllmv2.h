@@ -24,7 +24,8 @@
  *    negative status nothing was launched and no output was touched.
  *  - A kernel that waits on the GPU never waits without a bound: if an internal wait
  *    exceeds its limit the kernel stops early and sets a device error word, which
- *    infllmv2_device_error() reads (outputs of that call are then undefined).
+ *    infllmv2_device_error() reads.  The word is sticky: until it is cleared, later
+ *    waits give up at once, so outputs of that call and of later calls are undefined.
  *  - Query positions: prefill queries are tokens 0..L-1 of a fresh sequence; a decode
  *    query is the last token of its sequence, at position lens[b]-1, and its own key
  *    and value are already in the cache.

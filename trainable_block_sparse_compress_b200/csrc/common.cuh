@@ -3,7 +3,8 @@
 // PTX wrappers for mbarriers, TMA tile loads (never with cluster multicast),
 // ldmatrix and the bf16 m16n8k16 MMA, plus time-bounded mbarrier waits: a wait that
 // exceeds its limit sets a device error word and marks the CTA aborted, after which
-// every later wait in the CTA returns at once, so the kernel runs to its end instead
+// every later wait in the CTA -- and, through the sticky error word, in every other CTA
+// until the word is cleared -- returns at once, so the kernel runs to its end instead
 // of hanging.
 #pragma once
 
@@ -76,6 +77,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort) return false;
+      if (*reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0u) {  // another CTA gave up
+        *abort = 1;
+        return false;
+      }
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;
         atomicOr(&g_device_error, 1u);

@@ -266,15 +266,16 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
     if (G == kGroupRows && nk > 0 && sel_tc_smem_bytes(nblk_cap) <= kMaxSmem) {
       // tensor-core path: 8 tokens x 16 heads per 128-row UMMA tile
       static_assert(kTcTokens == kSelWarps, "both prefill selection kernels tile 8 tokens");
-      CUtensorMap tm_q3, tm_kc128;
-      if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * L, p->num_q_heads)) return INFLLMV2_ERR_CUDA;
-      if (!make_map(&tm_kc128, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kTcN))
+      CUtensorMap tm_q3, tm_kca, tm_kcb;
+      const uint64_t kc_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk;
+      if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * L, p->num_q_heads) ||
+          !make_map(&tm_kca, kc, kc_rows, kTcN) || !make_map(&tm_kcb, kc, kc_rows, kTcNB))
         return INFLLMV2_ERR_CUDA;
       const size_t smem = sel_tc_smem_bytes(nblk_cap);
       if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_tc_kernel), smem)) != INFLLMV2_OK) return st;
       const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
       if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
-      select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kc128, a);
+      select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kca, tm_kcb, a);
       return launch_status();
     }
     const size_t smem = sel_prefill_smem_bytes(nblk_cap);

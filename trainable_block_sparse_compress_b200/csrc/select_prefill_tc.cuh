@@ -6,17 +6,19 @@
 // block, sum over the group's heads, top-k with forced initial/local blocks.
 //
 // One CTA = 8 consecutive query tokens of one (sequence, kv-head): 8 x 16 heads = the 128
-// rows (M) of a UMMA tile.  Warp roles:
-//   warp 4  TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then
-//           128-kernel tiles of Kc (128 x 128 bf16, 32 KB) through a 3-stage ring, twice;
-//   warp 5  allocates 256 TMEM columns and, from one thread, issues for every Kc tile
-//           8 UMMAs (M128 N128 K16, bf16 -> fp32) into one of two TMEM accumulators;
-//   warps 0-3  epilogue: thread (w, lane) owns TMEM lane 32 w + lane = row
-//           (token, head).  Pass A keeps an online log-sum-exp of its row; pass B pools
-//           block maxima along its row, forms p = exp(m - lse), sums the 16 heads of a
-//           token with a 16-lane transpose-reduce (30 shuffles per 32 blocks) and stores
-//           the block keys in shared memory; then each warp radix-selects the top blocks
-//           of its two tokens.
+// rows (M) of a UMMA tile.  Warp roles (320 threads):
+//   warp 8  TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then Kc tiles
+//           through a 3-stage ring: pass A tiles of 128 kernels, pass B tiles of 144
+//           kernels that start 16 kernels early, so each pass-B tile also holds the
+//           kernel straddling its first block (4j - 1) and is self-contained;
+//   warp 9  allocates TMEM and, from one thread, issues per tile 8 UMMAs (M128 x N128 or
+//           N144, K16, bf16 -> fp32) into one of two TMEM accumulators;
+//   warps 0-7  two epilogue warpgroups taking alternate tiles; thread (w, lane) owns TMEM
+//           lane 32 (w % 4) + lane = row (token, head).  Pass A keeps an online
+//           log-sum-exp per row (the two warpgroups' partials are merged once); pass B
+//           pools block maxima along the row, forms p = exp(m - lse) and sums the 16
+//           heads of a token with a 16-lane transpose-reduce; block keys go to shared
+//           memory; finally warp w radix-selects the top blocks of token w.
 #pragma once
 #include "common.cuh"
 #include "select_prefill.cuh"
@@ -26,81 +28,81 @@
 namespace infllmv2 {
 
 constexpr int kTcTokens = 8;
-constexpr int kTcN = 128;
+constexpr int kTcN = 128;              // kernels per pass-A tile
+constexpr int kTcOverlap = 16;         // extra leading kernels of a pass-B tile
+constexpr int kTcNB = kTcN + kTcOverlap;  // 144 kernels per pass-B tile
 constexpr int kTcStages = 3;
-constexpr int kTcTileBytes = kTcN * kHeadDim * 2;  // 32 KB
-constexpr int kTcQBytes = 128 * kHeadDim * 2;      // 32 KB
-constexpr int kTcEpiWarps = 4;
+constexpr int kTcHalfBytes = kTcNB * 128;   // one 64-column half of a stage (144 rows x 128 B)
+constexpr int kTcStageBytes = 2 * kTcHalfBytes;
+constexpr int kTcQBytes = 128 * kHeadDim * 2;  // 32 KB
+constexpr int kTcEpiWarps = 8;
 constexpr int kTcThreads = 32 * (kTcEpiWarps + 2);
-constexpr uint32_t kTcTmemCols = 2 * kTcN;
+constexpr uint32_t kTcTmemCols = 512;
+constexpr uint32_t kTcAccStride = 256;  // TMEM column offset between the two accumulators
 
 struct SelTcSmem {
   uint64_t qbar, full[kTcStages], empty[kTcStages], tfull[2], tempty[2], mma_done;
+  float2 part[2][128];  // pass-A (max, sum) per warpgroup and row
   uint32_t tmem_base;
   volatile int abort;
 };
 
 inline size_t sel_tc_smem_bytes(int nblk_cap) {
-  return 1024 + kTcQBytes + static_cast<size_t>(kTcStages) * kTcTileBytes +
+  return 1024 + kTcQBytes + static_cast<size_t>(kTcStages) * kTcStageBytes +
          static_cast<size_t>(kTcTokens) * nblk_cap * 4 + kTcEpiWarps * 256 * 4 + sizeof(SelTcSmem);
 }
 
-// Sum of v over the 16 lanes sharing lane bits 4+ (one token's heads), scattered: lane
-// L (mod 16) returns the totals of entries 2L and 2L+1.
-__device__ __forceinline__ float2 reduce_scatter16(const float (&v)[32]) {
+// Sum of v over the 16 lanes that share lane bit 4 (one token's heads), scattered: lane
+// L (mod 16) returns the total of entry L.  15 shuffles.
+__device__ __forceinline__ float reduce_scatter16(const float (&v)[16]) {
   const int lane = threadIdx.x & 31;
-  float a[16];
+  float a[8];
   {
     const bool up = lane & 8;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float send = up ? v[i] : v[i + 16];
-      const float keep = up ? v[i + 16] : v[i];
+    for (int i = 0; i < 8; ++i) {
+      const float send = up ? v[i] : v[i + 8];
+      const float keep = up ? v[i + 8] : v[i];
       a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
     }
   }
-  float b8[8];
+  float b4[4];
   {
     const bool up = lane & 4;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float send = up ? a[i] : a[i + 8];
-      const float keep = up ? a[i + 8] : a[i];
-      b8[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    for (int i = 0; i < 4; ++i) {
+      const float send = up ? a[i] : a[i + 4];
+      const float keep = up ? a[i + 4] : a[i];
+      b4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
     }
   }
-  float c4[4];
+  float c2[2];
   {
     const bool up = lane & 2;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float send = up ? b8[i] : b8[i + 4];
-      const float keep = up ? b8[i + 4] : b8[i];
-      c4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-  }
-  float d2[2];
-  {
-    const bool up = lane & 1;
-#pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const float send = up ? c4[i] : c4[i + 2];
-      const float keep = up ? c4[i + 2] : c4[i];
-      d2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+      const float send = up ? b4[i] : b4[i + 2];
+      const float keep = up ? b4[i + 2] : b4[i];
+      c2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
     }
   }
-  return make_float2(d2[0], d2[1]);
+  const bool up = lane & 1;
+  const float send = up ? c2[0] : c2[1];
+  const float keep = up ? c2[1] : c2[0];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
-// grid = B * Hkv * ceil(L / 8) (latest tiles first), block = 192.  Requires G == 16.
+__device__ __forceinline__ float max4(float a, float b, float c, float d) { return fmaxf(fmaxf(a, b), fmaxf(c, d)); }
+
+// grid = B * Hkv * ceil(L / 8) (latest tiles first), block = 320.  Requires G == 16.
 __global__ void __launch_bounds__(kTcThreads, 1)
-    select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q3, const __grid_constant__ CUtensorMap tm_kc,
-                             const SelPrefillParams p) {
+    select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q3, const __grid_constant__ CUtensorMap tm_kca,
+                             const __grid_constant__ CUtensorMap tm_kcb, const SelPrefillParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = align_smem(smem_raw, 1024);
   unsigned char* qs = base;
   unsigned char* ring = qs + kTcQBytes;
-  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + kTcStages * kTcTileBytes);
+  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + kTcStages * kTcStageBytes);
   uint32_t* hist_all = keys_all + kTcTokens * p.nblk_cap;
   SelTcSmem& S = *reinterpret_cast<SelTcSmem*>(hist_all + kTcEpiWarps * 256);
 
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S.tfull[a], 1);
-      mbar_init(&S.tempty[a], kTcEpiWarps);
+      mbar_init(&S.tempty[a], 4);  // the four warps of the warpgroup that owns accumulator a
     }
     mbar_init(&S.mma_done, 1);
     S.abort = 0;
@@ -142,7 +144,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------------------------------------------------------- TMA warp
     if (lane == 0 && T > 0) {
       prefetch_tmap(&tm_q3);
-      prefetch_tmap(&tm_kc);
+      prefetch_tmap(&tm_kca);
+      prefetch_tmap(&tm_kcb);
       mbar_arrive_expect_tx(&S.qbar, kTcQBytes);
       tma_load_3d(qs, &tm_q3, &S.qbar, 0, g * kGroupRows, b * p.L + t0);
       tma_load_3d(qs + kTcQBytes / 2, &tm_q3, &S.qbar, 64, g * kGroupRows, b * p.L + t0);
@@ -151,11 +154,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int st = n % kTcStages, u = n / kTcStages;
         if (u > 0) mbar_wait(&S.empty[st], (u - 1) & 1, &S.abort);
         if (S.abort) break;
-        const int c = n < TA ? n : n - TA;
-        unsigned char* dst = ring + st * kTcTileBytes;
-        mbar_arrive_expect_tx(&S.full[st], kTcTileBytes);
-        tma_load_2d(dst, &tm_kc, &S.full[st], 0, row0 + c * kTcN);
-        tma_load_2d(dst + kTcTileBytes / 2, &tm_kc, &S.full[st], 64, row0 + c * kTcN);
+        unsigned char* dst = ring + st * kTcStageBytes;
+        if (n < TA) {
+          const int r = row0 + n * kTcN;
+          mbar_arrive_expect_tx(&S.full[st], 2 * kTcN * 128);
+          tma_load_2d(dst, &tm_kca, &S.full[st], 0, r);
+          tma_load_2d(dst + kTcHalfBytes, &tm_kca, &S.full[st], 64, r);
+        } else {
+          const int r = row0 + (n - TA) * kTcN - kTcOverlap;  // may start before row 0: zero fill
+          mbar_arrive_expect_tx(&S.full[st], 2 * kTcNB * 128);
+          tma_load_2d(dst, &tm_kcb, &S.full[st], 0, r);
+          tma_load_2d(dst + kTcHalfBytes, &tm_kcb, &S.full[st], 64, r);
+        }
       }
     }
     return;
@@ -164,7 +174,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kTcEpiWarps + 1) {
     // ---------------------------------------------------------------- MMA warp
     if (lane == 0 && T > 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kTcN, false, false);
+      constexpr uint32_t idesc_a = idesc_bf16_f32(128, kTcN, false, false);
+      constexpr uint32_t idesc_b = idesc_bf16_f32(128, kTcNB, false, false);
       mbar_wait(&S.qbar, 0, &S.abort);
       const uint32_t qa = smem_u32(qs);
       for (int n = 0; n < T; ++n) {
@@ -172,13 +183,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_wait(&S.full[st], (n / kTcStages) & 1, &S.abort);
         if (u > 0) mbar_wait(&S.tempty[acc], (u - 1) & 1, &S.abort);
         tc_fence_after();
-        const uint32_t kb = smem_u32(ring + st * kTcTileBytes);
+        const uint32_t kb = smem_u32(ring + st * kTcStageBytes);
+        const uint32_t idesc = n < TA ? idesc_a : idesc_b;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = static_cast<uint32_t>((k >> 2) * (kTcQBytes / 2) + (k & 3) * 32);
-          const uint32_t offb = static_cast<uint32_t>((k >> 2) * (kTcTileBytes / 2) + (k & 3) * 32);
-          umma_bf16(tmem + static_cast<uint32_t>(acc * kTcN), desc_k_sw128(qa + off), desc_k_sw128(kb + offb),
-                    idesc, k > 0 ? 1u : 0u);
+          const uint32_t offb = static_cast<uint32_t>((k >> 2) * kTcHalfBytes + (k & 3) * 32);
+          umma_bf16(tmem + static_cast<uint32_t>(acc) * kTcAccStride, desc_k_sw128(qa + off),
+                    desc_k_sw128(kb + offb), idesc, k > 0 ? 1u : 0u);
         }
         umma_commit(&S.empty[st]);
         umma_commit(&S.tfull[acc]);
@@ -195,39 +207,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ---------------------------------------------------------------- epilogue warps
-  const int w = warp;
-  const int tok = (32 * w + lane) >> 4;
-  const int t_raw = t0 + tok;
-  const bool tok_ok = t_raw < p.L;
-  const int t = tok_ok ? t_raw : p.L - 1;
+  const int wg = warp >> 2;   // warpgroup: takes tiles n with n % 2 == wg
+  const int wq = warp & 3;    // TMEM lane quarter
+  const int row = 32 * wq + lane;
+  const int tok = row >> 4;
+  const int t = min(t0 + tok, p.L - 1);  // rows of tokens past L compute but write nothing
   const int imax = last_visible_kernel(t);
   const int cur = t / kBlock;
-  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * w) << 16);
+  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
   const float sl2 = p.scale_log2;
 
-  // pass A: log-sum-exp of this row over its visible kernels (base 2)
+  // pass A: log-sum-exp of this row over its visible kernels (base 2), alternate tiles
   float m = -INFINITY, l = 0.f;
-  for (int n = 0; n < TA; ++n) {
+  for (int n = wg; n < TA; n += 2) {
     const int acc = n & 1;
     mbar_wait(&S.tfull[acc], (n >> 1) & 1, &S.abort);
     tc_fence_after();
 #pragma unroll 1
     for (int q = 0; q < kTcN / 32; ++q) {
       uint32_t v[32];
-      tmem_ld32(trow + static_cast<uint32_t>(acc * kTcN + 32 * q), v);
+      tmem_ld32(trow + static_cast<uint32_t>(acc) * kTcAccStride + static_cast<uint32_t>(32 * q), v);
       const int i0 = n * kTcN + 32 * q;
       float x[32];
-      float cm = -INFINITY;
+      if (i0 + 31 <= imax) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
-        cm = fmaxf(cm, x[e]);
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]) * sl2;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
       }
+      float c8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c8[e] = max4(x[e], x[e + 8], x[e + 16], x[e + 24]);
+      const float cm = fmaxf(max4(c8[0], c8[1], c8[2], c8[3]), max4(c8[4], c8[5], c8[6], c8[7]));
       if (cm != -INFINITY) {
         const float mn = fmaxf(m, cm);
-        float s = 0.f;
+        float s8[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s += ex2(x[e] - mn);
+        for (int e = 0; e < 8; ++e)
+          s8[e] = (ex2(x[e] - mn) + ex2(x[e + 8] - mn)) + (ex2(x[e + 16] - mn) + ex2(x[e + 24] - mn));
+        const float s = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
         l = l * ex2(m - mn) + s;
         m = mn;
       }
@@ -236,65 +255,78 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.tempty[acc]);
   }
-  const float lse = l > 0.f ? m + lg2(l) : INFINITY;
-
-  uint32_t* keys = keys_all + tok * p.nblk_cap;
-  for (int j = lane & 15; j <= cur; j += 16) keys[j] = 0u;
-  __syncwarp();
+  // zero the key row of token `warp` (blocks 0..cur) while the warpgroups meet
+  {
+    const int tz = min(t0 + warp, p.L - 1);
+    uint32_t* kz = keys_all + warp * p.nblk_cap;
+    for (int j = lane; j <= tz / kBlock; j += 32) kz[j] = 0u;
+  }
+  S.part[wg][row] = make_float2(m, l);
+  named_bar_sync(2, 32 * kTcEpiWarps);
+  float lse;
+  {
+    const float2 a0 = S.part[0][row], a1 = S.part[1][row];
+    const float M = fmaxf(a0.x, a1.x);
+    const float L = (M == -INFINITY) ? 0.f : a0.y * ex2(a0.x - M) + a1.y * ex2(a1.x - M);
+    lse = L > 0.f ? M + lg2(L) : INFINITY;
+  }
 
   // pass B: block maxima along the row, p = exp(m - lse), group sum over the 16 heads
-  float carry = -INFINITY;  // logit of the kernel just before the current tile
-  for (int n = TA; n < T; ++n) {
+  uint32_t* keys = keys_all + tok * p.nblk_cap;
+  for (int n = TA + ((TA & 1) != wg ? 1 : 0); n < T; n += 2) {
     const int c = n - TA;
     const int acc = n & 1;
     mbar_wait(&S.tfull[acc], (n >> 1) & 1, &S.abort);
     tc_fence_after();
-    float pb[32];
+    const uint32_t tacc = trow + static_cast<uint32_t>(acc) * kTcAccStride;
+    // column kTcOverlap-1 holds kernel 128c - 1, the straddle of block 32c
+    // (tcgen05.ld is warp-collective: load unconditionally, then mask)
+    const int istr = c * kTcN - 1;
+    const float cv = __uint_as_float(tmem_ld1(tacc + kTcOverlap - 1));
+    float carry = (istr >= 0 && istr <= imax) ? cv * sl2 : -INFINITY;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      float pb[16];
 #pragma unroll
-    for (int q = 0; q < kTcN / 32; ++q) {
-      uint32_t v[32];
-      tmem_ld32(trow + static_cast<uint32_t>(acc * kTcN + 32 * q), v);
-      const int i0 = c * kTcN + 32 * q;
-      float x[32];
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int q = 2 * half + q2;
+        uint32_t v[32];
+        tmem_ld32(tacc + static_cast<uint32_t>(kTcOverlap + 32 * q), v);
+        const int i0 = c * kTcN + 32 * q;
+        float x[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
+        for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
 #pragma unroll
-      for (int gq = 0; gq < 8; ++gq) {
-        float mb = fmaxf(fmaxf(x[4 * gq], x[4 * gq + 1]), fmaxf(x[4 * gq + 2], x[4 * gq + 3]));
-        mb = fmaxf(mb, gq == 0 ? carry : x[4 * gq - 1]);
-        pb[8 * q + gq] = ex2(mb - lse);
+        for (int gq = 0; gq < 8; ++gq) {
+          const float mb = fmaxf(max4(x[4 * gq], x[4 * gq + 1], x[4 * gq + 2], x[4 * gq + 3]),
+                                 gq == 0 ? carry : x[4 * gq - 1]);
+          pb[8 * q2 + gq] = ex2(mb - lse);
+        }
+        carry = x[31];
       }
-      carry = x[31];
+      const float sum = reduce_scatter16(pb);
+      const int j = 32 * c + 16 * half + (lane & 15);
+      if (j <= cur) {
+        const bool eligible = max(4 * j - 1, 0) <= imax;
+        const bool forced = j < p.n_init || j > cur - p.n_local;
+        keys[j] = (eligible && !forced) ? __float_as_uint(sum) + 1u : 0u;
+      }
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.tempty[acc]);
-    const float2 sum = reduce_scatter16(pb);
-    const int j0 = 32 * c + 2 * (lane & 15);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int j = j0 + e;
-      if (j <= cur) {
-        const bool eligible = max(4 * j - 1, 0) <= imax;
-        const bool forced = j < p.n_init || j > cur - p.n_local;
-        keys[j] = (eligible && !forced) ? __float_as_uint(e ? sum.y : sum.x) + 1u : 0u;
-      }
-    }
   }
   tc_fence_before();
-  named_bar_sync(1, 32 * (kTcEpiWarps + 1));  // TMEM no longer read: warp 5 may free it
-  __syncwarp();
+  named_bar_sync(1, 32 * (kTcEpiWarps + 1));  // TMEM no longer read: warp 9 may free it
+  named_bar_sync(2, 32 * kTcEpiWarps);        // all keys written
 
-  // top-k of this warp's two tokens
-#pragma unroll 1
-  for (int tt = 0; tt < 2; ++tt) {
-    const int tk = 2 * w + tt;
-    const int tr = t0 + tk;
-    if (tr >= p.L) break;
+  // top-k of token `warp`
+  const int tr = t0 + warp;
+  if (tr < p.L) {
     const int cu = tr / kBlock;
-    const uint32_t* kt = keys_all + tk * p.nblk_cap;
+    const uint32_t* kt = keys_all + warp * p.nblk_cap;
     const int want = p.topk - forced_count(cu, p.n_init, p.n_local);
-    const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + w * 256);
+    const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + warp * 256);
     int32_t* out = p.idx + ((bg * p.L + tr) * static_cast<long long>(p.topk));
     warp_emit_selection(kt, cu + 1, th, cu, p.n_init, p.n_local, p.topk, out);
   }

@@ -5,10 +5,9 @@
 // scoring blocks): higher score first, lower block index first among equal scores.
 // Scores are non-negative fp32 group sums, so their IEEE bit patterns order like the
 // values.  A candidate's key is bits(score) + 1 and a non-candidate's key is 0.
-// The k-th largest key is found by a most-significant-digit radix select (4 rounds of
-// 8 bits, shared-memory histogram); the list is then written in ascending block order
-// with forced blocks first-class members and ties at the threshold taken from the
-// lowest indices.
+// The k-th largest key is found by bisection on the key bits with warp-wide counts; the
+// list is then written in ascending block order with forced blocks first-class members
+// and ties at the threshold taken from the lowest indices.
 #pragma once
 #include "common.cuh"
 
@@ -19,10 +18,28 @@ struct TopkThreshold {
   int ties;      // how many keys equal to T are taken (0 when T == 0: take all > 0)
 };
 
-// One warp.  keys[0..n) in shared memory; `want` keys to take; hist: 256 words of
-// shared scratch owned by this warp.
+// One warp.  keys[0..n) in shared memory; `want` keys to take.  Finds the want-th
+// largest key T by bisection on its bits, most significant first: T >= c exactly when
+// at least `want` keys are >= c.  Each lane holds up to kTopkRegKeys keys in registers
+// (n <= 32 * kTopkRegKeys); larger n re-reads shared memory each step.  No atomics.
+constexpr int kTopkRegKeys = 64;
+
+__device__ __forceinline__ int warp_count_ge_regs(const uint32_t (&kr)[kTopkRegKeys], uint32_t c) {
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < kTopkRegKeys; ++i) cnt += kr[i] >= c ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
+}
+
+__device__ __forceinline__ int warp_count_ge_smem(const uint32_t* keys, int n, uint32_t c) {
+  const int lane = threadIdx.x & 31;
+  int cnt = 0;
+  for (int i = lane; i < n; i += 32) cnt += keys[i] >= c ? 1 : 0;
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
+}
+
 __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* keys, int n, int want,
-                                                              uint32_t* hist) {
+                                                              uint32_t* /*unused scratch*/) {
   const int lane = threadIdx.x & 31;
   TopkThreshold r;
   if (want <= 0) {
@@ -30,66 +47,40 @@ __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* ke
     r.ties = 0;
     return r;
   }
-  uint32_t prefix = 0, pmask = 0;
-  int need = want;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  uint32_t T = 0;
+  if (n <= 32 * kTopkRegKeys) {
+    uint32_t kr[kTopkRegKeys];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0;
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-      const uint32_t k = keys[i];
-      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    for (int i = 0; i < kTopkRegKeys; ++i) {
+      const int j = lane + 32 * i;
+      kr[i] = j < n ? keys[j] : 0u;
     }
-    __syncwarp();
-    // lane L owns bins 255-8L .. 248-8L (descending)
-    uint32_t cnt[8];
-    uint32_t tot = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      cnt[e] = hist[255 - 8 * lane - e];
-      tot += cnt[e];
-    }
-    uint32_t incl = tot;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    const uint32_t excl = incl - tot;
-    const uint32_t all = __shfl_sync(0xffffffffu, incl, 31);
-    if (all < static_cast<uint32_t>(need)) {  // fewer keys than wanted (first round only)
+    if (warp_count_ge_regs(kr, 1u) <= want) {  // at most `want` candidates: take them all
       r.key = 0;
       r.ties = 0;
-      __syncwarp();
       return r;
     }
-    const bool mine = excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl;
-    const unsigned owner_mask = __ballot_sync(0xffffffffu, mine);
-    const int owner = __ffs(owner_mask) - 1;
-    int digit = 0;
-    uint32_t above = 0;
-    if (mine) {
-      uint32_t c = excl;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (c + cnt[e] >= static_cast<uint32_t>(need)) {
-          digit = 255 - 8 * lane - e;
-          above = c;
-          break;
-        }
-        c += cnt[e];
-      }
+#pragma unroll 1
+    for (int bit = 30; bit >= 0; --bit) {
+      const uint32_t c = T | (1u << bit);
+      if (warp_count_ge_regs(kr, c) >= want) T = c;
     }
-    digit = __shfl_sync(0xffffffffu, digit, owner);
-    above = __shfl_sync(0xffffffffu, above, owner);
-    need -= static_cast<int>(above);
-    prefix |= static_cast<uint32_t>(digit) << shift;
-    pmask |= 255u << shift;
-    __syncwarp();
+    r.key = T;
+    r.ties = want - warp_count_ge_regs(kr, T + 1u);
+    return r;
   }
-  r.key = prefix;
-  r.ties = prefix == 0 ? 0 : need;
+  if (warp_count_ge_smem(keys, n, 1u) <= want) {
+    r.key = 0;
+    r.ties = 0;
+    return r;
+  }
+#pragma unroll 1
+  for (int bit = 30; bit >= 0; --bit) {
+    const uint32_t c = T | (1u << bit);
+    if (warp_count_ge_smem(keys, n, c) >= want) T = c;
+  }
+  r.key = T;
+  r.ties = want - warp_count_ge_smem(keys, n, T + 1u);
   return r;
 }
 
