@@ -1,0 +1,384 @@
+// attn_tc.cuh -- exact prefill attention over the selected KV blocks on the
+// 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// MiniCPM4 summary page (端设备上的超高效大型语言模型) s2.1.3: each token attends only to
+// its most relevant KV blocks; s2.1.2: the 16 query heads of a group share them, so a
+// block is fetched once per group.
+//
+// Work item = (sequence b, kv-head g, query token t).  The item's selected blocks are
+// taken in pairs (128 keys); a persistent CTA streams pairs with TMA (128-byte swizzle,
+// no multicast) through a 3-stage ring of 64 KB (K pair, V pair) and, per pair:
+//   warp 5 (one thread) issues  S^T = K_pair . Q^T   (UMMA M128 N16 K128: keys x heads)
+//          into one of two TMEM score buffers, and, once P is in shared memory,
+//          O^T += V^T . P^T   (UMMA M128 N16 K128: V read through an MN-major
+//          descriptor, P K-major) into the item's TMEM output buffer;
+//   warps 0-3 (128 threads, thread = key of the pair) read their key's 16 head scores,
+//          keep per-head reference maxima m_h: only when a score exceeds m_h by 2^8 (one
+//          barrier-OR vote) is the pair maximum reduced across threads and O^T rescaled
+//          in TMEM; then p = exp2(s - m_h) is written to shared memory as bf16 and the
+//          per-thread partial row sums are kept in registers.  At the end of the item the
+//          same threads (now thread = output column d) divide O^T by the row sums and
+//          write O and the log-sum-exp;
+//   warp 4 is the TMA producer (query tile per item, K and V block pairs).
+#pragma once
+#include "attn.cuh"
+#include "common.cuh"
+#include "tcgen05.cuh"
+
+namespace infllmv2 {
+
+constexpr int kAtStages = 3;
+constexpr int kAtKHalf = 2 * kKvTileBytes / 2;     // 16 KB: one 64-column half of 128 keys
+constexpr int kAtStageBytes = 4 * kKvTileBytes;    // 64 KB: K pair then V pair
+constexpr int kAtPBytes = kGroupRows * 128 * 2;    // 4 KB: P (16 heads x 128 keys bf16)
+constexpr int kAtThreads = 192;
+constexpr uint32_t kAtTmemCols = 64;  // scores S[2] at 0/16, outputs O[2] at 32/48
+
+struct AtSmem {
+  uint64_t kv_full[kAtStages], kv_empty[kAtStages], q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2], pv_done[2], mma_done;
+  int n_blocks[2];
+  int list[2][kMaxTopk];
+  float red[4][kGroupRows];
+  float fin[kGroupRows];
+  float lse_out[kGroupRows];
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+constexpr size_t attn_tc_smem_bytes() {
+  return 1024 + static_cast<size_t>(kAtStages) * kAtStageBytes + 2 * kQTileBytes + 2 * kAtPBytes + sizeof(AtSmem);
+}
+
+// Per-lane result of a 32-lane max / sum over 16 values: lane L holds the total for
+// value index L >> 1 (lanes 2h and 2h+1 agree).  16 shuffles.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool up = lane & 16;
+    const float send = up ? v[i] : v[i + 8];
+    const float keep = up ? v[i + 8] : v[i];
+    a[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+  float b4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool up = lane & 8;
+    const float send = up ? a[i] : a[i + 4];
+    const float keep = up ? a[i + 4] : a[i];
+    b4[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+  float c2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool up = lane & 4;
+    const float send = up ? b4[i] : b4[i + 2];
+    const float keep = up ? b4[i + 2] : b4[i];
+    c2[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+  const bool up = lane & 2;
+  const float send = up ? c2[0] : c2[1];
+  const float keep = up ? c2[1] : c2[0];
+  const float d = op(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+  return op(d, __shfl_xor_sync(0xffffffffu, d, 1));
+}
+
+// Cross-warp (4 warps) max or sum of 16 per-thread values; every thread gets all 16.
+template <bool kMax>
+__device__ __forceinline__ void wg_reduce16(const float (&v)[16], float (&out)[16], AtSmem& S) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float r = warp_reduce16<kMax>(v);
+  if ((lane & 1) == 0) S.red[warp][lane >> 1] = r;
+  named_bar_sync(1, 128);
+#pragma unroll
+  for (int h = 0; h < kGroupRows; ++h) {
+    const float a = S.red[0][h], b = S.red[1][h], c = S.red[2][h], d = S.red[3][h];
+    out[h] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+  }
+  named_bar_sync(1, 128);  // S.red may be reused afterwards
+}
+
+// grid = min(items, SMs) persistent CTAs, block = 192.  Prefill only (p.lens == nullptr).
+__global__ void __launch_bounds__(kAtThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = align_smem(smem_raw, 1024);
+  unsigned char* stages = base;
+  unsigned char* qtiles = stages + kAtStages * kAtStageBytes;
+  unsigned char* pbufs = qtiles + 2 * kQTileBytes;
+  AtSmem& S = *reinterpret_cast<AtSmem*>(pbufs + 2 * kAtPBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAtStages; ++s) {
+      mbar_init(&S.kv_full[s], 1);
+      mbar_init(&S.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&S.q_full[s], 1);
+      mbar_init(&S.q_empty[s], 2);  // last QK of the item done + softmax warps done with the item
+      mbar_init(&S.s_full[s], 1);
+      mbar_init(&S.p_full[s], 1);
+      mbar_init(&S.pv_done[s], 1);
+    }
+    mbar_init(&S.mma_done, 1);
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&S.tmem_base, kAtTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+    }
+    uint32_t gpair = 0;
+    int it = 0;
+    for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
+      const int slot = it & 1, use = it >> 1;
+      if (use > 0) mbar_wait(&S.q_empty[slot], (use - 1) & 1, &S.abort);
+      const AttnItem a = attn_item(p, item);
+      const int cur = a.t / kBlock;
+      const int32_t* row = p.idx + ((a.bg * p.Lq + a.t) * static_cast<long long>(p.topk));
+      int count = 0;
+      for (int e0 = 0; e0 < p.topk; e0 += 32) {
+        const int e = e0 + lane;
+        const int j = e < p.topk ? row[e] : -1;
+        const bool ok = j >= 0 && j <= cur;
+        const unsigned msk = __ballot_sync(0xffffffffu, ok);
+        const int pos = count + __popc(msk & ((1u << lane) - 1u));
+        if (ok) S.list[slot][pos] = j;
+        count += __popc(msk);
+      }
+      if (lane == 0) S.n_blocks[slot] = count;
+      __threadfence_block();
+      __syncwarp();
+      const int np = (count + 1) / 2;
+      if (lane == 0) {
+        unsigned char* qs = qtiles + slot * kQTileBytes;
+        mbar_arrive_expect_tx(&S.q_full[slot], kQTileBytes);
+        tma_load_2d(qs, &tm_q, &S.q_full[slot], 0, a.qrow);
+        tma_load_2d(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow);
+        const long long kvrow0 = a.bg * p.Lmax;
+        for (int i = 0; i < np; ++i, ++gpair) {
+          const int st = static_cast<int>(gpair % kAtStages);
+          const uint32_t u = gpair / kAtStages;
+          if (u > 0) mbar_wait(&S.kv_empty[st], (u - 1) & 1, &S.abort);
+          if (S.abort) continue;
+          const int ja = S.list[slot][2 * i];
+          const int jb = 2 * i + 1 < count ? S.list[slot][2 * i + 1] : -1;
+          const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
+          const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
+          unsigned char* sk = stages + st * kAtStageBytes;
+          unsigned char* sv = sk + 2 * kAtKHalf;
+          mbar_arrive_expect_tx(&S.kv_full[st], kAtStageBytes);
+          // rows 0-63 of each 128-key half: block a; rows 64-127: block b (zeros when absent)
+          tma_load_2d(sk, &tm_k, &S.kv_full[st], 0, ra);
+          tma_load_2d(sk + kAtKHalf, &tm_k, &S.kv_full[st], 64, ra);
+          tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.kv_full[st], 0, rb);
+          tma_load_2d(sk + kAtKHalf + kKvTileBytes / 2, &tm_k, &S.kv_full[st], 64, rb);
+          tma_load_2d(sv, &tm_v, &S.kv_full[st], 0, ra);
+          tma_load_2d(sv + kAtKHalf, &tm_v, &S.kv_full[st], 64, ra);
+          tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.kv_full[st], 0, rb);
+          tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.kv_full[st], 64, rb);
+        }
+      } else {
+        gpair += np;
+      }
+      gpair = __shfl_sync(0xffffffffu, gpair, 0);
+    }
+    return;
+  }
+
+  if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kGroupRows, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kGroupRows, true, false);
+    if (lane == 0) {
+      uint32_t gp = 0;
+      int it = 0;
+      for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
+        const int slot = it & 1, use = it >> 1;
+        mbar_wait(&S.q_full[slot], use & 1, &S.abort);
+        const int np = (S.n_blocks[slot] + 1) / 2;
+        const uint32_t qa = smem_u32(qtiles + slot * kQTileBytes);
+        const uint32_t obuf = tmem + 32u + static_cast<uint32_t>(it & 1) * 16u;
+        auto issue_pv = [&](uint32_t pp, int i_in_item) {
+          mbar_wait(&S.p_full[pp & 1], (pp >> 1) & 1, &S.abort);
+          tc_fence_after();
+          const uint32_t vb = smem_u32(stages + (pp % kAtStages) * kAtStageBytes) + 2 * kAtKHalf;
+          const uint32_t pb = smem_u32(pbufs + (pp & 1) * kAtPBytes);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {  // 16 keys per step
+            umma_bf16(obuf, desc_mn_sw128(vb + k * 2048, kAtKHalf, 1024),
+                      desc_k_sw128(pb + (k >> 2) * (kAtPBytes / 2) + (k & 3) * 32), idesc_pv,
+                      (i_in_item > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&S.pv_done[pp & 1]);
+          umma_commit(&S.kv_empty[pp % kAtStages]);
+        };
+        for (int i = 0; i < np; ++i) {
+          const uint32_t pp = gp + i;
+          mbar_wait(&S.kv_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
+          if (pp >= 2) mbar_wait(&S.p_full[pp & 1], ((pp - 2) >> 1) & 1, &S.abort);  // S buffer read
+          tc_fence_after();
+          const uint32_t kb = smem_u32(stages + (pp % kAtStages) * kAtStageBytes);
+          const uint32_t sbuf = tmem + static_cast<uint32_t>(pp & 1) * 16u;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            umma_bf16(sbuf, desc_k_sw128(kb + (k >> 2) * kAtKHalf + (k & 3) * 32),
+                      desc_k_sw128(qa + (k >> 2) * (kQTileBytes / 2) + (k & 3) * 32), idesc_qk, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&S.s_full[pp & 1]);
+          if (i == np - 1) umma_commit(&S.q_empty[slot]);
+          if (i >= 1) issue_pv(pp - 1, i - 1);
+        }
+        if (np > 0) {
+          issue_pv(gp + np - 1, np - 1);
+        } else {
+          umma_commit(&S.q_empty[slot]);
+        }
+        gp += np;
+      }
+      umma_commit(&S.mma_done);
+    }
+    __syncwarp();
+    named_bar_sync(2, 160);  // the softmax warps have read TMEM for the last time
+    if (lane == 0) mbar_wait_drain(&S.mma_done, 0);  // no MMA may still write TMEM
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kAtTmemCols);
+    return;
+  }
+
+  // ---------------------------------------------------------------- softmax warps
+  const int tid = threadIdx.x;  // 0..127: key of the pair, then output column d
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+  const float sl2 = p.scale_log2;
+  uint32_t gp = 0;
+  int it = 0;
+  for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
+    const int slot = it & 1, use = it >> 1;
+    mbar_wait(&S.q_full[slot], use & 1, &S.abort);
+    const AttnItem a = attn_item(p, item);
+    const int n = S.n_blocks[slot];
+    const int np = (n + 1) / 2;
+    const uint32_t obuf = tlane + 32u + static_cast<uint32_t>(it & 1) * 16u;
+    float m[kGroupRows], l[kGroupRows];
+#pragma unroll
+    for (int h = 0; h < kGroupRows; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+    }
+    for (int i = 0; i < np; ++i) {
+      const uint32_t pp = gp + i;
+      mbar_wait(&S.s_full[pp & 1], (pp >> 1) & 1, &S.abort);
+      tc_fence_after();
+      uint32_t sv[16];
+      tmem_ld16(tlane + static_cast<uint32_t>(pp & 1) * 16u, sv);
+      const int bi = 2 * i + (tid >> 6);
+      const int blk = bi < n ? S.list[slot][bi] : -1;
+      const int key = blk * kBlock + (tid & 63);
+      const bool valid = blk >= 0 && key <= a.t;
+      float x[kGroupRows];
+      bool viol = false;
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) {
+        x[h] = valid ? __uint_as_float(sv[h]) * sl2 : -INFINITY;
+        viol |= x[h] > m[h] + 8.f;
+      }
+      if (named_bar_or(1, 128, viol)) {
+        // a score rose more than 2^8 above its reference: move the references to the
+        // pair maxima and rescale what was accumulated so far
+        float mx[kGroupRows];
+        wg_reduce16<true>(x, mx, S);
+        float al[kGroupRows];
+#pragma unroll
+        for (int h = 0; h < kGroupRows; ++h) {
+          const float mn = fmaxf(m[h], mx[h]);
+          al[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
+          l[h] *= al[h];
+          m[h] = mn;
+        }
+        if (i >= 1) {
+          mbar_wait(&S.pv_done[(pp - 1) & 1], ((pp - 1) >> 1) & 1, &S.abort);
+          tc_fence_after();
+          uint32_t ov[16];
+          tmem_ld16(obuf, ov);
+#pragma unroll
+          for (int h = 0; h < kGroupRows; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * al[h]);
+          tmem_st16(obuf, ov);
+        }
+      }
+      float pv[kGroupRows];
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) {
+        pv[h] = (m[h] == -INFINITY) ? 0.f : ex2(x[h] - m[h]);
+        l[h] += pv[h];
+      }
+      if (pp >= 2) mbar_wait(&S.pv_done[pp & 1], ((pp - 2) >> 1) & 1, &S.abort);  // P buffer free
+      {
+        unsigned char* pbuf = pbufs + (pp & 1) * kAtPBytes + (tid >> 6) * (kAtPBytes / 2);
+        const int col = tid & 63;
+#pragma unroll
+        for (int h = 0; h < kGroupRows; ++h) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(pv[h]);
+          *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128(h, col >> 3) + (col & 7) * 2) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, 128);
+      if (tid == 0) mbar_arrive(&S.p_full[pp & 1]);
+    }
+
+    // ---- end of item: normalise O^T (thread = column d) and write O and lse
+    float L[kGroupRows];
+    wg_reduce16<false>(l, L, S);
+    float ov_f[kGroupRows];
+    if (np > 0) {
+      const uint32_t last = gp + np - 1;
+      mbar_wait(&S.pv_done[last & 1], (last >> 1) & 1, &S.abort);
+      tc_fence_after();
+      uint32_t ov[16];
+      tmem_ld16(obuf, ov);
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) ov_f[h] = L[h] > 0.f ? __uint_as_float(ov[h]) / L[h] : 0.f;
+    } else {
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) ov_f[h] = 0.f;
+    }
+#pragma unroll
+    for (int h = 0; h < kGroupRows; ++h)
+      if (h < p.G) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(ov_f[h]);
+    if (tid == 0) {
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h)
+        S.lse_out[h] = L[h] > 0.f ? (m[h] + lg2(L[h])) * 0.6931471805599453f : -INFINITY;
+    }
+    tc_fence_before();
+    named_bar_sync(1, 128);
+    if (p.lse != nullptr && tid < p.G)
+      p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.t] = S.lse_out[tid];
+    if (tid == 0) mbar_arrive(&S.q_empty[slot]);
+    named_bar_sync(1, 128);  // S.lse_out reuse
+    gp += np;
+  }
+  named_bar_sync(2, 160);  // TMEM may be freed
+}
+
+}  // namespace infllmv2

@@ -12,6 +12,7 @@
 
 #include "../../include/infllmv2.h"
 #include "attn.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "select_decode.cuh"
@@ -362,9 +363,22 @@ int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const 
   a.lse = lse;
   a.part_o = nullptr;
   a.part_lse = nullptr;
-  return launch_attn(p, q, static_cast<uint64_t>(p->batch) * L * p->num_q_heads, k, v,
-                     static_cast<uint64_t>(p->batch) * p->num_kv_heads * L, a,
-                     reinterpret_cast<cudaStream_t>(stream));
+  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * L * p->num_q_heads;
+  const uint64_t kv_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * L;
+  if (a.G == kGroupRows) {
+    // tensor-core path: per item, K/V block pairs against the group's 16 query rows
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
+        !make_map(&tv, v, kv_rows, kBlock))
+      return INFLLMV2_ERR_CUDA;
+    const size_t smem = attn_tc_smem_bytes();
+    if ((st = set_smem(reinterpret_cast<const void*>(attn_tc_kernel), smem)) != INFLLMV2_OK) return st;
+    const long long grid = std::min<long long>(a.num_items, num_sms());
+    attn_tc_kernel<<<static_cast<unsigned>(grid), kAtThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        tq, tk, tv, a);
+    return launch_status();
+  }
+  return launch_attn(p, q, q_rows, k, v, kv_rows, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,

@@ -203,8 +203,12 @@ __global__ void __launch_bounds__(kDecTopkThreads) select_decode_topk_kernel(con
   __syncthreads();
   if (threadIdx.x < 32) {
     const int want = p.topk - forced_count(cur, p.n_init, p.n_local);
-    const TopkThreshold th = warp_radix_threshold(keys, cur + 1, want, hist);
-    warp_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out);
+    if (cur + 1 <= 32 * kTopkRegKeys) {
+      warp_topk_select(keys, cur + 1, want, cur, p.n_init, p.n_local, p.topk, hist, out);
+    } else {
+      const TopkThreshold th = warp_radix_threshold(keys, cur + 1, want, hist);
+      warp_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out);
+    }
   }
 }
 

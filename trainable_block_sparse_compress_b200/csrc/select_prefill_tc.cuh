@@ -6,19 +6,19 @@
 // block, sum over the group's heads, top-k with forced initial/local blocks.
 //
 // One CTA = 8 consecutive query tokens of one (sequence, kv-head): 8 x 16 heads = the 128
-// rows (M) of a UMMA tile.  Warp roles (320 threads):
-//   warp 8  TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then Kc tiles
+// rows (M) of a UMMA tile.  Warp roles (448 threads):
+//   warp 12 TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then Kc tiles
 //           through a 3-stage ring: pass A tiles of 128 kernels, pass B tiles of 144
 //           kernels that start 16 kernels early, so each pass-B tile also holds the
 //           kernel straddling its first block (4j - 1) and is self-contained;
-//   warp 9  allocates TMEM and, from one thread, issues per tile 8 UMMAs (M128 x N128 or
-//           N144, K16, bf16 -> fp32) into one of two TMEM accumulators;
-//   warps 0-7  two epilogue warpgroups taking alternate tiles; thread (w, lane) owns TMEM
+//   warp 13 allocates TMEM and, from one thread, issues per tile 8 UMMAs (M128 x N128 or
+//           N144, K16, bf16 -> fp32) into one of three TMEM accumulators;
+//   warps 0-11 three epilogue warpgroups taking every third tile; thread (w, lane) owns TMEM
 //           lane 32 (w % 4) + lane = row (token, head).  Pass A keeps an online
-//           log-sum-exp per row (the two warpgroups' partials are merged once); pass B
+//           log-sum-exp per row (the warpgroups' partials are merged once); pass B
 //           pools block maxima along the row, forms p = exp(m - lse) and sums the 16
 //           heads of a token with a 16-lane transpose-reduce; block keys go to shared
-//           memory; finally warp w radix-selects the top blocks of token w.
+//           memory; finally warp w < 8 selects the top blocks of token w.
 #pragma once
 #include "common.cuh"
 #include "select_prefill.cuh"
@@ -35,21 +35,23 @@ constexpr int kTcStages = 3;
 constexpr int kTcHalfBytes = kTcNB * 128;   // one 64-column half of a stage (144 rows x 128 B)
 constexpr int kTcStageBytes = 2 * kTcHalfBytes;
 constexpr int kTcQBytes = 128 * kHeadDim * 2;  // 32 KB
-constexpr int kTcEpiWarps = 8;
+constexpr int kTcEpiWGs = 3;              // epilogue warpgroups = TMEM accumulators
+constexpr int kTcEpiWarps = 4 * kTcEpiWGs;
 constexpr int kTcThreads = 32 * (kTcEpiWarps + 2);
 constexpr uint32_t kTcTmemCols = 512;
-constexpr uint32_t kTcAccStride = 256;  // TMEM column offset between the two accumulators
+constexpr uint32_t kTcAccStride = 160;
+static_assert(kTcAccStride >= kTcNB && (kTcEpiWGs - 1) * kTcAccStride + kTcNB <= kTcTmemCols, "TMEM plan");  // TMEM column offset between accumulators (>= 144)
 
 struct SelTcSmem {
-  uint64_t qbar, full[kTcStages], empty[kTcStages], tfull[2], tempty[2], mma_done;
-  float2 part[2][128];  // pass-A (max, sum) per warpgroup and row
+  uint64_t qbar, full[kTcStages], empty[kTcStages], tfull[kTcEpiWGs], tempty[kTcEpiWGs], mma_done;
+  float2 part[kTcEpiWGs][128];  // pass-A (max, sum) per warpgroup and row
   uint32_t tmem_base;
   volatile int abort;
 };
 
 inline size_t sel_tc_smem_bytes(int nblk_cap) {
   return 1024 + kTcQBytes + static_cast<size_t>(kTcStages) * kTcStageBytes +
-         static_cast<size_t>(kTcTokens) * nblk_cap * 4 + kTcEpiWarps * 256 * 4 + sizeof(SelTcSmem);
+         static_cast<size_t>(kTcTokens) * nblk_cap * 4 + kTcTokens * 256 * 4 + sizeof(SelTcSmem);
 }
 
 // Sum of v over the 16 lanes that share lane bit 4 (one token's heads), scattered: lane
@@ -94,7 +96,7 @@ __device__ __forceinline__ float reduce_scatter16(const float (&v)[16]) {
 
 __device__ __forceinline__ float max4(float a, float b, float c, float d) { return fmaxf(fmaxf(a, b), fmaxf(c, d)); }
 
-// grid = B * Hkv * ceil(L / 8) (latest tiles first), block = 320.  Requires G == 16.
+// grid = B * Hkv * ceil(L / 8) (latest tiles first), block = 448.  Requires G == 16.
 __global__ void __launch_bounds__(kTcThreads, 1)
     select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q3, const __grid_constant__ CUtensorMap tm_kca,
                              const __grid_constant__ CUtensorMap tm_kcb, const SelPrefillParams p) {
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   unsigned char* ring = qs + kTcQBytes;
   uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + kTcStages * kTcStageBytes);
   uint32_t* hist_all = keys_all + kTcTokens * p.nblk_cap;
-  SelTcSmem& S = *reinterpret_cast<SelTcSmem*>(hist_all + kTcEpiWarps * 256);
+  SelTcSmem& S = *reinterpret_cast<SelTcSmem*>(hist_all + kTcTokens * 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long nbg = static_cast<long long>(p.B) * p.Hkv;
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kTcEpiWGs; ++a) {
       mbar_init(&S.tfull[a], 1);
       mbar_init(&S.tempty[a], 4);  // the four warps of the warpgroup that owns accumulator a
     }
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait(&S.qbar, 0, &S.abort);
       const uint32_t qa = smem_u32(qs);
       for (int n = 0; n < T; ++n) {
-        const int st = n % kTcStages, acc = n & 1, u = n >> 1;
+        const int st = n % kTcStages, acc = n % kTcEpiWGs, u = n / kTcEpiWGs;
         mbar_wait(&S.full[st], (n / kTcStages) & 1, &S.abort);
         if (u > 0) mbar_wait(&S.tempty[acc], (u - 1) & 1, &S.abort);
         tc_fence_after();
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ---------------------------------------------------------------- epilogue warps
-  const int wg = warp >> 2;   // warpgroup: takes tiles n with n % 2 == wg
+  const int wg = warp >> 2;   // warpgroup: takes tiles n with n % kTcEpiWGs == wg
   const int wq = warp & 3;    // TMEM lane quarter
   const int row = 32 * wq + lane;
   const int tok = row >> 4;
@@ -215,13 +217,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int imax = last_visible_kernel(t);
   const int cur = t / kBlock;
   const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
-  const float sl2 = p.scale_log2;
+  const float sl2 = p.scale_log2;  // > 0: maxima of raw logits scale to maxima of scaled ones
 
-  // pass A: log-sum-exp of this row over its visible kernels (base 2), alternate tiles
+  // pass A: log-sum-exp of this row over its visible kernels (base 2), every third tile
   float m = -INFINITY, l = 0.f;
-  for (int n = wg; n < TA; n += 2) {
-    const int acc = n & 1;
-    mbar_wait(&S.tfull[acc], (n >> 1) & 1, &S.abort);
+  for (int n = wg; n < TA; n += kTcEpiWGs) {
+    const int acc = n % kTcEpiWGs;
+    mbar_wait(&S.tfull[acc], (n / kTcEpiWGs) & 1, &S.abort);
     tc_fence_after();
 #pragma unroll 1
     for (int q = 0; q < kTcN / 32; ++q) {
@@ -231,21 +233,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float x[32];
       if (i0 + 31 <= imax) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]) * sl2;
+        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
+        for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) : -INFINITY;
       }
       float c8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) c8[e] = max4(x[e], x[e + 8], x[e + 16], x[e + 24]);
-      const float cm = fmaxf(max4(c8[0], c8[1], c8[2], c8[3]), max4(c8[4], c8[5], c8[6], c8[7]));
+      const float cm = fmaxf(max4(c8[0], c8[1], c8[2], c8[3]), max4(c8[4], c8[5], c8[6], c8[7])) * sl2;
       if (cm != -INFINITY) {
         const float mn = fmaxf(m, cm);
         float s8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          s8[e] = (ex2(x[e] - mn) + ex2(x[e + 8] - mn)) + (ex2(x[e + 16] - mn) + ex2(x[e + 24] - mn));
+          s8[e] = (ex2(fmaf(x[e], sl2, -mn)) + ex2(fmaf(x[e + 8], sl2, -mn))) +
+                  (ex2(fmaf(x[e + 16], sl2, -mn)) + ex2(fmaf(x[e + 24], sl2, -mn)));
         const float s = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
         l = l * ex2(m - mn) + s;
         m = mn;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) mbar_arrive(&S.tempty[acc]);
   }
   // zero the key row of token `warp` (blocks 0..cur) while the warpgroups meet
-  {
+  if (warp < kTcTokens) {
     const int tz = min(t0 + warp, p.L - 1);
     uint32_t* kz = keys_all + warp * p.nblk_cap;
     for (int j = lane; j <= tz / kBlock; j += 32) kz[j] = 0u;
@@ -265,44 +268,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   named_bar_sync(2, 32 * kTcEpiWarps);
   float lse;
   {
-    const float2 a0 = S.part[0][row], a1 = S.part[1][row];
-    const float M = fmaxf(a0.x, a1.x);
-    const float L = (M == -INFINITY) ? 0.f : a0.y * ex2(a0.x - M) + a1.y * ex2(a1.x - M);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kTcEpiWGs; ++w) M = fmaxf(M, S.part[w][row].x);
+    float L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kTcEpiWGs; ++w) L += S.part[w][row].y * ex2(S.part[w][row].x - M);
+    }
     lse = L > 0.f ? M + lg2(L) : INFINITY;
   }
 
   // pass B: block maxima along the row, p = exp(m - lse), group sum over the 16 heads
   uint32_t* keys = keys_all + tok * p.nblk_cap;
-  for (int n = TA + ((TA & 1) != wg ? 1 : 0); n < T; n += 2) {
+  int nb = TA;
+  while (nb % kTcEpiWGs != wg) ++nb;
+  for (int n = nb; n < T; n += kTcEpiWGs) {
     const int c = n - TA;
-    const int acc = n & 1;
-    mbar_wait(&S.tfull[acc], (n >> 1) & 1, &S.abort);
+    const int acc = n % kTcEpiWGs;
+    mbar_wait(&S.tfull[acc], (n / kTcEpiWGs) & 1, &S.abort);
     tc_fence_after();
     const uint32_t tacc = trow + static_cast<uint32_t>(acc) * kTcAccStride;
     // column kTcOverlap-1 holds kernel 128c - 1, the straddle of block 32c
     // (tcgen05.ld is warp-collective: load unconditionally, then mask)
     const int istr = c * kTcN - 1;
     const float cv = __uint_as_float(tmem_ld1(tacc + kTcOverlap - 1));
-    float carry = (istr >= 0 && istr <= imax) ? cv * sl2 : -INFINITY;
+    float carry = (istr >= 0 && istr <= imax) ? cv : -INFINITY;  // raw logit
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       float pb[16];
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {
-        const int q = 2 * half + q2;
         uint32_t v[32];
-        tmem_ld32(tacc + static_cast<uint32_t>(kTcOverlap + 32 * q), v);
-        const int i0 = c * kTcN + 32 * q;
+        tmem_ld32(tacc + static_cast<uint32_t>(kTcOverlap + 64 * half + 32 * q2), v);
+        const int i0 = c * kTcN + 64 * half + 32 * q2;
         float x[32];
+        if (i0 + 31 <= imax) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) * sl2 : -INFINITY;
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(v[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = (i0 + e <= imax) ? __uint_as_float(v[e]) : -INFINITY;
+        }
 #pragma unroll
         for (int gq = 0; gq < 8; ++gq) {
-          const float mb = fmaxf(max4(x[4 * gq], x[4 * gq + 1], x[4 * gq + 2], x[4 * gq + 3]),
-                                 gq == 0 ? carry : x[4 * gq - 1]);
-          pb[8 * q2 + gq] = ex2(mb - lse);
+          const float mb = fmaxf(max4(x[4 * gq], x[4 * gq + 1], x[4 * gq + 2], x[4 * gq + 3]), carry);
+          pb[8 * q2 + gq] = ex2(fmaf(mb, sl2, -lse));
+          carry = x[4 * gq + 3];
         }
-        carry = x[31];
       }
       const float sum = reduce_scatter16(pb);
       const int j = 32 * c + 16 * half + (lane & 15);
@@ -317,18 +330,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) mbar_arrive(&S.tempty[acc]);
   }
   tc_fence_before();
-  named_bar_sync(1, 32 * (kTcEpiWarps + 1));  // TMEM no longer read: warp 9 may free it
+  named_bar_sync(1, 32 * (kTcEpiWarps + 1));  // TMEM no longer read: the MMA warp may free it
   named_bar_sync(2, 32 * kTcEpiWarps);        // all keys written
 
   // top-k of token `warp`
   const int tr = t0 + warp;
-  if (tr < p.L) {
+  if (warp < kTcTokens && tr < p.L) {
     const int cu = tr / kBlock;
     const uint32_t* kt = keys_all + warp * p.nblk_cap;
     const int want = p.topk - forced_count(cu, p.n_init, p.n_local);
-    const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + warp * 256);
     int32_t* out = p.idx + ((bg * p.L + tr) * static_cast<long long>(p.topk));
-    warp_emit_selection(kt, cu + 1, th, cu, p.n_init, p.n_local, p.topk, out);
+    if (cu + 1 <= 32 * kTopkRegKeys) {
+      warp_topk_select(kt, cu + 1, want, cu, p.n_init, p.n_local, p.topk, hist_all + warp * 256, out);
+    } else {
+      const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + warp * 256);
+      warp_emit_selection(kt, cu + 1, th, cu, p.n_init, p.n_local, p.topk, out);
+    }
   }
 }
 
