@@ -6,20 +6,26 @@
 // block is fetched once per group.
 //
 // Work item = (sequence b, kv-head g, query token t).  The item's selected blocks are
-// taken in pairs (128 keys); a persistent CTA streams pairs with TMA (128-byte swizzle,
-// no multicast) through a 3-stage ring of 64 KB (K pair, V pair) and, per pair:
-//   warp 5 (one thread) issues  S^T = K_pair . Q^T   (UMMA M128 N16 K128: keys x heads)
-//          into one of two TMEM score buffers, and, once P is in shared memory,
+// taken in pairs (128 keys); a persistent CTA streams them with TMA (128-byte swizzle, no
+// multicast) through two 3-slot rings of 32 KB, one for K pairs (warp 8) and one for V
+// pairs (warp 11), so a K slot is free again right after its QK and a V slot right
+// after its PV; per pair:
+//   warp 9 (one thread) issues  S^T = K_pair . Q^T   (UMMA M128 N16 K128: keys x heads)
+//          into one of two TMEM score buffers as soon as the pair has landed;
+//   warp 10 (one thread) issues, as soon as P is in shared memory,
 //          O^T += V^T . P^T   (UMMA M128 N16 K128: V read through an MN-major
-//          descriptor, P K-major) into the item's TMEM output buffer;
-//   warps 0-3 (128 threads, thread = key of the pair) read their key's 16 head scores,
-//          keep per-head reference maxima m_h: only when a score exceeds m_h by 2^8 (one
-//          barrier-OR vote) is the pair maximum reduced across threads and O^T rescaled
-//          in TMEM; then p = exp2(s - m_h) is written to shared memory as bf16 and the
-//          per-thread partial row sums are kept in registers.  At the end of the item the
-//          same threads (now thread = output column d) divide O^T by the row sums and
-//          write O and the log-sum-exp;
-//   warp 4 is the TMA producer (query tile per item, K and V block pairs).
+//          descriptor, P K-major) into the TMEM output buffer of the pair's warpgroup.
+//          Two issuers keep a PV from waiting behind the next pair's loads;
+//   warps 0-7: two softmax warpgroups take alternate pairs (128 threads each, thread =
+//          key of the pair), each with its own TMEM output buffer, reference maxima and
+//          row sums (a split over the pairs inside the CTA).  A thread reads its key's 16
+//          head scores; only when a score exceeds the warpgroup's reference m_h by 2^8
+//          (one barrier-OR vote) is the pair maximum reduced across threads and that
+//          O^T rescaled in TMEM; p = exp2(s - m_h) goes to shared memory as bf16 and the
+//          partial row sums stay in registers.  At the end of the item the two partial
+//          states are merged (thread = output column d) and O and the log-sum-exp are
+//          written;
+//   warp 8 also loads the query tile and compacts the block list of each item.
 #pragma once
 #include "attn.cuh"
 #include "common.cuh"
@@ -27,27 +33,33 @@
 
 namespace infllmv2 {
 
-constexpr int kAtStages = 3;
+constexpr int kAtStages = 3;                       // slots per ring (K ring and V ring)
 constexpr int kAtKHalf = 2 * kKvTileBytes / 2;     // 16 KB: one 64-column half of 128 keys
-constexpr int kAtStageBytes = 4 * kKvTileBytes;    // 64 KB: K pair then V pair
+constexpr int kAtSlotBytes = 2 * kKvTileBytes;     // 32 KB: a pair of K (or V) blocks
 constexpr int kAtPBytes = kGroupRows * 128 * 2;    // 4 KB: P (16 heads x 128 keys bf16)
-constexpr int kAtThreads = 192;
-constexpr uint32_t kAtTmemCols = 64;  // scores S[2] at 0/16, outputs O[2] at 32/48
+constexpr int kAtSoftWGs = 2;
+constexpr int kAtThreads = 32 * (4 * kAtSoftWGs + 4);
+constexpr int kAtTmaWarp = 4 * kAtSoftWGs, kAtMmaWarp = kAtTmaWarp + 1, kAtPvWarp = kAtTmaWarp + 2,
+              kAtVTmaWarp = kAtTmaWarp + 3;
+constexpr int kAtBufs = 4;             // score (TMEM) and probability (shared) buffers in flight
+constexpr uint32_t kAtTmemCols = 128;  // scores S[4] at 16 s; outputs O[item parity][wg] at 64 + 16 (2 it + wg)
+constexpr uint32_t kAtOCol = 16 * kAtBufs;
 
 struct AtSmem {
-  uint64_t kv_full[kAtStages], kv_empty[kAtStages], q_full[2], q_empty[2];
-  uint64_t s_full[2], p_full[2], pv_done[2], mma_done;
+  uint64_t k_full[kAtStages], k_empty[kAtStages], v_full[kAtStages], v_empty[kAtStages], q_full[2], q_empty[2];
+  uint64_t s_full[kAtBufs], p_full[kAtBufs], pv_done[kAtBufs], mma_done[2];
   int n_blocks[2];
   int list[2][kMaxTopk];
-  float red[4][kGroupRows];
-  float fin[kGroupRows];
+  float red[kAtSoftWGs][4][kGroupRows];
+  float mstate[kAtSoftWGs][kGroupRows], lstate[kAtSoftWGs][kGroupRows];
   float lse_out[kGroupRows];
   uint32_t tmem_base;
   volatile int abort;
 };
 
 constexpr size_t attn_tc_smem_bytes() {
-  return 1024 + static_cast<size_t>(kAtStages) * kAtStageBytes + 2 * kQTileBytes + 2 * kAtPBytes + sizeof(AtSmem);
+  return 1024 + 2 * static_cast<size_t>(kAtStages) * kAtSlotBytes + 2 * kQTileBytes + kAtBufs * kAtPBytes +
+         sizeof(AtSmem);
 }
 
 // Per-lane result of a 32-lane max / sum over 16 values: lane L holds the total for
@@ -89,48 +101,54 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
 
 // Cross-warp (4 warps) max or sum of 16 per-thread values; every thread gets all 16.
 template <bool kMax>
-__device__ __forceinline__ void wg_reduce16(const float (&v)[16], float (&out)[16], AtSmem& S) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void wg_reduce16(const float (&v)[16], float (&out)[16], AtSmem& S, int wg) {
+  const int wq = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
   const float r = warp_reduce16<kMax>(v);
-  if ((lane & 1) == 0) S.red[warp][lane >> 1] = r;
-  named_bar_sync(1, 128);
+  if ((lane & 1) == 0) S.red[wg][wq][lane >> 1] = r;
+  named_bar_sync(1 + wg, 128);
 #pragma unroll
   for (int h = 0; h < kGroupRows; ++h) {
-    const float a = S.red[0][h], b = S.red[1][h], c = S.red[2][h], d = S.red[3][h];
+    const float a = S.red[wg][0][h], b = S.red[wg][1][h], c = S.red[wg][2][h], d = S.red[wg][3][h];
     out[h] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
   }
-  named_bar_sync(1, 128);  // S.red may be reused afterwards
+  named_bar_sync(1 + wg, 128);  // S.red may be reused afterwards
 }
 
-// grid = min(items, SMs) persistent CTAs, block = 192.  Prefill only (p.lens == nullptr).
+// grid = min(items, SMs) persistent CTAs, block = 384.  Prefill only (p.lens == nullptr).
 __global__ void __launch_bounds__(kAtThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = align_smem(smem_raw, 1024);
-  unsigned char* stages = base;
-  unsigned char* qtiles = stages + kAtStages * kAtStageBytes;
+  unsigned char* kring = base;
+  unsigned char* vring = kring + kAtStages * kAtSlotBytes;
+  unsigned char* qtiles = vring + kAtStages * kAtSlotBytes;
   unsigned char* pbufs = qtiles + 2 * kQTileBytes;
-  AtSmem& S = *reinterpret_cast<AtSmem*>(pbufs + 2 * kAtPBytes);
+  AtSmem& S = *reinterpret_cast<AtSmem*>(pbufs + kAtBufs * kAtPBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAtStages; ++s) {
-      mbar_init(&S.kv_full[s], 1);
-      mbar_init(&S.kv_empty[s], 1);
+      mbar_init(&S.k_full[s], 1);
+      mbar_init(&S.k_empty[s], 1);
+      mbar_init(&S.v_full[s], 1);
+      mbar_init(&S.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&S.q_full[s], 1);
-      mbar_init(&S.q_empty[s], 2);  // last QK of the item done + softmax warps done with the item
+      mbar_init(&S.q_empty[s], 3);  // last QK done + V producer and softmax warps done with the item
+    }
+    for (int s = 0; s < kAtBufs; ++s) {
       mbar_init(&S.s_full[s], 1);
       mbar_init(&S.p_full[s], 1);
       mbar_init(&S.pv_done[s], 1);
     }
-    mbar_init(&S.mma_done, 1);
+    mbar_init(&S.mma_done[0], 1);
+    mbar_init(&S.mma_done[1], 1);
     S.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kAtMmaWarp) {
     tmem_alloc(&S.tmem_base, kAtTmemCols);
     tmem_relinquish();
   }
@@ -139,7 +157,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kAtTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -177,24 +195,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int i = 0; i < np; ++i, ++gpair) {
           const int st = static_cast<int>(gpair % kAtStages);
           const uint32_t u = gpair / kAtStages;
-          if (u > 0) mbar_wait(&S.kv_empty[st], (u - 1) & 1, &S.abort);
+          if (u > 0) mbar_wait(&S.k_empty[st], (u - 1) & 1, &S.abort);
           if (S.abort) continue;
           const int ja = S.list[slot][2 * i];
           const int jb = 2 * i + 1 < count ? S.list[slot][2 * i + 1] : -1;
           const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
           const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
-          unsigned char* sk = stages + st * kAtStageBytes;
-          unsigned char* sv = sk + 2 * kAtKHalf;
-          mbar_arrive_expect_tx(&S.kv_full[st], kAtStageBytes);
+          unsigned char* sk = kring + st * kAtSlotBytes;
+          mbar_arrive_expect_tx(&S.k_full[st], kAtSlotBytes);
           // rows 0-63 of each 128-key half: block a; rows 64-127: block b (zeros when absent)
-          tma_load_2d(sk, &tm_k, &S.kv_full[st], 0, ra);
-          tma_load_2d(sk + kAtKHalf, &tm_k, &S.kv_full[st], 64, ra);
-          tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.kv_full[st], 0, rb);
-          tma_load_2d(sk + kAtKHalf + kKvTileBytes / 2, &tm_k, &S.kv_full[st], 64, rb);
-          tma_load_2d(sv, &tm_v, &S.kv_full[st], 0, ra);
-          tma_load_2d(sv + kAtKHalf, &tm_v, &S.kv_full[st], 64, ra);
-          tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.kv_full[st], 0, rb);
-          tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.kv_full[st], 64, rb);
+          tma_load_2d(sk, &tm_k, &S.k_full[st], 0, ra);
+          tma_load_2d(sk + kAtKHalf, &tm_k, &S.k_full[st], 64, ra);
+          tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.k_full[st], 0, rb);
+          tma_load_2d(sk + kAtKHalf + kKvTileBytes / 2, &tm_k, &S.k_full[st], 64, rb);
         }
       } else {
         gpair += np;
@@ -204,8 +217,45 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     return;
   }
 
-  if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  if (warp == kAtVTmaWarp) {
+    // ------------------------------------------------------------ V producer
+    // V pairs are loaded through their own ring, so a V slot is held only until its PV,
+    // and K slots recycle right after their QK.
+    if (lane == 0) {
+      uint32_t gpair = 0;
+      int it = 0;
+      for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
+        const int slot = it & 1, use = it >> 1;
+        mbar_wait(&S.q_full[slot], use & 1, &S.abort);  // the item's block list is ready
+        const AttnItem a = attn_item(p, item);
+        const int count = S.n_blocks[slot];
+        const int np = (count + 1) / 2;
+        const long long kvrow0 = a.bg * p.Lmax;
+        for (int i = 0; i < np; ++i, ++gpair) {
+          const int st = static_cast<int>(gpair % kAtStages);
+          const uint32_t u = gpair / kAtStages;
+          if (u > 0) mbar_wait(&S.v_empty[st], (u - 1) & 1, &S.abort);
+          if (S.abort) continue;
+          const int ja = S.list[slot][2 * i];
+          const int jb = 2 * i + 1 < count ? S.list[slot][2 * i + 1] : -1;
+          const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
+          const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
+          unsigned char* sv = vring + st * kAtSlotBytes;
+          mbar_arrive_expect_tx(&S.v_full[st], kAtSlotBytes);
+          tma_load_2d(sv, &tm_v, &S.v_full[st], 0, ra);
+          tma_load_2d(sv + kAtKHalf, &tm_v, &S.v_full[st], 64, ra);
+          tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.v_full[st], 0, rb);
+          tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.v_full[st], 64, rb);
+        }
+        mbar_arrive(&S.q_empty[slot]);  // done with the item's block list
+      }
+    }
+    return;
+  }
+
+  if (warp == kAtMmaWarp || warp == kAtPvWarp) {
+    // ------------------------------------------------------- MMA issuers (QK / PV)
+    const bool is_qk = warp == kAtMmaWarp;
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kGroupRows, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kGroupRows, true, false);
     if (lane == 0) {
@@ -215,59 +265,65 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const int slot = it & 1, use = it >> 1;
         mbar_wait(&S.q_full[slot], use & 1, &S.abort);
         const int np = (S.n_blocks[slot] + 1) / 2;
-        const uint32_t qa = smem_u32(qtiles + slot * kQTileBytes);
-        const uint32_t obuf = tmem + 32u + static_cast<uint32_t>(it & 1) * 16u;
-        auto issue_pv = [&](uint32_t pp, int i_in_item) {
-          mbar_wait(&S.p_full[pp & 1], (pp >> 1) & 1, &S.abort);
-          tc_fence_after();
-          const uint32_t vb = smem_u32(stages + (pp % kAtStages) * kAtStageBytes) + 2 * kAtKHalf;
-          const uint32_t pb = smem_u32(pbufs + (pp & 1) * kAtPBytes);
+        if (is_qk) {
+          const uint32_t qa = smem_u32(qtiles + slot * kQTileBytes);
+          for (int i = 0; i < np; ++i) {
+            const uint32_t pp = gp + i;
+            mbar_wait(&S.k_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
+            if (pp >= kAtBufs) mbar_wait(&S.p_full[pp % kAtBufs], ((pp / kAtBufs) - 1) & 1, &S.abort);  // S read
+            tc_fence_after();
+            const uint32_t kb = smem_u32(kring + (pp % kAtStages) * kAtSlotBytes);
+            const uint32_t sbuf = tmem + static_cast<uint32_t>(pp % kAtBufs) * 16u;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {  // 16 keys per step
-            umma_bf16(obuf, desc_mn_sw128(vb + k * 2048, kAtKHalf, 1024),
-                      desc_k_sw128(pb + (k >> 2) * (kAtPBytes / 2) + (k & 3) * 32), idesc_pv,
-                      (i_in_item > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 8; ++k) {
+              umma_bf16(sbuf, desc_k_sw128(kb + (k >> 2) * kAtKHalf + (k & 3) * 32),
+                        desc_k_sw128(qa + (k >> 2) * (kQTileBytes / 2) + (k & 3) * 32), idesc_qk,
+                        k > 0 ? 1u : 0u);
+            }
+            umma_commit(&S.s_full[pp % kAtBufs]);
+            umma_commit(&S.k_empty[pp % kAtStages]);
           }
-          umma_commit(&S.pv_done[pp & 1]);
-          umma_commit(&S.kv_empty[pp % kAtStages]);
-        };
-        for (int i = 0; i < np; ++i) {
-          const uint32_t pp = gp + i;
-          mbar_wait(&S.kv_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
-          if (pp >= 2) mbar_wait(&S.p_full[pp & 1], ((pp - 2) >> 1) & 1, &S.abort);  // S buffer read
-          tc_fence_after();
-          const uint32_t kb = smem_u32(stages + (pp % kAtStages) * kAtStageBytes);
-          const uint32_t sbuf = tmem + static_cast<uint32_t>(pp & 1) * 16u;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            umma_bf16(sbuf, desc_k_sw128(kb + (k >> 2) * kAtKHalf + (k & 3) * 32),
-                      desc_k_sw128(qa + (k >> 2) * (kQTileBytes / 2) + (k & 3) * 32), idesc_qk, k > 0 ? 1u : 0u);
-          }
-          umma_commit(&S.s_full[pp & 1]);
-          if (i == np - 1) umma_commit(&S.q_empty[slot]);
-          if (i >= 1) issue_pv(pp - 1, i - 1);
-        }
-        if (np > 0) {
-          issue_pv(gp + np - 1, np - 1);
+          umma_commit(&S.q_empty[slot]);  // the item's query tile is no longer read
         } else {
-          umma_commit(&S.q_empty[slot]);
+          for (int i = 0; i < np; ++i) {
+            const uint32_t pp = gp + i;
+            mbar_wait(&S.p_full[pp % kAtBufs], (pp / kAtBufs) & 1, &S.abort);
+            mbar_wait(&S.v_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
+            tc_fence_after();
+            const uint32_t obuf = tmem + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + (pp & 1)) * 16u;
+            const uint32_t vb = smem_u32(vring + (pp % kAtStages) * kAtSlotBytes);
+            const uint32_t pb = smem_u32(pbufs + (pp % kAtBufs) * kAtPBytes);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // 16 keys per step
+              umma_bf16(obuf, desc_mn_sw128(vb + k * 2048, kAtKHalf, 1024),
+                        desc_k_sw128(pb + (k >> 2) * (kAtPBytes / 2) + (k & 3) * 32), idesc_pv,
+                        (i >= kAtSoftWGs || k > 0) ? 1u : 0u);
+            }
+            umma_commit(&S.pv_done[pp % kAtBufs]);
+            umma_commit(&S.v_empty[pp % kAtStages]);
+          }
         }
         gp += np;
       }
-      umma_commit(&S.mma_done);
+      umma_commit(&S.mma_done[is_qk ? 0 : 1]);
     }
     __syncwarp();
-    named_bar_sync(2, 160);  // the softmax warps have read TMEM for the last time
-    if (lane == 0) mbar_wait_drain(&S.mma_done, 0);  // no MMA may still write TMEM
+    named_bar_sync(4, 32 * (4 * kAtSoftWGs + 2));  // the softmax warps have read TMEM for the last time
+    if (lane == 0) mbar_wait_drain(&S.mma_done[is_qk ? 0 : 1], 0);  // no MMA of this issuer still runs
     __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, kAtTmemCols);
+    named_bar_sync(5, 64);  // both issuers drained
+    if (is_qk) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kAtTmemCols);
+    }
     return;
   }
 
   // ---------------------------------------------------------------- softmax warps
-  const int tid = threadIdx.x;  // 0..127: key of the pair, then output column d
-  const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+  const int wg = warp >> 2;            // takes the pairs with global index % 2 == wg
+  const int tid = threadIdx.x & 127;   // key of the pair, then output column d
+  const int bar = 1 + wg;              // this warpgroup's named barrier
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
   const float sl2 = p.scale_log2;
   uint32_t gp = 0;
   int it = 0;
@@ -277,19 +333,21 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const AttnItem a = attn_item(p, item);
     const int n = S.n_blocks[slot];
     const int np = (n + 1) / 2;
-    const uint32_t obuf = tlane + 32u + static_cast<uint32_t>(it & 1) * 16u;
+    const uint32_t obuf = tlane + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + wg) * 16u;
     float m[kGroupRows], l[kGroupRows];
 #pragma unroll
     for (int h = 0; h < kGroupRows; ++h) {
       m[h] = -INFINITY;
       l[h] = 0.f;
     }
-    for (int i = 0; i < np; ++i) {
+    int i0 = 0;
+    while (i0 < np && ((gp + i0) & 1) != static_cast<uint32_t>(wg)) ++i0;
+    for (int i = i0; i < np; i += 2) {
       const uint32_t pp = gp + i;
-      mbar_wait(&S.s_full[pp & 1], (pp >> 1) & 1, &S.abort);
+      mbar_wait(&S.s_full[pp % kAtBufs], (pp / kAtBufs) & 1, &S.abort);
       tc_fence_after();
       uint32_t sv[16];
-      tmem_ld16(tlane + static_cast<uint32_t>(pp & 1) * 16u, sv);
+      tmem_ld16(tlane + static_cast<uint32_t>(pp % kAtBufs) * 16u, sv);
       const int bi = 2 * i + (tid >> 6);
       const int blk = bi < n ? S.list[slot][bi] : -1;
       const int key = blk * kBlock + (tid & 63);
@@ -301,11 +359,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         x[h] = valid ? __uint_as_float(sv[h]) * sl2 : -INFINITY;
         viol |= x[h] > m[h] + 8.f;
       }
-      if (named_bar_or(1, 128, viol)) {
+      if (named_bar_or(bar, 128, viol)) {
         // a score rose more than 2^8 above its reference: move the references to the
-        // pair maxima and rescale what was accumulated so far
+        // pair maxima and rescale what this warpgroup accumulated so far
         float mx[kGroupRows];
-        wg_reduce16<true>(x, mx, S);
+        wg_reduce16<true>(x, mx, S, wg);
         float al[kGroupRows];
 #pragma unroll
         for (int h = 0; h < kGroupRows; ++h) {
@@ -314,8 +372,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           l[h] *= al[h];
           m[h] = mn;
         }
-        if (i >= 1) {
-          mbar_wait(&S.pv_done[(pp - 1) & 1], ((pp - 1) >> 1) & 1, &S.abort);
+        if (i >= i0 + 2) {  // this warpgroup has accumulated into its O^T before
+          mbar_wait(&S.pv_done[(pp - 2) % kAtBufs], ((pp - 2) / kAtBufs) & 1, &S.abort);  // previous PV
           tc_fence_after();
           uint32_t ov[16];
           tmem_ld16(obuf, ov);
@@ -330,9 +388,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         pv[h] = (m[h] == -INFINITY) ? 0.f : ex2(x[h] - m[h]);
         l[h] += pv[h];
       }
-      if (pp >= 2) mbar_wait(&S.pv_done[pp & 1], ((pp - 2) >> 1) & 1, &S.abort);  // P buffer free
+      if (pp >= kAtBufs) mbar_wait(&S.pv_done[pp % kAtBufs], ((pp / kAtBufs) - 1) & 1, &S.abort);  // P free
       {
-        unsigned char* pbuf = pbufs + (pp & 1) * kAtPBytes + (tid >> 6) * (kAtPBytes / 2);
+        unsigned char* pbuf = pbufs + (pp % kAtBufs) * kAtPBytes + (tid >> 6) * (kAtPBytes / 2);
         const int col = tid & 63;
 #pragma unroll
         for (int h = 0; h < kGroupRows; ++h) {
@@ -342,43 +400,69 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_bar_sync(1, 128);
-      if (tid == 0) mbar_arrive(&S.p_full[pp & 1]);
+      named_bar_sync(bar, 128);
+      if (tid == 0) mbar_arrive(&S.p_full[pp % kAtBufs]);
     }
 
-    // ---- end of item: normalise O^T (thread = column d) and write O and lse
+    // ---- end of item: merge the two warpgroups' partial states (thread = column d)
     float L[kGroupRows];
-    wg_reduce16<false>(l, L, S);
-    float ov_f[kGroupRows];
-    if (np > 0) {
-      const uint32_t last = gp + np - 1;
-      mbar_wait(&S.pv_done[last & 1], (last >> 1) & 1, &S.abort);
-      tc_fence_after();
-      uint32_t ov[16];
-      tmem_ld16(obuf, ov);
-#pragma unroll
-      for (int h = 0; h < kGroupRows; ++h) ov_f[h] = L[h] > 0.f ? __uint_as_float(ov[h]) / L[h] : 0.f;
-    } else {
-#pragma unroll
-      for (int h = 0; h < kGroupRows; ++h) ov_f[h] = 0.f;
-    }
-#pragma unroll
-    for (int h = 0; h < kGroupRows; ++h)
-      if (h < p.G) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(ov_f[h]);
+    wg_reduce16<false>(l, L, S, wg);
     if (tid == 0) {
 #pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) {
+        S.mstate[wg][h] = m[h];
+        S.lstate[wg][h] = L[h];
+      }
+    }
+    const bool had = i0 < np;  // this warpgroup accumulated into its O^T
+    uint32_t ov[16];
+    if (had) {
+      const uint32_t last = gp + i0 + 2 * ((np - 1 - i0) / 2);
+      mbar_wait(&S.pv_done[last % kAtBufs], (last / kAtBufs) & 1, &S.abort);
+      tc_fence_after();
+      tmem_ld16(obuf, ov);
+    }
+    named_bar_sync(3, 32 * 4 * kAtSoftWGs);  // both warpgroups' states are in shared memory
+    float M[kGroupRows], Lt[kGroupRows], w0[kGroupRows], w1[kGroupRows];
+#pragma unroll
+    for (int h = 0; h < kGroupRows; ++h) {
+      const float m0 = S.mstate[0][h], m1 = S.mstate[1][h];
+      M[h] = fmaxf(m0, m1);
+      w0[h] = (m0 == -INFINITY) ? 0.f : ex2(m0 - M[h]);
+      w1[h] = (m1 == -INFINITY) ? 0.f : ex2(m1 - M[h]);
+      Lt[h] = S.lstate[0][h] * w0[h] + S.lstate[1][h] * w1[h];
+    }
+    // warpgroup 0 reads warpgroup 1's O^T buffer directly (same TMEM lanes) and merges
+    tc_fence_after();
+    if (wg == 0) {
+      uint32_t ov1[16];
+      const uint32_t obuf1 = tlane + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + 1) * 16u;
+      const bool had1 = ((gp & 1u) ? 0 : 1) < np;  // first pair of warpgroup 1 in this item
+      if (had1) tmem_ld16(obuf1, ov1);
+      float of[kGroupRows];
+#pragma unroll
+      for (int h = 0; h < kGroupRows; ++h) {
+        const float a0 = had ? __uint_as_float(ov[h]) * w0[h] : 0.f;
+        const float a1 = had1 ? __uint_as_float(ov1[h]) * w1[h] : 0.f;
+        of[h] = Lt[h] > 0.f ? (a0 + a1) / Lt[h] : 0.f;
+      }
+#pragma unroll
       for (int h = 0; h < kGroupRows; ++h)
-        S.lse_out[h] = L[h] > 0.f ? (m[h] + lg2(L[h])) * 0.6931471805599453f : -INFINITY;
+        if (h < p.G) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(of[h]);
+      if (p.lse != nullptr && tid < p.G) {
+        float lv = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < kGroupRows; ++h)
+          if (h == tid) lv = Lt[h] > 0.f ? (M[h] + lg2(Lt[h])) * 0.6931471805599453f : -INFINITY;
+        p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.t] = lv;
+      }
     }
     tc_fence_before();
-    named_bar_sync(1, 128);
-    if (p.lse != nullptr && tid < p.G)
-      p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.t] = S.lse_out[tid];
-    if (tid == 0) mbar_arrive(&S.q_empty[slot]);
-    named_bar_sync(1, 128);  // S.lse_out reuse
+    named_bar_sync(3, 32 * 4 * kAtSoftWGs);  // outputs read; states may be overwritten
+    if (threadIdx.x == 0) mbar_arrive(&S.q_empty[slot]);
     gp += np;
   }
-  named_bar_sync(2, 160);  // TMEM may be freed
+  named_bar_sync(4, 32 * (4 * kAtSoftWGs + 2));  // TMEM may be freed
 }
 
 }  // namespace infllmv2
