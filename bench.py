@@ -355,7 +355,7 @@ def run_decode(args, rank, world, device, pk, peak_src):
             "select": {"us": sel_med, "algorithmic_bytes": sel_b, "achieved_GBps": sel_b / sel_med / 1e3},
             "attn": {"us": att_med, "algorithmic_bytes": att_b, "achieved_GBps": att_b / att_med / 1e3},
         },
-        "gpu_launches_per_step": 4,
+        "gpu_launches_per_step": 2 if ws_a.numel() == 0 else 3,
     }
 
 

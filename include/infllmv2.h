@@ -135,7 +135,10 @@ INFLLMV2_API int infllmv2_compress_keys(const infllmv2_params* p, const void* k,
  *              block_idx int32 [B, Hkv, 1, topk].
  *   ws, ws_bytes  device workspace of at least infllmv2_workspace_size(p,
  *              INFLLMV2_OP_SELECT_PREFILL or _DECODE, L_or_Lmax) bytes (may be NULL
- *              when that size is 0).  Contents on entry do not matter. */
+ *              when that size is 0, which it is for both modes in this version).
+ *              Contents on entry do not matter.
+ *  Decode runs one thread-block cluster of up to 16 CTAs per (b, g); a device that
+ *  cannot co-schedule that cluster gets INFLLMV2_ERR_UNSUPPORTED before any launch. */
 INFLLMV2_API int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, const void* kc,
                            const int32_t* lens, int32_t L_or_Lmax, int32_t* block_idx,
                            void* ws, size_t ws_bytes, infllmv2_stream_t stream);
@@ -154,12 +157,14 @@ INFLLMV2_API int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const vo
 
 /* Sparse attention for one decode token per sequence ([S] s2.1.3, prefill *and*
  * decode per s2.1 of the same page).  Split over the selected blocks across CTAs,
- * then merged with the partial log-sum-exps.
+ * then merged with the partial log-sum-exps: inside a thread-block cluster per
+ * (b, kv-head) (no workspace) when B * Hkv >= SMs / 16, else through the workspace.
  *   q          bf16 [B, Hq, d];  k_cache, v_cache bf16 [B, Hkv, Lmax, d]
  *   lens       int32 [B] device, 1 <= lens[b] <= Lmax; the query sits at lens[b]-1
  *   block_idx  int32 [B, Hkv, 1, topk] (as for prefill)
  *   o          bf16 [B, Hq, d];  lse fp32 [B, Hq] or NULL
- *   ws         at least infllmv2_workspace_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax) bytes */
+ *   ws         at least infllmv2_workspace_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax) bytes;
+ *              may be NULL when that size is 0 */
 INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache,
                                 const void* v_cache, const int32_t* lens, int32_t Lmax,
                                 const int32_t* block_idx, void* o, float* lse, void* ws,
@@ -170,12 +175,15 @@ INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const voi
  * memory at call time -- e.g. an engine plugin whose execute step must not allocate, or
  * a service that reserves its whole memory budget at start-up and forbids later
  * cudaMalloc.  Same arguments and results as infllmv2_sparse_attn_decode without
- * ws/ws_bytes; the split partials live in a fixed 8 MiB array inside the library
+ * ws/ws_bytes; when the problem takes the workspace path (few sequences), the split
+ * partials live in a fixed 8 MiB array inside the library
  * (INFLLMV2_NOALLOC_SCRATCH_BYTES), which every GPU that loads the library holds until
  * the process exits.
  *  - Returns INFLLMV2_ERR_WORKSPACE, without launching anything, when the problem needs
  *    more scratch than that (the need is infllmv2_workspace_size(p,
- *    INFLLMV2_OP_ATTN_DECODE, Lmax); e.g. B * Hkv = 64 sequence-heads fit easily).
+ *    INFLLMV2_OP_ATTN_DECODE, Lmax)).  With the split rule of this version the need
+ *    stays below about 2.5 MB for every valid parameter set, so the check is a guard
+ *    against future split rules rather than a limit callers meet.
  *  - The first call on a device looks up the array's device address (one
  *    cudaGetSymbolAddress, with that device current); make that first call before any
  *    stream capture.

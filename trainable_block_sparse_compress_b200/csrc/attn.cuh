@@ -12,8 +12,8 @@
 // each block; each keeps an online softmax for the 16 heads (rows) over its keys and
 // accumulates O = P V with m16n8k16 bf16 MMAs (fp32 accumulators).  At the end of an
 // item the four partial states are merged in shared memory.
-// Decode splits an item's blocks over several items and writes partial (O, lse) to
-// the workspace; attn_merge_kernel combines them.
+// For decode with very few sequences, an item's blocks are split over several items
+// that write partial (O, lse) to the workspace; attn_merge_kernel combines them.
 #pragma once
 #include "common.cuh"
 
@@ -81,6 +81,108 @@ struct AttnSmem {
 constexpr size_t attn_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(kAttnStages) * kAttnStageBytes + 2 * kQTileBytes +
          static_cast<size_t>(kAttnConsumers) * kGroupRows * kMergeRowFloats * 4 + sizeof(AttnSmem);
+}
+
+// One consumer warp's share (keys [kofs, kofs + 16)) of a staged K/V block j (K then V,
+// 64 x 128 bf16 each, 128-byte swizzle) for the query rows at position t: S = Q K^T,
+// online softmax in base 2 (running max m, row sum l) and O += P V.  Keys past t are
+// masked; their V rows are zeroed first so that they contribute exactly 0.
+__device__ __forceinline__ void attn_block_update(unsigned char* sk_ptr, int j, int t, int kofs,
+                                                  const uint32_t (&qa)[8][4], float scale_log2, float& m0,
+                                                  float& m1, float& l0, float& l1, float (&o)[16][4]) {
+  const int lane = threadIdx.x & 31;
+  const int q4 = lane & 3;
+  const uint32_t sk = smem_u32(sk_ptr);
+  const uint32_t sv = sk + kKvTileBytes;
+  const int valid = t - j * kBlock + 1;  // keys of this block at positions <= t
+  const bool partial = valid < kofs + 16;  // some of this warp's 16 keys lie past t
+  if (partial) {
+    // zero this warp's V rows past t so that masked keys contribute exactly 0
+    uint4* vrow = reinterpret_cast<uint4*>(sk_ptr + kKvTileBytes);
+    for (int c = max(valid, kofs) * 8 + lane; c < (kofs + 16) * 8; c += 32) {
+      const int r = c >> 3, ch = c & 7;
+      vrow[r * 8 + ch] = make_uint4(0, 0, 0, 0);
+      vrow[(kKvTileBytes / 2) / 16 + r * 8 + ch] = make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();
+  }
+
+  // S = Q K^T for this warp's 16 keys: 16 x 16
+  float s[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int mi = lane >> 3;
+    const int key = kofs + (lane & 7) + ((mi >> 1) << 3);
+    const int d = 16 * ks + ((mi & 1) << 3);
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4(sk + (d >> 6) * (kKvTileBytes / 2) + sw128(key, (d & 63) >> 3), b0, b1, b2, b3);
+    mma_bf16(s[0], qa[ks], b0, b1);
+    mma_bf16(s[1], qa[ks], b2, b3);
+  }
+
+  // online softmax (base 2)
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int col = kofs + 8 * nt + 2 * q4 + e;
+      const bool ok = !partial || col < valid;
+      s[nt][e] = ok ? s[nt][e] * scale_log2 : -INFINITY;
+      s[nt][2 + e] = ok ? s[nt][2 + e] * scale_log2 : -INFINITY;
+      mx0 = fmaxf(mx0, s[nt][e]);
+      mx1 = fmaxf(mx1, s[nt][2 + e]);
+    }
+  }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+  if (mn0 != -INFINITY) {  // all 16 keys of this warp may lie past t
+    const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      s[nt][0] = ex2(s[nt][0] - mn0);
+      s[nt][1] = ex2(s[nt][1] - mn0);
+      s[nt][2] = ex2(s[nt][2] - mn1);
+      s[nt][3] = ex2(s[nt][3] - mn1);
+      rs0 += s[nt][0] + s[nt][1];
+      rs1 += s[nt][2] + s[nt][3];
+    }
+    l0 = l0 * al0 + rs0;
+    l1 = l1 * al1 + rs1;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      o[nt][0] *= al0;
+      o[nt][1] *= al0;
+      o[nt][2] *= al1;
+      o[nt][3] *= al1;
+    }
+
+    // O += P V : P (16 x 16) from registers, V rows of this warp via transposed ldmatrix
+    uint32_t pa[4];
+    pa[0] = pack_bf16(s[0][0], s[0][1]);
+    pa[1] = pack_bf16(s[0][2], s[0][3]);
+    pa[2] = pack_bf16(s[1][0], s[1][1]);
+    pa[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+    for (int dp = 0; dp < 8; ++dp) {
+      const int mi = lane >> 3;
+      const int key = kofs + (lane & 7) + ((mi & 1) << 3);
+      const int d = 16 * dp + ((mi >> 1) << 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(sv + (d >> 6) * (kKvTileBytes / 2) + sw128(key, (d & 63) >> 3), b0, b1, b2, b3);
+      mma_bf16(o[2 * dp], pa, b0, b1);
+      mma_bf16(o[2 * dp + 1], pa, b2, b3);
+    }
+  }
+  if (partial) fence_proxy_async_smem();
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -204,99 +306,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const long long gb = gbase + i;
       const int st = static_cast<int>(gb % kAttnStages);
       mbar_wait(&S.full[st], static_cast<uint32_t>((gb / kAttnStages) & 1), &S.abort);
-      const int j = S.list[slot][i];
-      unsigned char* sk_ptr = stages + st * kAttnStageBytes;
-      const uint32_t sk = smem_u32(sk_ptr);
-      const uint32_t sv = sk + kKvTileBytes;
-      const int valid = a.t - j * kBlock + 1;  // keys of this block at positions <= t
-      const bool partial = valid < kofs + 16;  // some of this warp's 16 keys lie past t
-      if (partial) {
-        // zero this warp's V rows past t so that masked keys contribute exactly 0
-        uint4* vrow = reinterpret_cast<uint4*>(sk_ptr + kKvTileBytes);
-        for (int c = max(valid, kofs) * 8 + lane; c < (kofs + 16) * 8; c += 32) {
-          const int r = c >> 3, ch = c & 7;
-          vrow[r * 8 + ch] = make_uint4(0, 0, 0, 0);
-          vrow[(kKvTileBytes / 2) / 16 + r * 8 + ch] = make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-      }
-
-      // S = Q K^T for this warp's 16 keys: 16 x 16
-      float s[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const int mi = lane >> 3;
-        const int key = kofs + (lane & 7) + ((mi >> 1) << 3);
-        const int d = 16 * ks + ((mi & 1) << 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sk + (d >> 6) * (kKvTileBytes / 2) + sw128(key, (d & 63) >> 3), b0, b1, b2, b3);
-        mma_bf16(s[0], qa[ks], b0, b1);
-        mma_bf16(s[1], qa[ks], b2, b3);
-      }
-
-      // online softmax (base 2)
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = kofs + 8 * nt + 2 * q4 + e;
-          const bool ok = !partial || col < valid;
-          s[nt][e] = ok ? s[nt][e] * p.scale_log2 : -INFINITY;
-          s[nt][2 + e] = ok ? s[nt][2 + e] * p.scale_log2 : -INFINITY;
-          mx0 = fmaxf(mx0, s[nt][e]);
-          mx1 = fmaxf(mx1, s[nt][2 + e]);
-        }
-      }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      if (mn0 != -INFINITY) {  // all 16 keys of this warp may lie past t
-        const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-        m0 = mn0;
-        m1 = mn1;
-        float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          s[nt][0] = ex2(s[nt][0] - mn0);
-          s[nt][1] = ex2(s[nt][1] - mn0);
-          s[nt][2] = ex2(s[nt][2] - mn1);
-          s[nt][3] = ex2(s[nt][3] - mn1);
-          rs0 += s[nt][0] + s[nt][1];
-          rs1 += s[nt][2] + s[nt][3];
-        }
-        l0 = l0 * al0 + rs0;
-        l1 = l1 * al1 + rs1;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[nt][0] *= al0;
-          o[nt][1] *= al0;
-          o[nt][2] *= al1;
-          o[nt][3] *= al1;
-        }
-
-        // O += P V : P (16 x 16) from registers, V rows of this warp via transposed ldmatrix
-        uint32_t pa[4];
-        pa[0] = pack_bf16(s[0][0], s[0][1]);
-        pa[1] = pack_bf16(s[0][2], s[0][3]);
-        pa[2] = pack_bf16(s[1][0], s[1][1]);
-        pa[3] = pack_bf16(s[1][2], s[1][3]);
-#pragma unroll
-        for (int dp = 0; dp < 8; ++dp) {
-          const int mi = lane >> 3;
-          const int key = kofs + (lane & 7) + ((mi & 1) << 3);
-          const int d = 16 * dp + ((mi >> 1) << 3);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sv + (d >> 6) * (kKvTileBytes / 2) + sw128(key, (d & 63) >> 3), b0, b1, b2, b3);
-          mma_bf16(o[2 * dp], pa, b0, b1);
-          mma_bf16(o[2 * dp + 1], pa, b2, b3);
-        }
-      }
-      if (partial) fence_proxy_async_smem();
+      attn_block_update(stages + st * kAttnStageBytes, S.list[slot][i], a.t, kofs, qa, p.scale_log2, m0, m1, l0,
+                        l1, o);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[st]);
     }
@@ -372,30 +383,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // Combines the decode splits: o = sum_s exp(lse_s - lse) o_s, lse = log sum_s exp(lse_s).
-// grid = B * Hkv, block = 128 (thread covers one column for all 16 rows).
+// grid = B * Hkv * G (one head row each), block = 128 (one column each; thread s also
+// carries split s's weight).
+constexpr int kMaxDecodeSplits = 128;
+
 __global__ void __launch_bounds__(128) attn_merge_kernel(const float* __restrict__ part_o,
                                                          const float* __restrict__ part_lse, int n_splits,
                                                          int Hq, int Hkv, int G, __nv_bfloat16* __restrict__ o,
                                                          float* __restrict__ lse) {
-  const long long bg = blockIdx.x;
+  __shared__ float w[kMaxDecodeSplits];
+  __shared__ float red_m[4], red_l[4];
+  const long long bg = blockIdx.x / G;
+  const int r = static_cast<int>(blockIdx.x % G);
   const int b = static_cast<int>(bg / Hkv), g = static_cast<int>(bg % Hkv);
-  const int d = threadIdx.x;
-  for (int r = 0; r < G; ++r) {
-    float M = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, part_lse[(bg * n_splits + s) * kGroupRows + r]);
-    float L = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < n_splits; ++s) {
-        const long long prow = (bg * n_splits + s) * kGroupRows + r;
-        const float w = __expf(part_lse[prow] - M);
-        L += w;
-        acc += w * part_o[prow * kHeadDim + d];
-      }
-    }
-    const long long orow = static_cast<long long>(b) * Hq + g * G + r;
-    o[orow * kHeadDim + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-    if (lse != nullptr && d == 0) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
-  }
+  const int d = threadIdx.x, lane = d & 31, wp = d >> 5;
+  const float x = d < n_splits ? part_lse[(bg * n_splits + d) * kGroupRows + r] : -INFINITY;
+  float M = x;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) red_m[wp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+  const float e = (d < n_splits && M != -INFINITY) ? __expf(x - M) : 0.f;
+  if (d < n_splits) w[d] = e;
+  float L = e;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  if (lane == 0) red_l[wp] = L;
+  __syncthreads();
+  L = (red_l[0] + red_l[1]) + (red_l[2] + red_l[3]);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < n_splits; ++s) acc += w[s] * part_o[((bg * n_splits + s) * kGroupRows + r) * kHeadDim + d];
+  const long long orow = static_cast<long long>(b) * Hq + g * G + r;
+  o[orow * kHeadDim + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+  if (lse != nullptr && d == 0) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
 }
 
 }  // namespace infllmv2

@@ -1,0 +1,235 @@
+// attn_dec.cuh -- sparse attention for one decode token per sequence, split over a
+// thread-block cluster and merged through distributed shared memory.
+//
+// MiniCPM4 summary page (端设备上的超高效大型语言模型) s2.1: InfLLM v2 speeds up decoding
+// as well as prefill; s2.1.3: the token attends only to its selected blocks, and the
+// query heads of a group share them (s2.1.2), so each block is read once per group.
+//
+// A decode step has only B x Hkv (sequence, kv-head) items, each reading its selected
+// 64-key blocks (32 KB of K and V per block) from HBM.  A cluster of C CTAs serves one
+// item: CTA c takes a contiguous share of the compacted block list, streams its blocks
+// through a TMA ring (128-byte swizzle, no multicast) and runs the four-warp m16n8k16
+// online softmax of the prefill fallback kernel (16 keys of each block per warp).  The
+// CTA's partial state -- running max and row sum (base 2) and unnormalised O for the 16
+// head rows -- stays in its shared memory.  After a cluster barrier CTA c merges head
+// rows [16 c / C, 16 (c + 1) / C) from every peer's state, read through distributed
+// shared memory, and writes O and the log-sum-exp.  No workspace, one launch; the
+// bound is HBM bandwidth (512 bytes of K and V per attended key and kv-head).
+#pragma once
+#include <cooperative_groups.h>
+
+#include "attn.cuh"
+#include "common.cuh"
+
+namespace infllmv2 {
+
+constexpr int kAdStages = 3;
+constexpr int kAdThreads = kAttnThreads;  // 4 consumer warps + 1 producer warp
+constexpr int kAdMaxCluster = 16;
+constexpr int kAdWarpRows = kGroupRows * kMergeRowFloats;  // floats of one warp's partial O
+static_assert((kAttnConsumers + 1) * kAdWarpRows * 4 <= kAdStages * kAttnStageBytes,
+              "the merge scratch reuses the drained ring");
+
+struct AdSmem {
+  uint64_t full[kAdStages], empty[kAdStages], qbar;
+  int n_blocks;
+  int list[kMaxTopk];
+  float m[kAttnConsumers][kGroupRows], l[kAttnConsumers][kGroupRows];
+  float cm[kGroupRows], cl[kGroupRows];  // this CTA's state per head: max (base 2), row sum
+  volatile int abort;
+};
+
+constexpr size_t attn_dec_smem_bytes() {
+  return 1024 + static_cast<size_t>(kAdStages) * kAttnStageBytes + kQTileBytes + sizeof(AdSmem);
+}
+
+// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.  C divides 16.
+__global__ void __launch_bounds__(kAdThreads)
+    attn_decode_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* ring = align_smem(smem_raw, 1024);
+  unsigned char* qtile = ring + kAdStages * kAttnStageBytes;
+  AdSmem& S = *reinterpret_cast<AdSmem*>(qtile + kQTileBytes);
+  float* part = reinterpret_cast<float*>(ring);      // [4 warps][16][kMergeRowFloats], once the ring drained
+  float* comb = part + kAttnConsumers * kAdWarpRows;  // [16][kMergeRowFloats]: this CTA's state
+
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int crank = static_cast<int>(cluster.block_rank());
+  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
+  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+  const int t = min(p.lens[b], p.Lmax) - 1;  // < 0: empty sequence
+  const int cur = t >= 0 ? t / kBlock : -1;
+  const int qrow = b * p.Hq + g * p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAdStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kAttnConsumers);
+    }
+    mbar_init(&S.qbar, 1);
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kAttnConsumers) {  // compact the item's valid block indices, in list order
+    const int32_t* row = p.idx + bg * static_cast<long long>(p.topk);
+    int count = 0;
+    for (int e0 = 0; e0 < p.topk; e0 += 32) {
+      const int e = e0 + lane;
+      const int j = e < p.topk ? row[e] : -1;
+      const bool ok = j >= 0 && j <= cur;
+      const unsigned msk = __ballot_sync(0xffffffffu, ok);
+      if (ok) S.list[count + __popc(msk & ((1u << lane) - 1u))] = j;
+      count += __popc(msk);
+    }
+    if (lane == 0) S.n_blocks = count;
+  }
+  __syncthreads();
+  const int n_all = S.n_blocks;
+  const int per = (n_all + C - 1) / C;
+  const int lo = min(crank * per, n_all);
+  const int n = min(lo + per, n_all) - lo;
+
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[16][4];
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  if (warp == kAttnConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(&S.qbar, kQTileBytes);
+      tma_load_2d(qtile, &tm_q, &S.qbar, 0, qrow);
+      tma_load_2d(qtile + kQTileBytes / 2, &tm_q, &S.qbar, 64, qrow);
+      const long long kvrow0 = bg * p.Lmax;
+      int i = 0;
+      for (; i < n; ++i) {
+        const int st = i % kAdStages, u = i / kAdStages;
+        if (u > 0 && !mbar_wait(&S.empty[st], (u - 1) & 1, &S.abort)) break;
+        const int krow = static_cast<int>(kvrow0 + static_cast<long long>(S.list[lo + i]) * kBlock);
+        unsigned char* sk = ring + st * kAttnStageBytes;
+        mbar_arrive_expect_tx(&S.full[st], kAttnStageBytes);
+        tma_load_2d(sk, &tm_k, &S.full[st], 0, krow);
+        tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.full[st], 64, krow);
+        tma_load_2d(sk + kKvTileBytes, &tm_v, &S.full[st], 0, krow);
+        tma_load_2d(sk + kKvTileBytes + kKvTileBytes / 2, &tm_v, &S.full[st], 64, krow);
+      }
+      mbar_wait_drain(&S.qbar, 0);
+      if (S.abort) {  // let every issued copy land before the ring is reused
+        for (int j = max(0, i - kAdStages); j < i; ++j) mbar_wait_drain(&S.full[j % kAdStages], (j / kAdStages) & 1);
+      }
+    }
+  } else if (n > 0) {
+    // --------------------------------------------------------- consumer warps
+    uint32_t qa[8][4];
+    if (mbar_wait(&S.qbar, 0, &S.abort)) {
+      const uint32_t qs = smem_u32(qtile);
+      const int mi = lane >> 3;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int row = (lane & 7) + ((mi & 1) << 3);
+        const int d = 16 * ks + ((mi >> 1) << 3);
+        ldsm_x4(qs + (d >> 6) * (kQTileBytes / 2) + sw128(row, (d & 63) >> 3), qa[ks][0], qa[ks][1], qa[ks][2],
+                qa[ks][3]);
+      }
+      for (int i = 0; i < n; ++i) {
+        const int st = i % kAdStages;
+        if (!mbar_wait(&S.full[st], (i / kAdStages) & 1, &S.abort)) break;
+        attn_block_update(ring + st * kAttnStageBytes, S.list[lo + i], t, 16 * warp, qa, p.scale_log2, m0, m1, l0,
+                          l1, o);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[st]);
+      }
+    }
+  }
+  __syncthreads();  // the ring is drained: it becomes the merge scratch
+  if (warp < kAttnConsumers) {
+    const int q4 = lane & 3, r0 = lane >> 2;
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    float* mo = part + warp * kAdWarpRows;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int col = 8 * nt + 2 * q4;
+      *reinterpret_cast<float2*>(mo + r0 * kMergeRowFloats + col) = make_float2(o[nt][0], o[nt][1]);
+      *reinterpret_cast<float2*>(mo + (r0 + 8) * kMergeRowFloats + col) = make_float2(o[nt][2], o[nt][3]);
+    }
+    if (q4 == 0) {
+      S.m[warp][r0] = m0;
+      S.m[warp][r0 + 8] = m1;
+      S.l[warp][r0] = l0;
+      S.l[warp][r0 + 8] = l1;
+    }
+  }
+  __syncthreads();
+  // this CTA's state: the four warps combined (warp w: rows 4 w .. 4 w + 3)
+  if (warp < kAttnConsumers) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int r = 4 * warp + rr;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kAttnConsumers; ++w) M = fmaxf(M, S.m[w][r]);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kAttnConsumers; ++w) {
+          const float wt = ex2(S.m[w][r] - M);
+          L += wt * S.l[w][r];
+          const float4 v = *reinterpret_cast<const float4*>(part + w * kAdWarpRows + r * kMergeRowFloats + 4 * lane);
+          acc.x += wt * v.x;
+          acc.y += wt * v.y;
+          acc.z += wt * v.z;
+          acc.w += wt * v.w;
+        }
+      }
+      *reinterpret_cast<float4*>(comb + r * kMergeRowFloats + 4 * lane) = acc;
+      if (lane == 0) {
+        S.cm[r] = M;
+        S.cl[r] = L;
+      }
+    }
+  }
+  cluster.sync();  // every CTA's state is final
+
+  // CTA crank merges head rows [crank h_per, (crank + 1) h_per) across the cluster
+  const int h_per = kGroupRows / C;
+  for (int hh = warp; hh < h_per; hh += kAdThreads / 32) {
+    const int h = crank * h_per + hh;
+    float M = -INFINITY;
+    for (int r = 0; r < C; ++r) M = fmaxf(M, cluster.map_shared_rank(&S.cm[0], r)[h]);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int r = 0; r < C; ++r) {
+        const float wt = ex2(cluster.map_shared_rank(&S.cm[0], r)[h] - M);
+        L += wt * cluster.map_shared_rank(&S.cl[0], r)[h];
+        const float4 v =
+            *reinterpret_cast<const float4*>(cluster.map_shared_rank(comb, r) + h * kMergeRowFloats + 4 * lane);
+        acc.x += wt * v.x;
+        acc.y += wt * v.y;
+        acc.z += wt * v.z;
+        acc.w += wt * v.w;
+      }
+    }
+    if (h < p.G) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      uint2 pk;
+      pk.x = pack_bf16(acc.x * inv, acc.y * inv);
+      pk.y = pack_bf16(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(p.o + (static_cast<long long>(qrow) + h) * kHeadDim + 4 * lane) = pk;
+      if (p.lse != nullptr && lane == 0)
+        p.lse[static_cast<long long>(qrow) + h] = L > 0.f ? (M + lg2(L)) * 0.6931471805599453f : -INFINITY;
+    }
+  }
+  cluster.sync();  // peers' shared memory stays valid until every CTA has read it
+}
+
+}  // namespace infllmv2

@@ -8,10 +8,14 @@
 
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <utility>
 
 #include "../../include/infllmv2.h"
 #include "attn.cuh"
+#include "attn_dec.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
@@ -121,14 +125,84 @@ int set_smem(const void* fn, size_t bytes) {
              : INFLLMV2_ERR_CUDA;
 }
 
-// Decode attention split: selected blocks per split and number of splits per (b, g).
-void decode_split(const infllmv2_params* p, int* n_splits, int* per_split) {
-  const long long bgs = static_cast<long long>(p->batch) * p->num_kv_heads;
-  const int sms = num_sms();
-  int s = static_cast<int>((4LL * sms + bgs - 1) / bgs);
-  s = std::max(1, std::min(s, (p->topk + 7) / 8));
-  *per_split = (p->topk + s - 1) / s;
-  *n_splits = (p->topk + *per_split - 1) / *per_split;
+// Launches `kern` on a 1-D grid in clusters of C CTAs.  Sizes above 8 need the
+// non-portable opt-in.  A cluster shape that the device cannot co-schedule is reported
+// as unsupported before any launch (checked once per kernel, size and device).
+template <typename... Params, typename... Args>
+int launch_cluster(void (*kern)(Params...), unsigned grid, int C, int threads, size_t smem, cudaStream_t s,
+                   Args&&... args) {
+  const void* fn = reinterpret_cast<const void*>(kern);
+  int st = set_smem(fn, smem);
+  if (st != INFLLMV2_OK) return st;
+  if (C > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return INFLLMV2_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, int>, int> fits;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(fn, C, dev);
+    auto it = fits.find(key);
+    if (it == fits.end()) {
+      int active = 0;
+      if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+      it = fits.emplace(key, active).first;
+    }
+    if (it->second < 1) return INFLLMV2_ERR_UNSUPPORTED;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  return launch_status();
+}
+
+// Decode work layout.  Each (sequence, kv-head) item's selected blocks are split over
+// CTAs.  Normally a cluster of C CTAs (a power of two up to 16, as large as keeps all
+// CTAs resident at two per SM) merges its partials in distributed shared memory.  When
+// even 16 CTAs per item leave most SMs idle (fewer items than SMs / 16), the blocks are
+// split further, two or more per CTA, and the partials meet in the workspace.
+struct DecodePlan {
+  int cluster;   // CTAs per cluster (cluster path), 0 for the workspace path
+  int n_splits;  // workspace path: splits per item
+  int per_split;
+};
+
+DecodePlan decode_plan(const infllmv2_params* p) {
+  const long long items = static_cast<long long>(p->batch) * p->num_kv_heads;
+  const long long target = 2LL * num_sms();
+  DecodePlan d{0, 1, p->topk};
+  if (items * kAdMaxCluster >= num_sms()) {
+    int c = 1;
+    while (c < kAdMaxCluster && items * c * 2 <= target) c *= 2;
+    d.cluster = c;
+    return d;
+  }
+  int s = static_cast<int>(std::min<long long>((target + items - 1) / items, (p->topk + 1) / 2));
+  s = std::max(1, std::min(s, kMaxDecodeSplits));
+  d.per_split = (p->topk + s - 1) / s;
+  d.n_splits = (p->topk + d.per_split - 1) / d.per_split;
+  return d;
+}
+
+// Selection cluster size: enough CTAs for the longest sequence's kernels (at most
+// kSdMaxChunk per CTA), and as many as keep all CTAs resident at two per SM.
+int select_cluster(const infllmv2_params* p, int64_t nk) {
+  const long long items = static_cast<long long>(p->batch) * p->num_kv_heads;
+  const long long target = 2LL * num_sms();
+  int c = 1;
+  while (c < kSdMaxCluster && (static_cast<int64_t>(c) * kSdMaxChunk < nk || items * c * 2 <= target)) c *= 2;
+  return c;
 }
 
 size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
@@ -138,16 +212,13 @@ size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
     case INFLLMV2_OP_SELECT_PREFILL:
     case INFLLMV2_OP_ATTN_PREFILL:
       return 0;
-    case INFLLMV2_OP_SELECT_DECODE: {
-      const int nch = static_cast<int>((num_kernels(L) + kDecChunk - 1) / kDecChunk);
-      return sel_decode_ws_bytes(p->batch, p->num_kv_heads, std::max(nch, 1));
-    }
+    case INFLLMV2_OP_SELECT_DECODE:
+      return 0;
     case INFLLMV2_OP_ATTN_DECODE: {
-      int ns, per;
-      decode_split(p, &ns, &per);
-      const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * ns * kGroupRows;
-      const size_t a = rows * kHeadDim * sizeof(float);
-      return a + rows * sizeof(float);
+      const DecodePlan d = decode_plan(p);
+      if (d.cluster > 0) return 0;
+      const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * d.n_splits * kGroupRows;
+      return rows * kHeadDim * sizeof(float) + rows * sizeof(float);
     }
     default:
       return static_cast<size_t>(-1);
@@ -225,12 +296,14 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
   if (q == nullptr || block_idx == nullptr || !aligned16(q) || !aligned16(block_idx)) return INFLLMV2_ERR_INVALID_ARG;
   const int64_t nk = num_kernels(L);
   if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
+  if (static_cast<uint64_t>(p->batch) * p->num_kv_heads * static_cast<uint64_t>(nk) > 0x7fffffffULL)
+    return INFLLMV2_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
   if (mode == INFLLMV2_MODE_PREFILL) {
     if (lens != nullptr) return INFLLMV2_ERR_INVALID_ARG;
   } else if (mode == INFLLMV2_MODE_DECODE) {
     if (lens == nullptr || (reinterpret_cast<uintptr_t>(lens) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
-    const size_t need = ws_size(p, INFLLMV2_OP_SELECT_DECODE, L);
-    if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return INFLLMV2_ERR_WORKSPACE;
+    (void)ws;  // decode selection needs no workspace
+    (void)ws_bytes;
   } else {
     return INFLLMV2_ERR_INVALID_ARG;
   }
@@ -299,23 +372,13 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
   a.topk = p->topk;
   a.n_init = p->n_init;
   a.n_local = p->n_local;
-  a.n_chunks = std::max(1, static_cast<int>((nk + kDecChunk - 1) / kDecChunk));
   a.scale_log2 = scale_log2(p);
-  const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * a.n_chunks;
-  a.ws_lse = static_cast<float2*>(ws);
-  const size_t lse_bytes = (rows * kGroupRows * sizeof(float2) + 255) & ~static_cast<size_t>(255);
-  a.ws_bm = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + lse_bytes);
-  if (nk > 0) {
-    const size_t smem = sel_decode_score_smem_bytes();
-    if ((st = set_smem(reinterpret_cast<const void*>(select_decode_score_kernel), smem)) != INFLLMV2_OK) return st;
-    dim3 grid(a.n_chunks, p->num_kv_heads, p->batch);
-    select_decode_score_kernel<<<grid, kDecScoreThreads, smem, s>>>(tm_kc, a);
-    if ((st = launch_status()) != INFLLMV2_OK) return st;
-  }
-  const size_t smem2 = static_cast<size_t>(nblk_cap) * 4 + kGroupRows * 4 + 256 * 4;
-  if ((st = set_smem(reinterpret_cast<const void*>(select_decode_topk_kernel), smem2)) != INFLLMV2_OK) return st;
-  select_decode_topk_kernel<<<dim3(p->num_kv_heads, p->batch), kDecTopkThreads, smem2, s>>>(a, nblk_cap);
-  return launch_status();
+  if (nk == 0 && !make_map(&tm_kc, q, kKcTile, kKcTile)) return INFLLMV2_ERR_CUDA;  // never read: no tiles
+  const int C = select_cluster(p, nk);
+  const long long grid = static_cast<long long>(C) * p->batch * p->num_kv_heads;
+  if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+  const size_t smem = sel_decode_smem_bytes();
+  return launch_cluster(select_decode_kernel, static_cast<unsigned>(grid), C, kSdThreads, smem, s, tm_kc, a);
 }
 
 static int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
@@ -393,9 +456,10 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
     return INFLLMV2_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
   const size_t need = ws_size(p, INFLLMV2_OP_ATTN_DECODE, Lmax);
-  if (ws == nullptr || ws_bytes < need || !aligned16(ws)) return INFLLMV2_ERR_WORKSPACE;
-  int ns, per;
-  decode_split(p, &ns, &per);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) return INFLLMV2_ERR_WORKSPACE;
+  const uint64_t kv_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * Lmax;
+  if (kv_rows > 0x7fffffffULL) return INFLLMV2_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  const DecodePlan d = decode_plan(p);
   AttnParams a;
   a.idx = block_idx;
   a.lens = lens;
@@ -406,21 +470,33 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
   a.Lq = 1;
   a.Lmax = Lmax;
   a.topk = p->topk;
-  a.n_splits = ns;
-  a.blocks_per_split = per;
+  a.n_splits = d.n_splits;
+  a.blocks_per_split = d.per_split;
   a.scale_log2 = scale_log2(p);
-  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * ns;
+  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * d.n_splits;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
-  const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * ns * kGroupRows;
+  a.part_o = nullptr;
+  a.part_lse = nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * p->num_q_heads;
+  if (d.cluster > 0) {
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k_cache, kv_rows, kBlock) ||
+        !make_map(&tv, v_cache, kv_rows, kBlock))
+      return INFLLMV2_ERR_CUDA;
+    const long long grid = static_cast<long long>(d.cluster) * p->batch * p->num_kv_heads;
+    if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+    return launch_cluster(attn_decode_cluster_kernel, static_cast<unsigned>(grid), d.cluster, kAdThreads,
+                          attn_dec_smem_bytes(), s, tq, tk, tv, a);
+  }
+  const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * d.n_splits * kGroupRows;
   a.part_o = static_cast<float*>(ws);
   a.part_lse = a.part_o + rows * kHeadDim;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = launch_attn(p, q, static_cast<uint64_t>(p->batch) * p->num_q_heads, k_cache, v_cache,
-                   static_cast<uint64_t>(p->batch) * p->num_kv_heads * Lmax, a, s);
+  st = launch_attn(p, q, q_rows, k_cache, v_cache, kv_rows, a, s);
   if (st != INFLLMV2_OK) return st;
-  attn_merge_kernel<<<static_cast<unsigned>(static_cast<long long>(p->batch) * p->num_kv_heads), 128, 0, s>>>(
-      a.part_o, a.part_lse, ns, p->num_q_heads, p->num_kv_heads, a.G, static_cast<__nv_bfloat16*>(o), lse);
+  attn_merge_kernel<<<static_cast<unsigned>(static_cast<long long>(p->batch) * p->num_kv_heads * a.G), 128, 0, s>>>(
+      a.part_o, a.part_lse, d.n_splits, p->num_q_heads, p->num_kv_heads, a.G, static_cast<__nv_bfloat16*>(o), lse);
   return launch_status();
 }
 

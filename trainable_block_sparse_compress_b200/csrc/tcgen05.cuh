@@ -144,18 +144,4 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Waits like mbar_wait but ignores the CTA abort flag (only the time limit): used for
-// the final drains that must complete before TMEM is released.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint32_t addr = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(addr, parity)) return true;
-    if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_device_error, 1u);
-      return false;
-    }
-  }
-}
-
 }  // namespace infllmv2
