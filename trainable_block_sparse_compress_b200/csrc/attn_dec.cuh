@@ -60,11 +60,11 @@ __global__ void __launch_bounds__(kAdThreads)
   const int crank = static_cast<int>(cluster.block_rank());
   const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
   const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int t = min(p.lens[b], p.Lmax) - 1;  // < 0: empty sequence
-  const int cur = t >= 0 ? t / kBlock : -1;
   const int qrow = b * p.Hq + g * p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // prologue that reads no input: it overlaps the end of the selection kernel
+  allow_dependent_launch();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAdStages; ++s) {
       mbar_init(&S.full[s], 1);
@@ -74,6 +74,14 @@ __global__ void __launch_bounds__(kAdThreads)
     S.abort = 0;
     fence_mbar_init();
   }
+  if (warp == kAttnConsumers && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  grid_dependency_wait();  // block_idx (and q, the caches, lens) are complete from here on
+  const int t = min(p.lens[b], p.Lmax) - 1;  // < 0: empty sequence
+  const int cur = t >= 0 ? t / kBlock : -1;
   if (warp == kAttnConsumers) {  // compact the item's valid block indices, in list order
     const int32_t* row = p.idx + bg * static_cast<long long>(p.topk);
     int count = 0;
@@ -100,8 +108,6 @@ __global__ void __launch_bounds__(kAdThreads)
   if (warp == kAttnConsumers) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n > 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(&S.qbar, kQTileBytes);
       tma_load_2d(qtile, &tm_q, &S.qbar, 0, qrow);
       tma_load_2d(qtile + kQTileBytes / 2, &tm_q, &S.qbar, 64, qrow);

@@ -126,6 +126,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  grid_dependency_wait() returns once every grid this
+// one depends on has completed and its memory writes are visible (at once when there is
+// none); nothing may read what an earlier kernel on the stream wrote before it.
+// allow_dependent_launch() lets the next kernel on the stream, when launched with
+// programmatic stream serialization, start its own prologue early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a tile written by
 // TMA with 128-byte swizzling (rows of 128 bytes, tile base 1024-byte aligned).
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {

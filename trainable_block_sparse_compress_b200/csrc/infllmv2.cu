@@ -126,11 +126,12 @@ int set_smem(const void* fn, size_t bytes) {
 }
 
 // Launches `kern` on a 1-D grid in clusters of C CTAs.  Sizes above 8 need the
-// non-portable opt-in.  A cluster shape that the device cannot co-schedule is reported
+// non-portable opt-in.  With `pdl` the kernel may start while the previous kernel on the
+// stream finishes (it must call grid_dependency_wait() before reading any input).  A cluster shape that the device cannot co-schedule is reported
 // as unsupported before any launch (checked once per kernel, size and device).
 template <typename... Params, typename... Args>
 int launch_cluster(void (*kern)(Params...), unsigned grid, int C, int threads, size_t smem, cudaStream_t s,
-                   Args&&... args) {
+                   bool pdl, Args&&... args) {
   const void* fn = reinterpret_cast<const void*>(kern);
   int st = set_smem(fn, smem);
   if (st != INFLLMV2_OK) return st;
@@ -141,13 +142,15 @@ int launch_cluster(void (*kern)(Params...), unsigned grid, int C, int threads, s
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   {
     static std::mutex mu;
     static std::map<std::tuple<const void*, int, int>, int> fits;
@@ -378,7 +381,8 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
   const long long grid = static_cast<long long>(C) * p->batch * p->num_kv_heads;
   if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
   const size_t smem = sel_decode_smem_bytes();
-  return launch_cluster(select_decode_kernel, static_cast<unsigned>(grid), C, kSdThreads, smem, s, tm_kc, a);
+  return launch_cluster(select_decode_kernel, static_cast<unsigned>(grid), C, kSdThreads, smem, s, true, tm_kc,
+                        a);
 }
 
 static int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
@@ -488,7 +492,7 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
     const long long grid = static_cast<long long>(d.cluster) * p->batch * p->num_kv_heads;
     if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
     return launch_cluster(attn_decode_cluster_kernel, static_cast<unsigned>(grid), d.cluster, kAdThreads,
-                          attn_dec_smem_bytes(), s, tq, tk, tv, a);
+                          attn_dec_smem_bytes(), s, true, tq, tk, tv, a);
   }
   const size_t rows = static_cast<size_t>(p->batch) * p->num_kv_heads * d.n_splits * kGroupRows;
   a.part_o = static_cast<float*>(ws);

@@ -6,14 +6,18 @@
 // is split over the C CTAs of a cluster; CTA c takes a contiguous chunk of whole
 // 64-kernel tiles and streams them from HBM with TMA (128-byte swizzle, no multicast):
 //   1. per tile, four warps (16 kernels each) compute the 16 x 64 logits with m16n8k16
-//      MMAs, keep an online (max, sum of exp2) per head, and store per head the max of
-//      every aligned quad of kernels 4q .. 4q+3 and the quad's last kernel;
-//   2. after a cluster barrier each CTA forms lse_h from the C partial states (read
-//      through distributed shared memory) and, for its share of the blocks, the block
-//      maxima m_h(j) = max(quad j, last kernel of quad j-1) -- block j pools kernels
-//      4j-1 .. 4j+3 -- and S(j) = sum_h exp(m_h(j) - lse_h); the keys go to CTA 0;
+//      MMAs and keep an online (max, sum of exp2) per head.  Block j pools kernels
+//      4j-1 .. 4j+3, so each aligned quad of kernels 4q .. 4q+3 goes into the block max
+//      of block q and its last kernel also into that of block q+1 (shared-memory atomic
+//      max on an order-preserving integer image of the float);
+//   2. after a cluster barrier each CTA forms lse_h from the C partial states and takes
+//      the previous CTA's carry into its first block (both read through distributed
+//      shared memory, all loads in parallel), computes S(j) = sum_h exp(m_h(j) - lse_h)
+//      for its blocks and stores the keys into CTA 0;
 //   3. CTA 0 finds the k-th largest key by a 32-way radix search (lane l of every warp
-//      counts the keys at or above candidate digit l) and writes the ascending list.
+//      counts the keys at or above candidate digit l; once the digit's bucket holds at
+//      most 32 keys they are ranked directly) and all its threads write the ascending
+//      list (prefix sums place ties and outputs).
 // No workspace, one launch; reading Kc once bounds it (HBM).
 #pragma once
 #include <cooperative_groups.h>
@@ -28,9 +32,9 @@ constexpr int kSdConsumers = 4;
 constexpr int kSdWarps = kSdConsumers + 1;  // + the TMA producer warp
 constexpr int kSdThreads = 32 * kSdWarps;
 constexpr int kSdStages = 4;
-constexpr int kSdMaxChunk = 1024;  // kernels per CTA at most
+constexpr int kSdMaxChunk = 2048;  // kernels per CTA at most
 constexpr int kSdMaxQuads = kSdMaxChunk / 4;
-constexpr int kSdQStride = kSdMaxQuads + 4;  // per-head quad arrays, padded against bank conflicts
+constexpr int kSdBStride = kSdMaxQuads + 4;  // per-head block-max rows (quads + 1 carry), padded
 constexpr int kSdMaxCluster = 16;
 static_assert(kSdStages * kKcTileBytes >= 4 * (INFLLMV2_MAX_SEQ_LEN / kBlock),
               "the block keys of CTA 0 reuse its tile ring");
@@ -49,21 +53,43 @@ struct SdSmem {
   uint64_t full[kSdStages], empty[kSdStages];
   float m[kSdConsumers][kGroupRows], l[kSdConsumers][kGroupRows];
   float cm[kGroupRows], cl[kGroupRows];  // this CTA's (max, sum of exp2) per head
-  float lse2[kGroupRows];                // log2-sum-exp2 per head over the whole sequence
+  float pm[kSdMaxCluster][kGroupRows], pl[kSdMaxCluster][kGroupRows];  // every CTA's, gathered
+  float lse2[kGroupRows];  // log2-sum-exp2 per head over the whole sequence
+  float carry[kGroupRows];  // previous CTA's last kernel, for this CTA's first block
   int cnt[2][kSdWarps][32];
+  int scan[2][kSdWarps];
+  int nlist;
+  uint32_t list[32];
   volatile int abort;
 };
 
 constexpr size_t sel_decode_smem_bytes() {
-  return 1024 + static_cast<size_t>(kSdStages) * kKcTileBytes + 2 * kGroupRows * kSdQStride * 4 + sizeof(SdSmem);
+  return 1024 + static_cast<size_t>(kSdStages) * kKcTileBytes + static_cast<size_t>(kGroupRows) * kSdBStride * 4 +
+         sizeof(SdSmem);
+}
+
+// Order-preserving image of a float in uint32 (a < b exactly when enc(a) < enc(b)), so
+// that integer atomicMax computes a float max.
+__device__ __forceinline__ uint32_t ord_enc(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_dec(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ int ge4(const uint4 v, uint32_t c) {
+  return (v.x >= c ? 1 : 0) + (v.y >= c ? 1 : 0) + (v.z >= c ? 1 : 0) + (v.w >= c ? 1 : 0);
 }
 
 // k-th largest of n keys in shared memory (zero-padded to a multiple of 4) by all
-// kSdThreads threads: 31 key bits in digits of 5,5,5,5,5,5,1 bits, lane l of each warp
-// counting the keys >= T | l << shift over the warp's share; partial counts meet in
-// `cnt` (double-buffered: one barrier per digit).  Same result as warp_radix_threshold.
-__device__ __forceinline__ TopkThreshold cta_radix_threshold(const uint32_t* keys, int n, int want,
-                                                             int (*cnt)[kSdWarps][32]) {
+// kSdThreads threads; same result as warp_radix_threshold.  Radix search on the 31 key
+// bits in digits of 5 (the last one 1): lane l of every warp counts the keys >= T | l <<
+// shift over the warp's share, the counts meet in S.cnt (double-buffered: one barrier per
+// digit) and the largest digit with at least `want` keys at or above it is taken.  As
+// soon as the chosen digit's bucket holds at most 32 keys, they are gathered and ranked
+// directly.
+__device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys, int n, int want, SdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   TopkThreshold r;
   if (want <= 0) {
@@ -75,45 +101,136 @@ __device__ __forceinline__ TopkThreshold cta_radix_threshold(const uint32_t* key
   const int n4 = (n + 3) >> 2;
   int buf = 0;
   auto count_ge = [&](uint32_t c) -> int {
-    int a = 0, b = 0;
-    for (int i = warp; i < n4; i += kSdWarps) {
-      const uint4 v = k4[i];
-      a += (v.x >= c ? 1 : 0) + (v.y >= c ? 1 : 0);
-      b += (v.z >= c ? 1 : 0) + (v.w >= c ? 1 : 0);
+    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+    int i = warp;
+#pragma unroll 1
+    for (; i + 3 * kSdWarps < n4; i += 4 * kSdWarps) {
+      const uint4 v0 = k4[i], v1 = k4[i + kSdWarps], v2 = k4[i + 2 * kSdWarps], v3 = k4[i + 3 * kSdWarps];
+      a0 += ge4(v0, c);
+      a1 += ge4(v1, c);
+      a2 += ge4(v2, c);
+      a3 += ge4(v3, c);
     }
-    cnt[buf][warp][lane] = a + b;
+    for (; i < n4; i += kSdWarps) a0 += ge4(k4[i], c);
+    S.cnt[buf][warp][lane] = (a0 + a1) + (a2 + a3);
     __syncthreads();
     int tot = 0;
 #pragma unroll
-    for (int w = 0; w < kSdWarps; ++w) tot += cnt[buf][w][lane];
+    for (int w = 0; w < kSdWarps; ++w) tot += S.cnt[buf][w][lane];
     buf ^= 1;
     return tot;
   };
-  // top digit; lane 0 counts the candidates (keys >= 1) instead of testing digit 0
+  // first digit (bits 30..26); lane 0 counts the candidates (keys >= 1): bucket 0 is [1, 2^26)
+  int tot = count_ge(lane == 0 ? 1u : static_cast<uint32_t>(lane) << 26);
+  if (__shfl_sync(0xffffffffu, tot, 0) <= want) {  // at most `want` candidates: take them all
+    r.key = 0;
+    r.ties = 0;
+    return r;
+  }
   uint32_t T = 0;
-  {
-    const int tot = count_ge(lane == 0 ? 1u : static_cast<uint32_t>(lane) << 26);
-    if (__shfl_sync(0xffffffffu, tot, 0) <= want) {  // at most `want` candidates: take them all
-      r.key = 0;
-      r.ties = 0;
-      return r;
-    }
-    const unsigned ok = __ballot_sync(0xffffffffu, lane > 0 && tot >= want);
-    if (ok != 0u) T = static_cast<uint32_t>(31 - __clz(ok)) << 26;
+  int shift = 26, above = 0, inb = 0;  // bucket [max(T, 1), T + 2^shift): `inb` keys, `above` keys above it
+  for (;;) {
+    const unsigned ok = __ballot_sync(0xffffffffu, tot >= want);  // lane 0 always qualifies
+    const int l = 31 - __clz(ok);
+    const int nxt = __shfl_sync(0xffffffffu, tot, min(l + 1, 31));
+    if (l < 31) above = nxt;
+    inb = __shfl_sync(0xffffffffu, tot, l) - above;
+    T |= static_cast<uint32_t>(l) << shift;
+    if (inb <= 32 || shift == 0) break;
+    shift = shift > 5 ? shift - 5 : 0;
+    // the last digit is bit 0 alone: lanes >= 2 test the bucket's upper end (count = above)
+    tot = count_ge(shift > 0 ? T | (static_cast<uint32_t>(lane) << shift) : (lane < 2 ? T | lane : T + 2u));
   }
-#pragma unroll 1
-  for (int shift = 21; shift >= 1; shift -= 5) {
-    const int tot = count_ge(T | (static_cast<uint32_t>(lane) << shift));
-    const unsigned ok = __ballot_sync(0xffffffffu, tot >= want);  // lane 0 tests T itself
-    T |= static_cast<uint32_t>(31 - __clz(ok)) << shift;
+  if (shift == 0) {  // the bucket is the single value T
+    r.key = T;
+    r.ties = want - above;
+    return r;
   }
-  {
-    const int tot = count_ge(T | (lane == 1 ? 1u : 0u));
-    if (__shfl_sync(0xffffffffu, tot, 1) >= want) T |= 1u;
+  // rank the <= 32 keys of the bucket directly: the answer is the (want - above)-th largest
+  const uint32_t lo = max(T, 1u), hi = T + (1u << shift);
+  if (threadIdx.x == 0) S.nlist = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += kSdThreads) {
+    const uint32_t k = keys[j];
+    if (k >= lo && k < hi) S.list[atomicAdd(&S.nlist, 1)] = k;
   }
-  r.key = T;
-  r.ties = want - count_ge(T + 1u);
+  __syncthreads();
+  const int nl = S.nlist;  // == inb
+  const uint32_t x = lane < nl ? S.list[lane] : 0u;
+  int gt = 0, ge = 0;
+  for (int i = 0; i < nl; ++i) {
+    const uint32_t v = S.list[i];
+    gt += v > x ? 1 : 0;
+    ge += v >= x ? 1 : 0;
+  }
+  const int rank = want - above;
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < nl && gt < rank && rank <= ge);
+  const int src = __ffs(hit) - 1;
+  r.key = __shfl_sync(0xffffffffu, x, src);
+  r.ties = want - above - __shfl_sync(0xffffffffu, gt, src);
   return r;
+}
+
+// Exclusive prefix sum of v over the kSdThreads threads (thread order); *total gets the
+// sum.  buf holds kSdWarps ints and must not be in use by another scan.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* buf, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) buf[warp] = x;
+  __syncthreads();
+  int base = 0, sum = 0;
+#pragma unroll
+  for (int w = 0; w < kSdWarps; ++w) {
+    base += w < warp ? buf[w] : 0;
+    sum += buf[w];
+  }
+  *total = sum;
+  return base + x - v;
+}
+
+// All kSdThreads threads write the selected blocks of one row, ascending, padded with
+// -1: block j in [0, n) is taken when forced, or key > T, or key == T among the first
+// `ties` such keys in ascending j (the rule of warp_emit_selection).  Thread i scans the
+// contiguous keys [i s, (i + 1) s); two prefix sums place the tie ranks and the outputs.
+__device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, TopkThreshold th, int cur,
+                                                   int n_init, int n_local, int topk, int32_t* out,
+                                                   int (*scan)[kSdWarps]) {
+  const int seg = (n + kSdThreads - 1) / kSdThreads;
+  const int j0 = min(static_cast<int>(threadIdx.x) * seg, n), j1 = min(j0 + seg, n);
+  const bool all = th.key == 0u;  // take every candidate
+  int my_ties = 0;
+  if (!all)
+    for (int j = j0; j < j1; ++j) my_ties += keys[j] == th.key ? 1 : 0;
+  int total = 0;
+  const int tie0 = cta_exclusive_scan(my_ties, scan[0], &total);
+  auto take = [&](int j, uint32_t k, int& tr) -> bool {
+    const bool forced = j < n_init || j > cur - n_local;
+    if (all) return forced || k > 0u;
+    const bool tie = k == th.key;
+    const bool t = forced || (k > th.key && th.key != 0xffffffffu) || (tie && tr < th.ties);
+    if (tie) ++tr;
+    return t;
+  };
+  int my_take = 0;
+  {
+    int tr = tie0;
+    for (int j = j0; j < j1; ++j) my_take += take(j, keys[j], tr) ? 1 : 0;
+  }
+  int pos = cta_exclusive_scan(my_take, scan[1], &total);
+  {
+    int tr = tie0;
+    for (int j = j0; j < j1; ++j)
+      if (take(j, keys[j], tr)) {
+        if (pos < topk) out[pos] = j;
+        ++pos;
+      }
+  }
+  for (int e = total + static_cast<int>(threadIdx.x); e < topk; e += kSdThreads) out[e] = -1;
 }
 
 // grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.
@@ -123,20 +240,21 @@ __global__ void __launch_bounds__(kSdThreads)
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ unsigned char smem_raw[];
   unsigned char* ring = align_smem(smem_raw, 1024);
-  float* qmax = reinterpret_cast<float*>(ring + kSdStages * kKcTileBytes);  // [16][kSdQStride]
-  float* qlast = qmax + kGroupRows * kSdQStride;                             // [16][kSdQStride]
-  SdSmem& S = *reinterpret_cast<SdSmem*>(qlast + kGroupRows * kSdQStride);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(ring + kSdStages * kKcTileBytes);  // [16][kSdBStride], ord_enc
+  SdSmem& S = *reinterpret_cast<SdSmem*>(bm + kGroupRows * kSdBStride);
   uint32_t* keys = reinterpret_cast<uint32_t*>(ring);  // CTA 0 only, once every tile is consumed
 
   const int C = static_cast<int>(cluster.num_blocks());
   const int c = static_cast<int>(cluster.block_rank());
   const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
   const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+  allow_dependent_launch();  // the decode attention may set up while this selection runs
+  grid_dependency_wait();    // q, Kc and lens may come from the previous kernel
   const int n = min(max(p.lens[b], 0), p.Lmax);
   const int nk = n >= kKernel ? (n - kKernel) / kStride + 1 : 0;
   const int cur = n > 0 ? (n - 1) / kBlock : -1;
   const int chunk = ((nk + C - 1) / C + kKcTile - 1) / kKcTile * kKcTile;  // kernels per CTA
-  const int nq = chunk / 4;                                                 // quads per CTA
+  const int nq = chunk / 4;                                                 // blocks per CTA
   const int k0 = c * chunk;
   const int ntiles = nk > k0 ? (min(chunk, nk - k0) + kKcTile - 1) / kKcTile : 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -149,12 +267,10 @@ __global__ void __launch_bounds__(kSdThreads)
     S.abort = 0;
     fence_mbar_init();
   }
-  // quads past this CTA's tiles (and the one after its chunk) hold no visible kernel
-  for (int e = threadIdx.x; e < kGroupRows * (nq + 1 - 16 * ntiles); e += kSdThreads) {
-    const int h = e / (nq + 1 - 16 * ntiles), qd = 16 * ntiles + e % (nq + 1 - 16 * ntiles);
-    qmax[h * kSdQStride + qd] = -INFINITY;
-    qlast[h * kSdQStride + qd] = -INFINITY;
-  }
+  // bm[h][q]: max over this CTA's kernels 4q-1 .. 4q+3 (local numbering); q = nq holds
+  // the chunk's last kernel, carried into the next CTA's first block
+  for (int e = threadIdx.x; e < kGroupRows * (nq + 1); e += kSdThreads)
+    bm[(e / (nq + 1)) * kSdBStride + e % (nq + 1)] = ord_enc(-INFINITY);
   __syncthreads();
 
   if (warp == kSdConsumers) {
@@ -216,7 +332,8 @@ __global__ void __launch_bounds__(kSdThreads)
             mx1 = fmaxf(mx1, s[nt][2 + e]);
           }
         }
-        // quad maxima and each quad's last kernel (lanes q4 = 0, 2 own quads 2 nt, 2 nt + 1)
+        // quad q (lanes q4 = 0, 2 of n-tile nt: quads 2 nt, 2 nt + 1 of the warp's four):
+        // its max feeds block q, its last kernel block q + 1
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const float pm0 = fmaxf(s[nt][0], s[nt][1]), pm1 = fmaxf(s[nt][2], s[nt][3]);
@@ -225,10 +342,10 @@ __global__ void __launch_bounds__(kSdThreads)
           const float la1 = __shfl_xor_sync(0xffffffffu, s[nt][3], 1);
           if ((q4 & 1) == 0) {
             const int qd = (i * kKcTile + kofs + 8 * nt + 4 * (q4 >> 1)) >> 2;
-            qmax[r0 * kSdQStride + qd] = fmaxf(pm0, om0);
-            qlast[r0 * kSdQStride + qd] = la0;
-            qmax[(r0 + 8) * kSdQStride + qd] = fmaxf(pm1, om1);
-            qlast[(r0 + 8) * kSdQStride + qd] = la1;
+            atomicMax(&bm[r0 * kSdBStride + qd], ord_enc(fmaxf(pm0, om0)));
+            atomicMax(&bm[r0 * kSdBStride + qd + 1], ord_enc(la0));
+            atomicMax(&bm[(r0 + 8) * kSdBStride + qd], ord_enc(fmaxf(pm1, om1)));
+            atomicMax(&bm[(r0 + 8) * kSdBStride + qd + 1], ord_enc(la1));
           }
         }
         // online (max, sum of exp2) per head
@@ -276,25 +393,34 @@ __global__ void __launch_bounds__(kSdThreads)
   }
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
 
-  if (threadIdx.x < kGroupRows) {
-    const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int r = 0; r < C; ++r) M = fmaxf(M, cluster.map_shared_rank(&S.cm[0], r)[h]);
-    float L = 0.f;
-    if (M != -INFINITY) {
-      for (int r = 0; r < C; ++r)
-        L += cluster.map_shared_rank(&S.cl[0], r)[h] * ex2(cluster.map_shared_rank(&S.cm[0], r)[h] - M);
-    }
-    S.lse2[h] = L > 0.f ? M + lg2(L) : INFINITY;
+  // gather every CTA's (max, sum) and the previous CTA's carry, all loads in flight at once
+  for (int e = threadIdx.x; e < kGroupRows * C; e += kSdThreads) {
+    const int r = e / kGroupRows, h = e % kGroupRows;
+    S.pm[r][h] = cluster.map_shared_rank(&S.cm[0], r)[h];
+    S.pl[r][h] = cluster.map_shared_rank(&S.cl[0], r)[h];
+  }
+  if (threadIdx.x >= kSdThreads - kGroupRows) {
+    const int h = threadIdx.x - (kSdThreads - kGroupRows);
+    S.carry[h] = c > 0 ? ord_dec(cluster.map_shared_rank(bm, c - 1)[h * kSdBStride + nq]) : -INFINITY;
   }
   if (c == 0) {  // zero padding up to a multiple of 4 keys for the vector scan
     for (int j = cur + 1 + threadIdx.x; j < ((cur + 4) & ~3); j += kSdThreads) keys[j] = 0u;
   }
   __syncthreads();
-  // this CTA's blocks: quads [c nq, (c + 1) nq); the last CTA also takes the rest up to cur
+  if (threadIdx.x < kGroupRows) {
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int r = 0; r < C; ++r) M = fmaxf(M, S.pm[r][h]);
+    float L = 0.f;
+    if (M != -INFINITY) {
+      for (int r = 0; r < C; ++r) L += S.pl[r][h] * ex2(S.pm[r][h] - M);
+    }
+    S.lse2[h] = L > 0.f ? M + lg2(L) : INFINITY;
+  }
+  __syncthreads();
+  // this CTA's blocks: [c nq, (c + 1) nq); the last CTA also takes the rest up to cur
   {
     uint32_t* keys0 = cluster.map_shared_rank(keys, 0);
-    const float* prev_last = c > 0 ? cluster.map_shared_rank(qlast, c - 1) : nullptr;
     const int jb0 = c * nq;
     const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
     for (int j = jb0 + threadIdx.x; j < jb1; j += kSdThreads) {
@@ -305,8 +431,8 @@ __global__ void __launch_bounds__(kSdThreads)
       if (eligible && !forced && ql <= nq) {
         float sc = 0.f;
         for (int h = 0; h < p.G; ++h) {
-          float mb = qmax[h * kSdQStride + ql];
-          if (j > 0) mb = fmaxf(mb, ql > 0 ? qlast[h * kSdQStride + ql - 1] : prev_last[h * kSdQStride + nq - 1]);
+          float mb = ord_dec(bm[h * kSdBStride + ql]);
+          if (ql == 0) mb = fmaxf(mb, S.carry[h]);
           sc += ex2(mb - S.lse2[h]);
         }
         key = __float_as_uint(sc) + 1u;
@@ -323,8 +449,8 @@ __global__ void __launch_bounds__(kSdThreads)
     return;
   }
   const int want = p.topk - forced_count(cur, p.n_init, p.n_local);
-  const TopkThreshold th = cta_radix_threshold(keys, cur + 1, want, S.cnt);
-  if (warp == 0) warp_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out);
+  const TopkThreshold th = cta_topk_threshold(keys, cur + 1, want, S);
+  cta_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out, S.scan);
 }
 
 }  // namespace infllmv2
