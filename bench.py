@@ -48,21 +48,30 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha(name: str) -> str:
-    with open(os.path.join(ROOT, "trainable_block_sparse_compress_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha() -> str:
+    """Hash of every CUDA source of the library: a DRAM-traffic figure counts only when it
+    was taken on exactly these sources."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "trainable_block_sparse_compress_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
-def dram_traffic(kernel: str, source: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+def dram_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch from the committed ncu summary, if it was
+    taken on the current sources and the same workload (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get(kernel, {})
-    if e.get("source_sha") != source_sha(source) or e.get("workload") != workload:
+    if d.get("source_sha") != source_sha():
+        return None
+    e = d.get("kernels", {}).get(kernel, {})
+    if e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -226,11 +235,17 @@ def run_ours(args, rank, world, device):
     for kv in kern.values():
         kv["frac"] = kv["achieved"] / kv["peak"]
     top = max(kern, key=lambda n: kern[n]["ms"])
-    src = {"compress": "compress.cuh", "select": "select_prefill.cuh", "attn": "attn.cuh"}[top]
-    kname = {"compress": "compress_kernel", "select": "select_prefill_kernel", "attn": "attn_kernel"}[top]
+    tc = p.num_q_heads // p.num_kv_heads == 16  # the tensor-core (tcgen05) prefill kernels serve G = 16
+    names = {"compress": "compress_kernel",
+             "select": "select_prefill_tc_kernel" if tc else "select_prefill_kernel",
+             "attn": "attn_tc_kernel" if tc else "attn_kernel"}
+    for n, kv in kern.items():
+        kv["kernel"] = names[n]
+        kv["traffic"] = dram_traffic(names[n], args.workload)
+    kname = names[top]
     roof = {"kernel": kname, "bound": kern[top]["bound"], "achieved": kern[top]["achieved"],
             "peak": kern[top]["peak"], "unit": kern[top]["unit"], "frac": kern[top]["frac"],
-            "traffic": dram_traffic(kname, src, args.workload),
+            "traffic": kern[top]["traffic"],
             "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kern[top]['bound'] == 'tensor' else 'hbm_gbs'})"}
 
     result = {
@@ -358,18 +373,26 @@ def run_decode(args, rank, world, device, pk, peak_src):
         torch.distributed.all_reduce(us_t, op=torch.distributed.ReduceOp.MAX)
     us = float(us_t.item())
     sel_b, att_b = decode_bytes(p, x.lens.numpy())
+    att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
     sel_med, att_med = statistics.median(sel_us), statistics.median(att_us)
+    tr_s = dram_traffic("select_decode_kernel", args.decode_workload)
+    tr_a = dram_traffic(att_kernel, args.decode_workload)
     return {
         "workload": args.decode_workload, "value": us, "unit": "us/step", "higher_is_better": False,
         "batch": p.batch, "mean_len": float(x.lens.float().mean()), "steps": n,
         "l2": "flushed before every step (write then read a 2x L2 buffer, outside the timed events)",
         "roofline": {"bound": "hbm", "achieved": (sel_b + att_b) / us / 1e3, "peak": hbm, "unit": "GB/s",
                      "frac": (sel_b + att_b) / us / 1e3 / hbm, "algorithmic_bytes": sel_b + att_b,
+                     "traffic": tr_s + tr_a if tr_s is not None and tr_a is not None else None,
                      "peak_source": f"{peak_src} (hbm_gbs)"},
         "kernels": {
-            "select": {"us": sel_med, "algorithmic_bytes": sel_b, "achieved_GBps": sel_b / sel_med / 1e3},
-            "attn": {"us": att_med, "algorithmic_bytes": att_b, "achieved_GBps": att_b / att_med / 1e3},
+            "select": {"kernel": "select_decode_kernel", "us": sel_med, "algorithmic_bytes": sel_b,
+                       "achieved_GBps": sel_b / sel_med / 1e3,
+                       "traffic": tr_s},
+            "attn": {"kernel": att_kernel, "us": att_med, "algorithmic_bytes": att_b,
+                     "achieved_GBps": att_b / att_med / 1e3,
+                     "traffic": tr_a},
         },
         "gpu_launches_per_step": 2 if ws_a.numel() == 0 else 3,
     }
