@@ -92,6 +92,7 @@ __device__ __forceinline__ int ge4(const uint4 v, uint32_t c) {
 __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys, int n, int want, SdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   TopkThreshold r;
+  r.all_ties = false;
   if (want <= 0) {
     r.key = 0xffffffffu;
     r.ties = 0;
@@ -144,6 +145,7 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   if (shift == 0) {  // the bucket is the single value T
     r.key = T;
     r.ties = want - above;
+    r.all_ties = above + inb == want;
     return r;
   }
   // rank the <= 32 keys of the bucket directly: the answer is the (want - above)-th largest
@@ -168,6 +170,7 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   const int src = __ffs(hit) - 1;
   r.key = __shfl_sync(0xffffffffu, x, src);
   r.ties = want - above - __shfl_sync(0xffffffffu, gt, src);
+  r.all_ties = above + __shfl_sync(0xffffffffu, ge, src) == want;
   return r;
 }
 
@@ -202,17 +205,18 @@ __device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, 
                                                    int (*scan)[kSdWarps]) {
   const int seg = (n + kSdThreads - 1) / kSdThreads;
   const int j0 = min(static_cast<int>(threadIdx.x) * seg, n), j1 = min(j0 + seg, n);
-  const bool all = th.key == 0u;  // take every candidate
+  const bool simple = topk_simple(th);  // no tie ranks needed: take forced or key >= lo
+  const uint32_t lo = take_from(th);
   int my_ties = 0;
-  if (!all)
+  if (!simple)
     for (int j = j0; j < j1; ++j) my_ties += keys[j] == th.key ? 1 : 0;
   int total = 0;
-  const int tie0 = cta_exclusive_scan(my_ties, scan[0], &total);
+  const int tie0 = simple ? 0 : cta_exclusive_scan(my_ties, scan[0], &total);
   auto take = [&](int j, uint32_t k, int& tr) -> bool {
     const bool forced = j < n_init || j > cur - n_local;
-    if (all) return forced || k > 0u;
+    if (simple) return forced || k >= lo;
     const bool tie = k == th.key;
-    const bool t = forced || (k > th.key && th.key != 0xffffffffu) || (tie && tr < th.ties);
+    const bool t = forced || k > th.key || (tie && tr < th.ties);
     if (tie) ++tr;
     return t;
   };

@@ -5,18 +5,29 @@
 // scoring blocks): higher score first, lower block index first among equal scores.
 // Scores are non-negative fp32 group sums, so their IEEE bit patterns order like the
 // values.  A candidate's key is bits(score) + 1 and a non-candidate's key is 0.
-// The k-th largest key is found by bisection on the key bits with warp-wide counts; the
-// list is then written in ascending block order with forced blocks first-class members
-// and ties at the threshold taken from the lowest indices.
+// The k-th largest key T is found either by sorting a prefiltered candidate set
+// (warp_topk_select) or by bisection on the key bits with warp-wide counts; the list is
+// then written in ascending block order with forced blocks first-class members and
+// ties at the threshold taken from the lowest indices.  When every key equal to T is
+// taken (the usual case: no duplicate straddles the cut), a block is taken exactly when
+// forced or key >= T, and the emission needs no tie ranks.
 #pragma once
 #include "common.cuh"
 
 namespace infllmv2 {
 
 struct TopkThreshold {
-  uint32_t key;  // threshold key T (0xffffffff when nothing is to be taken)
-  int ties;      // how many keys equal to T are taken (0 when T == 0: take all > 0)
+  uint32_t key;   // threshold key T (0xffffffff when nothing is to be taken)
+  int ties;       // how many keys equal to T are taken (0 when T == 0: take all > 0)
+  bool all_ties;  // every key equal to T is taken
 };
+
+// Smallest key taken without a tie rank: every key >= take_from(th) is taken when
+// th.all_ties, T == 0 (all candidates) or T == 0xffffffff (none: keys stay below it).
+__device__ __forceinline__ bool topk_simple(const TopkThreshold& th) {
+  return th.all_ties || th.key == 0u || th.key == 0xffffffffu;
+}
+__device__ __forceinline__ uint32_t take_from(const TopkThreshold& th) { return th.key == 0u ? 1u : th.key; }
 
 // One warp.  keys[0..n) in shared memory; `want` keys to take.  Finds the want-th
 // largest key T by bisection on its bits, most significant first: T >= c exactly when
@@ -43,6 +54,7 @@ __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* ke
                                                               uint32_t* /*unused scratch*/) {
   const int lane = threadIdx.x & 31;
   TopkThreshold r;
+  r.all_ties = false;
   if (want <= 0) {
     r.key = 0xffffffffu;
     r.ties = 0;
@@ -85,14 +97,92 @@ __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* ke
   return r;
 }
 
+// Descending bitonic sort of 256 keys held 8 per lane (element i = 8 lane + e): 36
+// compare-exchange stages, the 21 with stride < 8 inside a lane, the 15 others across
+// lanes by shuffles.
+__device__ __forceinline__ void warp_bitonic256_desc(uint32_t (&a)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 256; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 8) {
+        const int lj = j >> 3;
+        const bool keep_max = ((lane & lj) == 0) == (((lane * 8) & k) == 0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t b = __shfl_xor_sync(0xffffffffu, a[e], lj);
+          a[e] = keep_max ? max(a[e], b) : min(a[e], b);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if ((e & j) == 0) {
+            const int f = e | j;
+            const bool up = (((lane * 8) + e) & k) == 0;
+            const uint32_t x = a[e], y = a[f];
+            a[e] = up ? max(x, y) : min(x, y);
+            a[f] = up ? min(x, y) : max(x, y);
+          }
+        }
+      }
+    }
+  }
+}
+
+// One warp writes the selected blocks of one row, ascending, padded with -1, from keys
+// held in registers (key j = kr[i] with j = 32 i + lane, j < n).  Block j is taken when
+// forced, or key > T, or key == T among the first `ties` such keys (ascending j).
+__device__ __forceinline__ void warp_emit_regs(const uint32_t (&kr)[kTopkRegKeys], int n, const TopkThreshold& th,
+                                               int cur, int n_init, int n_local, int topk, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  int written = 0;
+  if (topk_simple(th)) {
+    const uint32_t lo = take_from(th);
+#pragma unroll
+    for (int i = 0; i < kTopkRegKeys; ++i) {
+      if (32 * i < n) {
+        const int j = 32 * i + lane;
+        const bool take = j < n && (j < n_init || j > cur - n_local || kr[i] >= lo);
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        const int pos = written + __popc(m & lt);
+        if (take && pos < topk) out[pos] = j;
+        written += __popc(m);
+      }
+    }
+  } else {
+    int ties_seen = 0;
+#pragma unroll
+    for (int i = 0; i < kTopkRegKeys; ++i) {
+      if (32 * i < n) {
+        const int j = 32 * i + lane;
+        const bool in = j < n;
+        const uint32_t k = kr[i];
+        const bool forced = in && (j < n_init || j > cur - n_local);
+        const bool tie = in && k == th.key;
+        const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
+        const int tie_rank = ties_seen + __popc(tie_mask & lt);
+        const bool take = forced || (in && k > th.key) || (tie && tie_rank < th.ties);
+        const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+        const int pos = written + __popc(take_mask & lt);
+        if (take && pos < topk) out[pos] = j;
+        written += __popc(take_mask);
+        ties_seen += __popc(tie_mask);
+      }
+    }
+  }
+  for (int q = written + lane; q < topk; q += 32) out[q] = -1;
+}
+
 // One warp: threshold and ordered emission for n <= 32 * kTopkRegKeys keys, with the
-// keys held in registers (key j = keys[lane + 32 i] in kr[i]).  The search is narrowed
-// first: every lane keeps its 4 largest keys; with r = ceil(want / 32) <= 4, c0 = the
-// warp minimum of the lanes' r-th largest keys bounds the threshold from below (each
-// lane holds r keys >= c0, so at least 32 r >= want keys are >= c0).  Only the keys
-// >= c0 (usually a few hundred) are copied to `cand` (kTopkCand words of this warp's
-// shared scratch) and bisected; when the bound does not apply or too many keys pass it,
-// the search runs over all keys.  Same result either way: the want-th largest key.
+// keys held in registers.  The search is narrowed first: every lane keeps its 4 largest
+// keys; with r = ceil(want / 32) <= 4, c0 = the warp minimum of the lanes' r-th largest
+// keys bounds the threshold from below (each lane holds r keys >= c0, so at least
+// 32 r >= want keys are >= c0).  The keys >= c0 (usually a few hundred) are compacted
+// into `cand` (kTopkCand words of this warp's shared scratch) and sorted; T is the
+// want-th of them.  When the bound does not apply or too many keys pass it, T comes from
+// bisection over all keys.  Same result either way: the want-th largest key.
 constexpr int kTopkCand = 256;
 
 __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, int want, int cur, int n_init,
@@ -106,100 +196,83 @@ __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, in
     kr[i] = j < n ? keys[j] : 0u;
   }
   TopkThreshold th;
+  th.all_ties = false;
   if (want <= 0) {
     th.key = 0xffffffffu;
     th.ties = 0;
-  } else if (warp_count_ge_regs(kr, 1u) <= want) {
-    th.key = 0;
-    th.ties = 0;
   } else {
-    // lower bound c0 from each lane's r-th largest key
+    // per-lane top 4 and candidate count in one pass
     const int r = (want + 31) / 32;
-    uint32_t c0 = 0;
-    if (r <= 4) {
-      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;  // descending top-4 of this lane
+    uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
+    int c1 = 0;
 #pragma unroll
-      for (int i = 0; i < kTopkRegKeys; ++i) {
-        uint32_t x = kr[i], y;
-        y = max(x, t0); x = min(x, t0); t0 = y;
-        y = max(x, t1); x = min(x, t1); t1 = y;
-        y = max(x, t2); x = min(x, t2); t2 = y;
-        t3 = max(x, t3);
-      }
-      const uint32_t cl = r == 1 ? t0 : (r == 2 ? t1 : (r == 3 ? t2 : t3));
-      c0 = __reduce_min_sync(0xffffffffu, cl);
+    for (int i = 0; i < kTopkRegKeys; ++i) {
+      uint32_t x = kr[i], y;
+      c1 += x != 0u ? 1 : 0;
+      y = max(x, t0); x = min(x, t0); t0 = y;
+      y = max(x, t1); x = min(x, t1); t1 = y;
+      y = max(x, t2); x = min(x, t2); t2 = y;
+      t3 = max(x, t3);
     }
-    int nc = c0 > 0 ? warp_count_ge_regs(kr, c0) : kTopkCand + 1;
-    uint32_t T = 0;
-    if (nc <= kTopkCand) {
-      int base = 0;
-#pragma unroll
-      for (int i = 0; i < kTopkRegKeys; ++i) {
-        const bool in = kr[i] >= c0;
-        const unsigned msk = __ballot_sync(0xffffffffu, in);
-        if (in) cand[base + __popc(msk & lt)] = kr[i];
-        base += __popc(msk);
-      }
-      __syncwarp();
-      uint32_t cr[kTopkCand / 32];
-#pragma unroll
-      for (int i = 0; i < kTopkCand / 32; ++i) {
-        const int j = lane + 32 * i;
-        cr[i] = j < nc ? cand[j] : 0u;
-      }
-      __syncwarp();
-#pragma unroll 1
-      for (int bit = 30; bit >= 0; --bit) {
-        const uint32_t c = T | (1u << bit);
-        bool ok = c <= c0;  // every c <= c0 has >= want keys above it
-        if (!ok) {
-          int cnt = 0;
-#pragma unroll
-          for (int i = 0; i < kTopkCand / 32; ++i) cnt += cr[i] >= c ? 1 : 0;
-          ok = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt))) >= want;
-        }
-        if (ok) T = c;
-      }
-      int above = 0;
-#pragma unroll
-      for (int i = 0; i < kTopkCand / 32; ++i) above += cr[i] > T ? 1 : 0;
-      th.key = T;
-      th.ties = want - static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(above)));
+    const int ncand = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c1)));
+    if (ncand <= want) {  // at most `want` candidates: take them all
+      th.key = 0;
+      th.ties = 0;
     } else {
-#pragma unroll 1
-      for (int bit = 30; bit >= 0; --bit) {
-        const uint32_t c = T | (1u << bit);
-        if (warp_count_ge_regs(kr, c) >= want) T = c;
-      }
-      th.key = T;
-      th.ties = want - warp_count_ge_regs(kr, T + 1u);
-    }
-  }
-  // emission in ascending block order, straight from the registers
-  int written = 0, ties_seen = 0;
+      uint32_t c0 = 0;
+      if (r <= 4) c0 = __reduce_min_sync(0xffffffffu, r == 1 ? t0 : (r == 2 ? t1 : (r == 3 ? t2 : t3)));
+      int nc = kTopkCand + 1;
+      if (c0 > 0) {
+        int base = 0;
 #pragma unroll
-  for (int i = 0; i < kTopkRegKeys; ++i) {
-    if (32 * i < n) {
-      const int j = 32 * i + lane;
-      const bool in = j < n;
-      const uint32_t k = kr[i];
-      const bool forced = in && (j < n_init || j > cur - n_local);
-      const bool tie = in && th.key != 0u && k == th.key;
-      const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
-      const int tie_rank = ties_seen + __popc(tie_mask & lt);
-      bool take;
-      if (th.key == 0u)
-        take = forced || (in && k > 0u);
-      else
-        take = forced || (in && k > th.key && th.key != 0xffffffffu) || (tie && tie_rank < th.ties);
-      const unsigned take_mask = __ballot_sync(0xffffffffu, take);
-      const int pos = written + __popc(take_mask & lt);
-      if (take && pos < topk) out[pos] = j;
-      written += __popc(take_mask);
-      ties_seen += __popc(tie_mask);
+        for (int i = 0; i < kTopkRegKeys; ++i) {
+          const bool in = kr[i] >= c0;
+          const unsigned m = __ballot_sync(0xffffffffu, in);
+          const int pos = base + __popc(m & lt);
+          if (in && pos < kTopkCand) cand[pos] = kr[i];
+          base += __popc(m);
+        }
+        nc = base;
+        __syncwarp();
+      }
+      if (nc <= kTopkCand) {
+        uint32_t a[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int idx = 8 * lane + e;
+          a[e] = idx < nc ? cand[idx] : 0u;
+        }
+        __syncwarp();
+        warp_bitonic256_desc(a);
+        const int wl = (want - 1) >> 3, we = (want - 1) & 7;
+        uint32_t v = a[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e) v = e == we ? a[e] : v;
+        const uint32_t T = __shfl_sync(0xffffffffu, v, wl);
+        int above = 0, eq = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          above += a[e] > T ? 1 : 0;
+          eq += a[e] == T ? 1 : 0;
+        }
+        above = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(above)));
+        eq = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(eq)));
+        th.key = T;
+        th.ties = want - above;
+        th.all_ties = above + eq == want;
+      } else {
+        uint32_t T = 0;
+#pragma unroll 1
+        for (int bit = 30; bit >= 0; --bit) {
+          const uint32_t c = T | (1u << bit);
+          if (warp_count_ge_regs(kr, c) >= want) T = c;
+        }
+        th.key = T;
+        th.ties = want - warp_count_ge_regs(kr, T + 1u);
+      }
     }
   }
-  for (int q = written + lane; q < topk; q += 32) out[q] = -1;
+  warp_emit_regs(kr, n, th, cur, n_init, n_local, topk, out);
 }
 
 // One warp writes the selected blocks of one row, ascending, padded with -1.
@@ -209,25 +282,28 @@ __device__ __forceinline__ void warp_emit_selection(const uint32_t* keys, int n,
                                                     int n_init, int n_local, int topk, int32_t* out) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
+  const bool simple = topk_simple(th);
+  const uint32_t lo = take_from(th);
   int written = 0, ties_seen = 0;
   for (int b0 = 0; b0 < n; b0 += 32) {
     const int j = b0 + lane;
     const bool in = j < n;
     const uint32_t k = in ? keys[j] : 0u;
     const bool forced = in && (j < n_init || j > cur - n_local);
-    const bool tie = in && th.key != 0u && k == th.key;
-    const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
-    const int tie_rank = ties_seen + __popc(tie_mask & lt);
     bool take;
-    if (th.key == 0u)
-      take = forced || (in && k > 0u);
-    else
-      take = forced || (in && k > th.key && th.key != 0xffffffffu) || (tie && tie_rank < th.ties);
+    if (simple) {
+      take = forced || (in && k >= lo);
+    } else {
+      const bool tie = in && k == th.key;
+      const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
+      const int tie_rank = ties_seen + __popc(tie_mask & lt);
+      take = forced || (in && k > th.key) || (tie && tie_rank < th.ties);
+      ties_seen += __popc(tie_mask);
+    }
     const unsigned take_mask = __ballot_sync(0xffffffffu, take);
     const int pos = written + __popc(take_mask & lt);
     if (take && pos < topk) out[pos] = j;
     written += __popc(take_mask);
-    ties_seen += __popc(tie_mask);
   }
   for (int q = written + lane; q < topk; q += 32) out[q] = -1;
 }
