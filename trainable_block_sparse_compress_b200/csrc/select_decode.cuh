@@ -36,6 +36,8 @@ constexpr int kSdMaxChunk = 2048;  // kernels per CTA at most
 constexpr int kSdMaxQuads = kSdMaxChunk / 4;
 constexpr int kSdBStride = kSdMaxQuads + 4;  // per-head block-max rows (quads + 1 carry), padded
 constexpr int kSdMaxCluster = 16;
+// CTA 0's top-k visits the keys slot-major: thread i takes keys i + kSdThreads s.
+constexpr int kSdMaxR = (INFLLMV2_MAX_SEQ_LEN / kBlock + kSdThreads - 1) / kSdThreads;
 static_assert(kSdStages * kKcTileBytes >= 4 * (INFLLMV2_MAX_SEQ_LEN / kBlock),
               "the block keys of CTA 0 reuse its tile ring");
 static_assert(kSdMaxCluster * kSdMaxChunk >= (INFLLMV2_MAX_SEQ_LEN - kKernel) / kStride + 1,
@@ -57,7 +59,10 @@ struct SdSmem {
   float lse2[kGroupRows];  // log2-sum-exp2 per head over the whole sequence
   float carry[kGroupRows];  // previous CTA's last kernel, for this CTA's first block
   int cnt[2][kSdWarps][32];
-  int scan[2][kSdWarps];
+  int wc[kSdMaxR][kSdWarps];          // per (slot, warp) counts of the emission
+  int sbase[kSdMaxR];                 // flagged keys in earlier slots
+  int total;
+  unsigned char tflag[kSdMaxR][kSdThreads];  // take flags when tie ranks are needed
   int nlist;
   uint32_t list[32];
   volatile int abort;
@@ -78,19 +83,56 @@ __device__ __forceinline__ float ord_dec(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ int ge4(const uint4 v, uint32_t c) {
-  return (v.x >= c ? 1 : 0) + (v.y >= c ? 1 : 0) + (v.z >= c ? 1 : 0) + (v.w >= c ? 1 : 0);
+// For each lane l: how many of this warp's keys (thread i takes keys i + kSdThreads s,
+// s < R) are >= T | l << shift, where the bits of T below shift + w are zero and l < 2^w
+// (lanes l >= 2^w count the keys at or above T + 2^(shift + w), the bucket's upper end).
+// `first`: lane 0 counts the keys >= 1 instead (the candidates).  Bit-sliced: one
+// ballot per digit bit and slot, then a comparison of the lane's digit l against every
+// key's digit on the ballot masks.
+__device__ __forceinline__ int warp_count_digits(const uint32_t* keys, int n, int R, uint32_t T, int shift, int w,
+                                                 bool first) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t hT = T >> (shift + w);
+  const uint32_t dmask = (1u << w) - 1u;
+  int cnt = 0;
+#pragma unroll 2
+  for (int s = 0; s < R; ++s) {
+    const int j = static_cast<int>(threadIdx.x) + kSdThreads * s;
+    const uint32_t k = j < n ? keys[j] : 0u;
+    const uint32_t hk = k >> (shift + w);
+    const bool in = hk == hT;
+    const uint32_t d = (k >> shift) & dmask;
+    const unsigned A = __ballot_sync(0xffffffffu, hk > hT);
+    unsigned gt = 0u, eq = __ballot_sync(0xffffffffu, in);
+#pragma unroll
+    for (int i = 4; i >= 0; --i) {
+      if (i < w) {
+        const unsigned Bi = __ballot_sync(0xffffffffu, in && ((d >> i) & 1u));
+        const unsigned tt = eq & Bi;
+        const bool one = (lane >> i) & 1;
+        gt = one ? gt : (gt | tt);
+        eq = one ? tt : (eq & ~Bi);
+      }
+    }
+    int c = __popc(A) + (lane < (1 << w) ? __popc(gt | eq) : 0);
+    if (first) {
+      const int cand = __popc(__ballot_sync(0xffffffffu, k != 0u));
+      if (lane == 0) c = cand;
+    }
+    cnt += c;
+  }
+  return cnt;
 }
 
-// k-th largest of n keys in shared memory (zero-padded to a multiple of 4) by all
-// kSdThreads threads; same result as warp_radix_threshold.  Radix search on the 31 key
-// bits in digits of 5 (the last one 1): lane l of every warp counts the keys >= T | l <<
-// shift over the warp's share, the counts meet in S.cnt (double-buffered: one barrier per
-// digit) and the largest digit with at least `want` keys at or above it is taken.  As
-// soon as the chosen digit's bucket holds at most 32 keys, they are gathered and ranked
-// directly.
+// k-th largest of the n keys in shared memory by all kSdThreads threads; same result as
+// warp_radix_threshold.  Radix search on the 31 key bits in digits of 5 (the last one
+// 1): lane l of every warp counts the keys >= T | l << shift (warp_count_digits), the
+// counts meet in S.cnt (double-buffered: one barrier per digit) and the largest digit
+// with at least `want` keys at or above it is taken.  As soon as the chosen digit's
+// bucket holds at most 32 keys, they are gathered and ranked directly.
 __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys, int n, int want, SdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int R = (n + kSdThreads - 1) / kSdThreads;
   TopkThreshold r;
   r.all_ties = false;
   if (want <= 0) {
@@ -98,31 +140,18 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     r.ties = 0;
     return r;
   }
-  const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-  const int n4 = (n + 3) >> 2;
   int buf = 0;
-  auto count_ge = [&](uint32_t c) -> int {
-    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-    int i = warp;
-#pragma unroll 1
-    for (; i + 3 * kSdWarps < n4; i += 4 * kSdWarps) {
-      const uint4 v0 = k4[i], v1 = k4[i + kSdWarps], v2 = k4[i + 2 * kSdWarps], v3 = k4[i + 3 * kSdWarps];
-      a0 += ge4(v0, c);
-      a1 += ge4(v1, c);
-      a2 += ge4(v2, c);
-      a3 += ge4(v3, c);
-    }
-    for (; i < n4; i += kSdWarps) a0 += ge4(k4[i], c);
-    S.cnt[buf][warp][lane] = (a0 + a1) + (a2 + a3);
+  auto count_ge = [&](uint32_t T, int shift, int w, bool first) -> int {
+    S.cnt[buf][warp][lane] = warp_count_digits(keys, n, R, T, shift, w, first);
     __syncthreads();
     int tot = 0;
 #pragma unroll
-    for (int w = 0; w < kSdWarps; ++w) tot += S.cnt[buf][w][lane];
+    for (int ww = 0; ww < kSdWarps; ++ww) tot += S.cnt[buf][ww][lane];
     buf ^= 1;
     return tot;
   };
   // first digit (bits 30..26); lane 0 counts the candidates (keys >= 1): bucket 0 is [1, 2^26)
-  int tot = count_ge(lane == 0 ? 1u : static_cast<uint32_t>(lane) << 26);
+  int tot = count_ge(0u, 26, 5, true);
   if (__shfl_sync(0xffffffffu, tot, 0) <= want) {  // at most `want` candidates: take them all
     r.key = 0;
     r.ties = 0;
@@ -138,9 +167,9 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     inb = __shfl_sync(0xffffffffu, tot, l) - above;
     T |= static_cast<uint32_t>(l) << shift;
     if (inb <= 32 || shift == 0) break;
-    shift = shift > 5 ? shift - 5 : 0;
-    // the last digit is bit 0 alone: lanes >= 2 test the bucket's upper end (count = above)
-    tot = count_ge(shift > 0 ? T | (static_cast<uint32_t>(lane) << shift) : (lane < 2 ? T | lane : T + 2u));
+    const int w = shift > 5 ? 5 : 1;  // 26, 21, 16, 11, 6, 1 (5 bits each), then bit 0
+    shift -= w;
+    tot = count_ge(T, shift, w, false);
   }
   if (shift == 0) {  // the bucket is the single value T
     r.key = T;
@@ -174,67 +203,99 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   return r;
 }
 
-// Exclusive prefix sum of v over the kSdThreads threads (thread order); *total gets the
-// sum.  buf holds kSdWarps ints and must not be in use by another scan.
-__device__ __forceinline__ int cta_exclusive_scan(int v, int* buf, int* total) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) buf[warp] = x;
-  __syncthreads();
-  int base = 0, sum = 0;
-#pragma unroll
-  for (int w = 0; w < kSdWarps; ++w) {
-    base += w < warp ? buf[w] : 0;
-    sum += buf[w];
-  }
-  *total = sum;
-  return base + x - v;
-}
-
 // All kSdThreads threads write the selected blocks of one row, ascending, padded with
 // -1: block j in [0, n) is taken when forced, or key > T, or key == T among the first
-// `ties` such keys in ascending j (the rule of warp_emit_selection).  Thread i scans the
-// contiguous keys [i s, (i + 1) s); two prefix sums place the tie ranks and the outputs.
+// `ties` such keys in ascending j (the rule of warp_emit_selection).  Keys are visited
+// slot-major (thread i, slot s: key i + kSdThreads s), which is ascending j: one pass
+// counts the taken keys per (slot, warp) with ballots, a warp scan turns the slot totals
+// into slot bases, and a second pass writes each taken key at its base plus its rank in
+// the warp and in the slot.  Tie ranks (only when some keys equal to T stay out) come
+// from the same two passes run on the tie flags first.
 __device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, TopkThreshold th, int cur,
-                                                   int n_init, int n_local, int topk, int32_t* out,
-                                                   int (*scan)[kSdWarps]) {
-  const int seg = (n + kSdThreads - 1) / kSdThreads;
-  const int j0 = min(static_cast<int>(threadIdx.x) * seg, n), j1 = min(j0 + seg, n);
+                                                   int n_init, int n_local, int topk, int32_t* out, SdSmem& S) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int R = (n + kSdThreads - 1) / kSdThreads;
   const bool simple = topk_simple(th);  // no tie ranks needed: take forced or key >= lo
   const uint32_t lo = take_from(th);
-  int my_ties = 0;
-  if (!simple)
-    for (int j = j0; j < j1; ++j) my_ties += keys[j] == th.key ? 1 : 0;
-  int total = 0;
-  const int tie0 = simple ? 0 : cta_exclusive_scan(my_ties, scan[0], &total);
-  auto take = [&](int j, uint32_t k, int& tr) -> bool {
-    const bool forced = j < n_init || j > cur - n_local;
-    if (simple) return forced || k >= lo;
-    const bool tie = k == th.key;
-    const bool t = forced || k > th.key || (tie && tr < th.ties);
-    if (tie) ++tr;
-    return t;
-  };
-  int my_take = 0;
-  {
-    int tr = tie0;
-    for (int j = j0; j < j1; ++j) my_take += take(j, keys[j], tr) ? 1 : 0;
-  }
-  int pos = cta_exclusive_scan(my_take, scan[1], &total);
-  {
-    int tr = tie0;
-    for (int j = j0; j < j1; ++j)
-      if (take(j, keys[j], tr)) {
-        if (pos < topk) out[pos] = j;
-        ++pos;
+  // per (slot, warp) counts of a flag, then S.sbase[s] = flagged keys in slots < s
+  auto slot_counts = [&](auto flag) -> int {
+    for (int s = 0; s < R; ++s) {
+      const unsigned m = __ballot_sync(0xffffffffu, flag(s));
+      if (lane == 0) S.wc[s][warp] = __popc(m);
+    }
+    __syncthreads();
+    int total = 0;
+    if (warp == 0) {
+      int v = 0;
+      if (lane < R)
+#pragma unroll
+        for (int ww = 0; ww < kSdWarps; ++ww) v += S.wc[lane][ww];
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
+      if (lane < R) S.sbase[lane] = incl - v;
+      if (lane == 31) S.total = incl;
+    }
+    __syncthreads();
+    total = S.total;
+    return total;
+  };
+  auto rank_of = [&](int s, unsigned m) -> int {  // flagged keys before this thread's key of slot s
+    int before = S.sbase[s];
+#pragma unroll
+    for (int ww = 0; ww < kSdWarps; ++ww) before += ww < warp ? S.wc[s][ww] : 0;
+    return before + __popc(m & lt);
+  };
+  auto key_at = [&](int s, int& j) -> uint32_t {
+    j = static_cast<int>(threadIdx.x) + kSdThreads * s;
+    return j < n ? keys[j] : 0u;
+  };
+  auto forced = [&](int j) { return j < n && (j < n_init || j > cur - n_local); };
+  if (simple) {
+    auto take = [&](int s) {
+      int j;
+      const uint32_t k = key_at(s, j);
+      return j < n && (forced(j) || k >= lo);
+    };
+    const int total = slot_counts(take);
+    for (int s = 0; s < R; ++s) {
+      const bool f = take(s);
+      const int pos = rank_of(s, __ballot_sync(0xffffffffu, f));
+      if (f && pos < topk) out[pos] = static_cast<int>(threadIdx.x) + kSdThreads * s;
+    }
+    for (int e = total + static_cast<int>(threadIdx.x); e < topk; e += kSdThreads) out[e] = -1;
+    __syncthreads();  // S.wc, S.sbase are free again
+    return;
+  }
+  // tie ranks first: S.tie_base[s] + warp part, recomputed per slot below
+  auto tie = [&](int s) {
+    int j;
+    const uint32_t k = key_at(s, j);
+    return j < n && k == th.key;
+  };
+  slot_counts(tie);
+  for (int s = 0; s < R; ++s) {  // keep each slot's tie base for this thread's warp
+    const bool f = tie(s);
+    const int rk = rank_of(s, __ballot_sync(0xffffffffu, f));
+    int j;
+    const uint32_t k = key_at(s, j);
+    S.tflag[s][threadIdx.x] = static_cast<unsigned char>(
+        j < n && (forced(j) || k > th.key || (k == th.key && rk < th.ties)) ? 1 : 0);
+  }
+  __syncthreads();
+  auto take = [&](int s) { return S.tflag[s][threadIdx.x] != 0; };
+  const int total = slot_counts(take);
+  for (int s = 0; s < R; ++s) {
+    const bool f = take(s);
+    const int pos = rank_of(s, __ballot_sync(0xffffffffu, f));
+    if (f && pos < topk) out[pos] = static_cast<int>(threadIdx.x) + kSdThreads * s;
   }
   for (int e = total + static_cast<int>(threadIdx.x); e < topk; e += kSdThreads) out[e] = -1;
+  __syncthreads();
 }
 
 // grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.
@@ -454,7 +515,7 @@ __global__ void __launch_bounds__(kSdThreads)
   }
   const int want = p.topk - forced_count(cur, p.n_init, p.n_local);
   const TopkThreshold th = cta_topk_threshold(keys, cur + 1, want, S);
-  cta_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out, S.scan);
+  cta_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out, S);
 }
 
 }  // namespace infllmv2
