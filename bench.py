@@ -29,6 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from trainable_block_sparse_compress_b200 import build as lib_build  # noqa: E402
+from trainable_block_sparse_compress_b200 import dist  # noqa: E402
 from trainable_block_sparse_compress_b200 import ops  # noqa: E402
 from trainable_block_sparse_compress_b200.synthetic import WORKLOADS, as_u16, make_inputs  # noqa: E402
 
@@ -164,7 +165,7 @@ def run_ours(args, rank, world, device):
     wl = WORKLOADS[args.workload]
     p = ops.Params.from_workload(wl)
     L = wl.seq_len
-    x = make_inputs(wl, seed=args.seed + rank)
+    x = make_inputs(wl, seed=dist.rank_seed(args.seed, rank))
     q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
     nk = ops.num_kernels(p, L)
     kc = torch.empty((p.batch, p.num_kv_heads, nk, p.head_dim), dtype=torch.bfloat16, device=device)
@@ -198,8 +199,7 @@ def run_ours(args, rank, world, device):
                for i, n in enumerate(names)}
 
     # the timed region: exactly K steps, barrier + synchronize on both sides
-    if world > 1:
-        torch.distributed.barrier()
+    dist.barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -209,16 +209,11 @@ def run_ours(args, rank, world, device):
             step()
         t1.record(stream)
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    ms = t0.elapsed_time(t1)
-    ms_t = torch.tensor([ms], device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    dist.barrier(world)
+    ms = dist.max_over_ranks(t0.elapsed_time(t1), world, device)
     ms_per_step = ms / args.steps
     tokens_per_step = p.batch * L
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = dist.weak_scaling_rate(world, tokens_per_step, args.steps, ms / 1e3)
 
     sel_flops, attn_flops, gather_bytes = prefill_flops(p, L)
     comp_bytes = p.batch * p.num_kv_heads * (L + nk) * p.head_dim * 2
@@ -320,7 +315,7 @@ def run_decode(args, rank, world, device, pk, peak_src):
     every step (outside the timed events)."""
     wl = WORKLOADS[args.decode_workload]
     p = ops.Params.from_workload(wl)
-    x = make_inputs(wl, seed=args.seed + 1000 + rank)
+    x = make_inputs(wl, seed=dist.rank_seed(args.seed + 1000, rank))
     Lmax = wl.seq_len
     q, k, v, lens = x.q.to(device), x.k.to(device), x.v.to(device), x.lens.to(device)
     kc = ops.compress_keys(p, k, lens=lens)  # cache maintenance, not timed
@@ -368,10 +363,7 @@ def run_decode(args, rank, world, device, pk, peak_src):
     sel_us = [evk[s][0].elapsed_time(evk[s][1]) * 1e3 for s in range(n)]
     att_us = [evk[s][1].elapsed_time(evk[s][2]) * 1e3 for s in range(n)]
     us = statistics.median(step_us)
-    us_t = torch.tensor([us], device=device)
-    if world > 1:
-        torch.distributed.all_reduce(us_t, op=torch.distributed.ReduceOp.MAX)
-    us = float(us_t.item())
+    us = dist.max_over_ranks(us, world, device)
     sel_b, att_b = decode_bytes(p, x.lens.numpy())
     att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
@@ -476,9 +468,8 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ri = dist.rank_info()
+    rank, world, local = ri.rank, ri.world, ri.local
 
     if args.impl == "reference":
         if rank == 0:
