@@ -34,6 +34,7 @@ __device__ __forceinline__ uint32_t take_from(const TopkThreshold& th) { return 
 // at least `want` keys are >= c.  Each lane holds up to kTopkRegKeys keys in registers
 // (n <= 32 * kTopkRegKeys); larger n re-reads shared memory each step.  No atomics.
 constexpr int kTopkRegKeys = 64;
+constexpr int kTopkVoteBatch = 16;  // ballots issued back to back before their stores
 
 __device__ __forceinline__ int warp_count_ge_regs(const uint32_t (&kr)[kTopkRegKeys], uint32_t c) {
   int cnt[4] = {0, 0, 0, 0};  // four independent chains
@@ -139,16 +140,24 @@ __device__ __forceinline__ void warp_emit_regs(const uint32_t (&kr)[kTopkRegKeys
   const unsigned lt = (1u << lane) - 1u;
   int written = 0;
   if (topk_simple(th)) {
+    // 16 ballots first, then their stores: the votes pipeline instead of alternating
+    // with dependent stores
     const uint32_t lo = take_from(th);
 #pragma unroll
-    for (int i = 0; i < kTopkRegKeys; ++i) {
-      if (32 * i < n) {
-        const int j = 32 * i + lane;
-        const bool take = j < n && (j < n_init || j > cur - n_local || kr[i] >= lo);
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        const int pos = written + __popc(m & lt);
-        if (take && pos < topk) out[pos] = j;
-        written += __popc(m);
+    for (int g = 0; g < kTopkRegKeys; g += kTopkVoteBatch) {
+      if (32 * g < n) {
+        unsigned m[kTopkVoteBatch];
+#pragma unroll
+        for (int u = 0; u < kTopkVoteBatch; ++u) {
+          const int j = 32 * (g + u) + lane;
+          m[u] = __ballot_sync(0xffffffffu, j < n && (j < n_init || j > cur - n_local || kr[g + u] >= lo));
+        }
+#pragma unroll
+        for (int u = 0; u < kTopkVoteBatch; ++u) {
+          const int pos = written + __popc(m[u] & lt);
+          if (((m[u] >> lane) & 1u) && pos < topk) out[pos] = 32 * (g + u) + lane;
+          written += __popc(m[u]);
+        }
       }
     }
   } else {
@@ -225,12 +234,16 @@ __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, in
       if (c0 > 0) {
         int base = 0;
 #pragma unroll
-        for (int i = 0; i < kTopkRegKeys; ++i) {
-          const bool in = kr[i] >= c0;
-          const unsigned m = __ballot_sync(0xffffffffu, in);
-          const int pos = base + __popc(m & lt);
-          if (in && pos < kTopkCand) cand[pos] = kr[i];
-          base += __popc(m);
+        for (int g = 0; g < kTopkRegKeys; g += kTopkVoteBatch) {
+          unsigned m[kTopkVoteBatch];
+#pragma unroll
+          for (int u = 0; u < kTopkVoteBatch; ++u) m[u] = __ballot_sync(0xffffffffu, kr[g + u] >= c0);
+#pragma unroll
+          for (int u = 0; u < kTopkVoteBatch; ++u) {
+            const int pos = base + __popc(m[u] & lt);
+            if (((m[u] >> lane) & 1u) && pos < kTopkCand) cand[pos] = kr[g + u];
+            base += __popc(m[u]);
+          }
         }
         nc = base;
         __syncwarp();
