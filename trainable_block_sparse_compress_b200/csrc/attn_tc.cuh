@@ -7,11 +7,11 @@
 //
 // Work item = (sequence b, kv-head g, query token t).  The item's selected blocks are
 // taken in pairs (128 keys); a persistent CTA streams them with TMA (128-byte swizzle, no
-// multicast) through two 3-slot rings of 32 KB, one for K pairs (warp 8) and one for V
+// multicast) through two rings of 32 KB slots, one for K pairs (warp 8) and one for V
 // pairs (warp 11), so a K slot is free again right after its QK and a V slot right
 // after its PV; per pair:
 //   warp 9 (one thread) issues  S^T = K_pair . Q^T   (UMMA M128 N16 K128: keys x heads)
-//          into one of two TMEM score buffers as soon as the pair has landed;
+//          into one of six TMEM score buffers as soon as the pair has landed;
 //   warp 10 (one thread) issues, as soon as P is in shared memory,
 //          O^T += V^T . P^T   (UMMA M128 N16 K128: V read through an MN-major
 //          descriptor, P K-major) into the TMEM output buffer of the pair's warpgroup.
@@ -33,7 +33,8 @@
 
 namespace infllmv2 {
 
-constexpr int kAtStages = 3;                       // slots per ring (K ring and V ring)
+constexpr int kAtKStages = 3;                      // slots of the K ring
+constexpr int kAtVStages = 2;                      // slots of the V ring
 constexpr int kAtKHalf = 2 * kKvTileBytes / 2;     // 16 KB: one 64-column half of 128 keys
 constexpr int kAtSlotBytes = 2 * kKvTileBytes;     // 32 KB: a pair of K (or V) blocks
 constexpr int kAtPBytes = kGroupRows * 128 * 2;    // 4 KB: P (16 heads x 128 keys bf16)
@@ -41,12 +42,14 @@ constexpr int kAtSoftWGs = 2;
 constexpr int kAtThreads = 32 * (4 * kAtSoftWGs + 4);
 constexpr int kAtTmaWarp = 4 * kAtSoftWGs, kAtMmaWarp = kAtTmaWarp + 1, kAtPvWarp = kAtTmaWarp + 2,
               kAtVTmaWarp = kAtTmaWarp + 3;
-constexpr int kAtBufs = 4;             // score (TMEM) and probability (shared) buffers in flight
-constexpr uint32_t kAtTmemCols = 128;  // scores S[4] at 16 s; outputs O[item parity][wg] at 64 + 16 (2 it + wg)
+constexpr int kAtBufs = 6;  // score (TMEM) and probability (shared) buffers in flight
+// TMEM columns: scores S[b] at 16 b, outputs O[item parity][wg] at 16 kAtBufs + 16 (2 it + wg);
+// the allocation is the next power of two
 constexpr uint32_t kAtOCol = 16 * kAtBufs;
+constexpr uint32_t kAtTmemCols = kAtOCol + 64 <= 128 ? 128 : (kAtOCol + 64 <= 256 ? 256 : 512);
 
 struct AtSmem {
-  uint64_t k_full[kAtStages], k_empty[kAtStages], v_full[kAtStages], v_empty[kAtStages], q_full[2], q_empty[2];
+  uint64_t k_full[kAtKStages], k_empty[kAtKStages], v_full[kAtVStages], v_empty[kAtVStages], q_full[2], q_empty[2];
   uint64_t s_full[kAtBufs], p_full[kAtBufs], pv_done[kAtBufs], mma_done[2];
   int n_blocks[2];
   int list[2][kMaxTopk];
@@ -58,9 +61,10 @@ struct AtSmem {
 };
 
 constexpr size_t attn_tc_smem_bytes() {
-  return 1024 + 2 * static_cast<size_t>(kAtStages) * kAtSlotBytes + 2 * kQTileBytes + kAtBufs * kAtPBytes +
+  return 1024 + static_cast<size_t>(kAtKStages + kAtVStages) * kAtSlotBytes + 2 * kQTileBytes + kAtBufs * kAtPBytes +
          sizeof(AtSmem);
 }
+static_assert(attn_tc_smem_bytes() <= 227 * 1024, "shared memory of one CTA");
 
 // Per-lane result of a 32-lane max / sum over 16 values: lane L holds the total for
 // value index L >> 1 (lanes 2h and 2h+1 agree).  16 shuffles.
@@ -121,16 +125,18 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = align_smem(smem_raw, 1024);
   unsigned char* kring = base;
-  unsigned char* vring = kring + kAtStages * kAtSlotBytes;
-  unsigned char* qtiles = vring + kAtStages * kAtSlotBytes;
+  unsigned char* vring = kring + kAtKStages * kAtSlotBytes;
+  unsigned char* qtiles = vring + kAtVStages * kAtSlotBytes;
   unsigned char* pbufs = qtiles + 2 * kQTileBytes;
   AtSmem& S = *reinterpret_cast<AtSmem*>(pbufs + kAtBufs * kAtPBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAtStages; ++s) {
+    for (int s = 0; s < kAtKStages; ++s) {
       mbar_init(&S.k_full[s], 1);
       mbar_init(&S.k_empty[s], 1);
+    }
+    for (int s = 0; s < kAtVStages; ++s) {
       mbar_init(&S.v_full[s], 1);
       mbar_init(&S.v_empty[s], 1);
     }
@@ -193,8 +199,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         tma_load_2d(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow);
         const long long kvrow0 = a.bg * p.Lmax;
         for (int i = 0; i < np; ++i, ++gpair) {
-          const int st = static_cast<int>(gpair % kAtStages);
-          const uint32_t u = gpair / kAtStages;
+          const int st = static_cast<int>(gpair % kAtKStages);
+          const uint32_t u = gpair / kAtKStages;
           if (u > 0) mbar_wait(&S.k_empty[st], (u - 1) & 1, &S.abort);
           if (S.abort) continue;
           const int ja = S.list[slot][2 * i];
@@ -232,8 +238,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const int np = (count + 1) / 2;
         const long long kvrow0 = a.bg * p.Lmax;
         for (int i = 0; i < np; ++i, ++gpair) {
-          const int st = static_cast<int>(gpair % kAtStages);
-          const uint32_t u = gpair / kAtStages;
+          const int st = static_cast<int>(gpair % kAtVStages);
+          const uint32_t u = gpair / kAtVStages;
           if (u > 0) mbar_wait(&S.v_empty[st], (u - 1) & 1, &S.abort);
           if (S.abort) continue;
           const int ja = S.list[slot][2 * i];
@@ -269,10 +275,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const uint32_t qa = smem_u32(qtiles + slot * kQTileBytes);
           for (int i = 0; i < np; ++i) {
             const uint32_t pp = gp + i;
-            mbar_wait(&S.k_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
+            mbar_wait(&S.k_full[pp % kAtKStages], (pp / kAtKStages) & 1, &S.abort);
             if (pp >= kAtBufs) mbar_wait(&S.p_full[pp % kAtBufs], ((pp / kAtBufs) - 1) & 1, &S.abort);  // S read
             tc_fence_after();
-            const uint32_t kb = smem_u32(kring + (pp % kAtStages) * kAtSlotBytes);
+            const uint32_t kb = smem_u32(kring + (pp % kAtKStages) * kAtSlotBytes);
             const uint32_t sbuf = tmem + static_cast<uint32_t>(pp % kAtBufs) * 16u;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -281,17 +287,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                         k > 0 ? 1u : 0u);
             }
             umma_commit(&S.s_full[pp % kAtBufs]);
-            umma_commit(&S.k_empty[pp % kAtStages]);
+            umma_commit(&S.k_empty[pp % kAtKStages]);
           }
           umma_commit(&S.q_empty[slot]);  // the item's query tile is no longer read
         } else {
           for (int i = 0; i < np; ++i) {
             const uint32_t pp = gp + i;
             mbar_wait(&S.p_full[pp % kAtBufs], (pp / kAtBufs) & 1, &S.abort);
-            mbar_wait(&S.v_full[pp % kAtStages], (pp / kAtStages) & 1, &S.abort);
+            mbar_wait(&S.v_full[pp % kAtVStages], (pp / kAtVStages) & 1, &S.abort);
             tc_fence_after();
             const uint32_t obuf = tmem + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + (pp & 1)) * 16u;
-            const uint32_t vb = smem_u32(vring + (pp % kAtStages) * kAtSlotBytes);
+            const uint32_t vb = smem_u32(vring + (pp % kAtVStages) * kAtSlotBytes);
             const uint32_t pb = smem_u32(pbufs + (pp % kAtBufs) * kAtPBytes);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {  // 16 keys per step
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                         (i >= kAtSoftWGs || k > 0) ? 1u : 0u);
             }
             umma_commit(&S.pv_done[pp % kAtBufs]);
-            umma_commit(&S.v_empty[pp % kAtStages]);
+            umma_commit(&S.v_empty[pp % kAtVStages]);
           }
         }
         gp += np;
