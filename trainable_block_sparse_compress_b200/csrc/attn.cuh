@@ -49,10 +49,11 @@ struct AttnItem {
 
 __device__ __forceinline__ AttnItem attn_item(const AttnParams& p, long long item) {
   AttnItem it;
-  const long long nbg = static_cast<long long>(p.B) * p.Hkv;
-  if (p.lens == nullptr) {  // prefill: latest tokens first
-    it.t = p.Lq - 1 - static_cast<int>(item / nbg);
-    it.bg = item % nbg;
+  if (p.lens == nullptr) {
+    // prefill: one (sequence, kv-head) after another, so the blocks in use at a time are
+    // those of one K/V stream (64 MB at 128K, which L2 holds); latest tokens first
+    it.bg = item / p.Lq;
+    it.t = p.Lq - 1 - static_cast<int>(item % p.Lq);
     it.split = 0;
   } else {
     it.bg = item / p.n_splits;
