@@ -173,6 +173,32 @@ def test_attn_decode_matches_oracle(lens, Lmax, Hq, Hkv, topk):
     compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
 
 
+def test_decode_at_the_maximum_length():
+    # caches of INFLLMV2_MAX_SEQ_LEN tokens: 16383 kernels per sequence, so the selection's
+    # clusters run at their 2048-kernel-per-CTA limit (20 items: clusters of 8), next to
+    # sequences of 1, 33, 64 and 65 tokens in the same batch
+    Lmax = 262144
+    lens = [262144, 262143, 131072, 65, 64, 1, 200000, 5000, 262100, 33]
+    B, Hq, Hkv, topk = len(lens), 32, 2, 96
+    x = inputs(B, Lmax, Hq, Hkv, seed=800, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    k, v, q, ln = x.k.cuda(), x.v.cuda(), x.q.cuda(), x.lens.cuda()
+    kc_g = ops.compress_keys(p, k, lens=ln)
+    for b, n in enumerate(lens):
+        nk = oracle.num_kernels(op, n)
+        assert np.array_equal(u16(kc_g)[b, :, :nk], kc_o[b, :, :nk])
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_decode(p, q, kc_t, ln, Lmax).cpu().numpy()
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    compare_selection(idx_g, idx_o, sc, (lens_np - 1)[:, None], p)
+    o_g, lse_g = ops.sparse_attn_decode(p, q, k, v, ln, torch.from_numpy(idx_o).cuda())
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
+
+
 def test_attn_decode_many_items_per_cta_is_deterministic():
     # more work items than CTAs, ragged lengths: repeated runs must agree bit for bit
     # and match the oracle
