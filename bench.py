@@ -388,6 +388,23 @@ def run_decode(args, rank, world, device, pk, peak_src):
     att_us = [evk[s][1].elapsed_time(evk[s][2]) * 1e3 for s in range(n)]
     us = statistics.median(step_us)
     us = dist.max_over_ranks(us, world, device)
+    # cache maintenance of the step (measured apart from the step above): re-append each
+    # sequence's last token, which rewrites the same rows and kernel and leaves lens as it was
+    last = (lens.long() - 1).clamp(min=0)
+    bidx = torch.arange(p.batch, device=device)
+    k_new = k[bidx, :, last].contiguous()
+    v_new = v[bidx, :, last].contiguous()
+    lens_w = torch.empty_like(lens)
+    eva = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for s in range(n):
+        lens_w.copy_(lens - 1)
+        flush_l2()
+        eva[s][0].record(stream)
+        ops.append_kv(p, k_new, v_new, k, v, lens_w, kc)
+        eva[s][1].record(stream)
+    torch.cuda.synchronize()
+    app_us = statistics.median(eva[s][0].elapsed_time(eva[s][1]) * 1e3 for s in range(n))
+    app_bytes = p.batch * p.num_kv_heads * 2 * 2 * p.head_dim  # the new K and V rows read and written
     sel_b, att_b = decode_bytes(p, x.lens.numpy())
     att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
@@ -411,6 +428,8 @@ def run_decode(args, rank, world, device, pk, peak_src):
                      "traffic": tr_a},
         },
         "gpu_launches_per_step": 2 if ws_a.numel() == 0 else 3,
+        "append": {"kernel": "append_kv_kernel", "us": app_us, "bytes_per_step": app_bytes,
+                   "note": "cache maintenance of a decode step (new K/V rows, completed kernels), timed apart"},
     }
 
 

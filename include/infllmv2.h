@@ -24,8 +24,9 @@
  *    negative status nothing was launched and no output was touched.
  *  - A kernel that waits on the GPU never waits without a bound: if an internal wait
  *    exceeds its limit the kernel stops early and sets a device error word, which
- *    infllmv2_device_error() reads.  The word is sticky: until it is cleared, later
- *    waits give up at once, so outputs of that call and of later calls are undefined.
+ *    infllmv2_device_error() reads.  The word is sticky: until its wait-timeout bit
+ *    is cleared, later waits give up at once, so outputs of that call and of later
+ *    calls are undefined.
  *  - Query positions: prefill queries are tokens 0..L-1 of a fresh sequence; a decode
  *    query is the last token of its sequence, at position lens[b]-1, and its own key
  *    and value are already in the cache.
@@ -61,7 +62,8 @@ enum {
 
 /* Device error word bits (infllmv2_device_error). */
 enum {
-  INFLLMV2_DEVERR_WAIT_TIMEOUT = 1 /* an internal wait ran out of its time limit */
+  INFLLMV2_DEVERR_WAIT_TIMEOUT = 1, /* an internal wait ran out of its time limit */
+  INFLLMV2_DEVERR_CACHE_FULL = 2    /* infllmv2_append_kv met lens[b] outside [0, Lmax) */
 };
 
 enum { INFLLMV2_MODE_PREFILL = 0, INFLLMV2_MODE_DECODE = 1 };
@@ -197,6 +199,24 @@ INFLLMV2_API int infllmv2_sparse_attn_decode_noalloc(const infllmv2_params* p, c
                                                      const int32_t* lens, int32_t Lmax,
                                                      const int32_t* block_idx, void* o, float* lse,
                                                      infllmv2_stream_t stream);
+
+/* Decode cache maintenance: appends one token per sequence ([S] s2.1: decoding; s2.1.2:
+ * the semantic kernels summarise the cached keys).  For every b and kv-head g the new
+ * key and value rows are written at position lens[b] of the caches; when the new length
+ * n = lens[b] + 1 completes a semantic kernel (n >= 32 and (n - 32) % 16 == 0), kernel
+ * i = (n - 32) / 16, the mean of key rows [16 i, 16 i + 32), is written to kc -- the value
+ * infllmv2_compress_keys gives for the same cache; then lens[b] = n.  The caller runs it
+ * once per decode step, before infllmv2_select_blocks, on the same stream.
+ *   k_new, v_new      bf16 [B, Hkv, d]
+ *   k_cache, v_cache  bf16 [B, Hkv, Lmax, d] (updated in place)
+ *   lens              int32 [B] device (in: cached tokens; out: + 1)
+ *   kc                bf16 [B, Hkv, NK(Lmax), d] (updated in place)
+ * A sequence with lens[b] outside [0, Lmax) is left untouched and sets
+ * INFLLMV2_DEVERR_CACHE_FULL in the device error word (checked on the GPU: lens lives
+ * there).  No workspace. */
+INFLLMV2_API int infllmv2_append_kv(const infllmv2_params* p, const void* k_new, const void* v_new, void* k_cache,
+                                    void* v_cache, int32_t* lens, int32_t Lmax, void* kc,
+                                    infllmv2_stream_t stream);
 
 /* Workspace bytes needed by `op` (INFLLMV2_OP_*) for sequence length L_or_Lmax, or 0
  * when the op needs none; (size_t)-1 for invalid parameters. */

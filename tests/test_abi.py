@@ -78,6 +78,18 @@ def test_num_kernels(lib):
         assert lib.infllmv2_num_kernels(cp(), n) == want
 
 
+def test_append_rejects_bad_arguments_before_launch(lib):
+    good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    f = lib.infllmv2_append_kv
+    assert f(cp(), None, good, good, good, good, 1024, good, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(), good, good, good, good, None, 1024, good, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(), good, good, good, good, good + 2, 1024, good, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(), good, good + 8, good, good, good, 1024, good, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(), good, good, good, good, good, 1024, None, None) == _lib.ERR_INVALID_ARG  # kc needed
+    assert f(cp(), good, good, good, good, good, 0, good, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(head_dim=64), good, good, good, good, good, 1024, good, None) == _lib.ERR_UNSUPPORTED
+
+
 def test_workspace_sizes(lib):
     ws = lib.infllmv2_workspace_size
     assert ws(cp(), _lib.OP_COMPRESS, 4096) == 0

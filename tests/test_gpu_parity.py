@@ -312,3 +312,87 @@ def test_decode_workload_end_to_end(name):
     row_ok = np.repeat(same[:, :, 0], p.group, axis=1)  # [B, Hq]
     compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], mask=row_ok)
     assert float(np.abs(lse_g.cpu().numpy() - lse_o[:, :, 0])[row_ok].max()) <= 1e-3
+
+
+# ------------------------------------------------------------ decode cache append
+
+def test_append_kv_matches_a_full_compression():
+    # one appended token per sequence: lengths chosen so that the new token completes
+    # kernel 0 (n = 32), kernel 1 (n = 48), kernel 2 (n = 64), the last kernel of the
+    # cache (n = Lmax), or no kernel (n = 1, 40)
+    Lmax = 4096
+    lens0 = [0, 31, 47, 63, 4095, 39]
+    B, Hq, Hkv = len(lens0), 32, 2
+    x = inputs(B, Lmax, Hq, Hkv, seed=900, mode="decode", lens=lens0)
+    new = inputs(B, 1, Hq, Hkv, seed=901, mode="prefill")  # k, v [B, Hkv, 1, d]: the appended rows
+    p = ops.Params(B, Hq, Hkv, topk=16)
+    op = oparams(p)
+    k, v, ln = x.k.clone().cuda(), x.v.clone().cuda(), x.lens.cuda()
+    kc = ops.compress_keys(p, k, lens=ln)
+    ops.append_kv(p, new.k[:, :, 0].contiguous().cuda(), new.v[:, :, 0].contiguous().cuda(), k, v, ln, kc)
+    lens1 = [n + 1 for n in lens0]
+    assert ln.cpu().tolist() == lens1
+    k_ref, v_ref = x.k.clone(), x.v.clone()
+    for b, n in enumerate(lens0):
+        k_ref[b, :, n] = new.k[b, :, 0]
+        v_ref[b, :, n] = new.v[b, :, 0]
+    assert torch.equal(k.cpu(), k_ref) and torch.equal(v.cpu(), v_ref)
+    kc_o = oracle.compress(op, as_u16(k_ref), lens=np.array(lens1, np.int32))
+    for b, n in enumerate(lens1):
+        nk = oracle.num_kernels(op, n)
+        assert np.array_equal(u16(kc)[b, :, :nk], kc_o[b, :, :nk]), b
+    assert ops.device_error(clear=True) == 0
+
+
+def test_append_kv_over_many_steps_then_decode():
+    # 40 decode steps on a 20-token sequence (kernels complete at 32, 48) and a longer one;
+    # after the appends the caches, kernels and one decode step match the oracle
+    Lmax = 256
+    lens0 = [20, 150]
+    B, Hq, Hkv, steps = len(lens0), 16, 1, 40
+    x = inputs(B, Lmax, Hq, Hkv, seed=910, mode="decode", lens=lens0)
+    new = inputs(B, steps, Hq, Hkv, seed=911, mode="prefill")  # row s of k/v: the token of step s
+    p = ops.Params(B, Hq, Hkv, topk=4)
+    op = oparams(p)
+    k, v, ln = x.k.clone().cuda(), x.v.clone().cuda(), x.lens.cuda()
+    kc = ops.compress_keys(p, k, lens=ln)
+    nk_, nv_ = new.k.cuda(), new.v.cuda()
+    for s in range(steps):
+        ops.append_kv(p, nk_[:, :, s].contiguous(), nv_[:, :, s].contiguous(), k, v, ln, kc)
+    lens1 = [n + steps for n in lens0]
+    assert ln.cpu().tolist() == lens1
+    k_ref, v_ref = x.k.clone(), x.v.clone()
+    for b, n in enumerate(lens0):
+        k_ref[b, :, n:n + steps] = new.k[b, :, :steps]
+        v_ref[b, :, n:n + steps] = new.v[b, :, :steps]
+    assert torch.equal(k.cpu(), k_ref) and torch.equal(v.cpu(), v_ref)
+    lens_np = np.array(lens1, np.int32)
+    kc_o = oracle.compress(op, as_u16(k_ref), lens=lens_np)
+    for b, n in enumerate(lens1):
+        nk = oracle.num_kernels(op, n)
+        assert np.array_equal(u16(kc)[b, :, :nk], kc_o[b, :, :nk]), b
+    o_g, lse_g, idx_g = ops.decode(p, x.q.cuda(), k, v, kc, ln, Lmax)
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    compare_selection(idx_g.cpu().numpy(), idx_o, sc, (lens_np - 1)[:, None], p)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(k_ref), as_u16(v_ref), idx_g.cpu().numpy(),
+                             lens=lens_np)
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
+    assert ops.device_error(clear=True) == 0
+
+
+def test_append_kv_into_a_full_cache_is_refused_on_the_gpu():
+    Lmax = 128
+    B, Hq, Hkv = 2, 16, 1
+    x = inputs(B, Lmax, Hq, Hkv, seed=920, mode="decode", lens=[128, 5])
+    p = ops.Params(B, Hq, Hkv, topk=4)
+    k, v, ln = x.k.clone().cuda(), x.v.clone().cuda(), x.lens.cuda()
+    kc = ops.compress_keys(p, k, lens=ln)
+    kc0 = kc.clone()
+    kn = torch.zeros((B, Hkv, 128), dtype=torch.bfloat16, device="cuda")
+    assert ops.device_error(clear=True) == 0
+    ops.append_kv(p, kn, kn, k, v, ln, kc)
+    err = ops.device_error(clear=True)
+    assert err == 2, err  # INFLLMV2_DEVERR_CACHE_FULL, set by the full sequence only
+    assert ln.cpu().tolist() == [128, 6]  # the full one untouched, the other appended
+    assert torch.equal(k[0].cpu(), x.k[0]) and torch.equal(kc[0], kc0[0])
+    assert torch.equal(k[1, :, 5].cpu(), torch.zeros((Hkv, 128), dtype=torch.bfloat16))

@@ -6,6 +6,7 @@ synthetic-input generator used by the tests and the benchmark.
 """
 from .ops import (  # noqa: F401
     Params,
+    append_kv,
     compress_keys,
     decode,
     device_error,
@@ -15,6 +16,7 @@ from .ops import (  # noqa: F401
     select_blocks_decode,
     select_blocks_prefill,
     sparse_attn_decode,
+    sparse_attn_decode_noalloc,
     sparse_attn_prefill,
     workspace_size,
 )

@@ -62,6 +62,7 @@ SIGNATURES = {
     "infllmv2_sparse_attn_prefill": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode_noalloc": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "infllmv2_append_kv": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
     "infllmv2_workspace_size": (_sz, [_P, _int, _i32]),
     "infllmv2_check_params": (_int, [_P]),
     "infllmv2_status_string": (ctypes.c_char_p, [_int]),

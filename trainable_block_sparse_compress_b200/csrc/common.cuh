@@ -24,6 +24,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // Device error word (one per device), read by infllmv2_device_error().
 __device__ unsigned int g_device_error;
+constexpr unsigned int kDevErrWaitTimeout = 1u;  // a bounded wait ran out (later waits give up at once)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -77,13 +78,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 63u) {
       if (*abort) return false;
-      if (*reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0u) {  // another CTA gave up
+      if ((*reinterpret_cast<volatile unsigned int*>(&g_device_error) & kDevErrWaitTimeout) != 0u) {  // another CTA gave up
         *abort = 1;
         return false;
       }
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;
-        atomicOr(&g_device_error, 1u);
+        atomicOr(&g_device_error, kDevErrWaitTimeout);
         return false;
       }
     }
@@ -98,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_device_error, 1u);
+      atomicOr(&g_device_error, kDevErrWaitTimeout);
       return false;
     }
   }

@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "../../include/infllmv2.h"
+#include "append.cuh"
 #include "attn.cuh"
 #include "attn_dec.cuh"
 #include "attn_tc.cuh"
@@ -287,6 +288,24 @@ int infllmv2_compress_keys(const infllmv2_params* p, const void* k, const int32_
   dim3 grid((halfwarps + 7) / 8, p->num_kv_heads, p->batch);
   compress_kernel<<<grid, kCompressThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(k), lens, Lmax, nk, p->num_kv_heads, static_cast<__nv_bfloat16*>(kc));
+  return launch_status();
+}
+
+int infllmv2_append_kv(const infllmv2_params* p, const void* k_new, const void* v_new, void* k_cache,
+                       void* v_cache, int32_t* lens, int32_t Lmax, void* kc, infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(Lmax)) != INFLLMV2_OK) return st;
+  if (!k_new || !v_new || !k_cache || !v_cache || !lens) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(lens) & 3u))
+    return INFLLMV2_ERR_INVALID_ARG;
+  const int64_t nk = num_kernels(Lmax);
+  if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
+  append_kv_kernel<<<static_cast<unsigned>(p->batch), kHeadDim, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+      static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), lens, Lmax,
+      static_cast<int>(nk), p->num_kv_heads, static_cast<__nv_bfloat16*>(kc));
   return launch_status();
 }
 

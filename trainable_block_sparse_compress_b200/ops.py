@@ -207,6 +207,23 @@ def sparse_attn_decode_noalloc(p: Params, q: torch.Tensor, k_cache: torch.Tensor
     return out, lse
 
 
+def append_kv(p: Params, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              lens: torch.Tensor, kc: torch.Tensor) -> None:
+    """Appends one token per sequence: k_new / v_new bf16 [B, Hkv, d] go to position lens[b]
+    of the caches [B, Hkv, Lmax, d], a completed semantic kernel goes to kc
+    [B, Hkv, NK(Lmax), d], and lens (int32 [B], on the GPU) is incremented in place."""
+    Lmax = k_cache.shape[2]
+    _need(k_new, "k_new", torch.bfloat16, (p.batch, p.num_kv_heads, p.head_dim))
+    _need(v_new, "v_new", torch.bfloat16, (p.batch, p.num_kv_heads, p.head_dim))
+    _need(k_cache, "k_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(v_cache, "v_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(lens, "lens", torch.int32, (p.batch,))
+    _need(kc, "kc", torch.bfloat16, (p.batch, p.num_kv_heads, num_kernels(p, Lmax), p.head_dim))
+    st = _lib.load().infllmv2_append_kv(ctypes.byref(p.c()), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(lens), Lmax, _ptr(kc), _stream())
+    _lib.check("infllmv2_append_kv", st)
+
+
 def device_error(clear: bool = True) -> int:
     v = int(_lib.load().infllmv2_device_error(1 if clear else 0))
     if v < 0:
