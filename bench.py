@@ -49,30 +49,41 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha() -> str:
-    """Hash of every CUDA source of the library: a DRAM-traffic figure counts only when it
-    was taken on exactly these sources."""
+# CUDA sources each kernel is built from (its own header, the headers it includes, and the
+# host file that sets its launch shape)
+KERNEL_SOURCES = {
+    "compress_kernel": ["compress.cuh", "common.cuh", "infllmv2.cu"],
+    "select_prefill_tc_kernel": ["select_prefill_tc.cuh", "select_prefill.cuh", "topk.cuh", "tcgen05.cuh",
+                                 "common.cuh", "infllmv2.cu"],
+    "select_prefill_kernel": ["select_prefill.cuh", "topk.cuh", "common.cuh", "infllmv2.cu"],
+    "attn_tc_kernel": ["attn_tc.cuh", "attn.cuh", "tcgen05.cuh", "common.cuh", "infllmv2.cu"],
+    "attn_kernel": ["attn.cuh", "common.cuh", "infllmv2.cu"],
+    "select_decode_kernel": ["select_decode.cuh", "select_prefill.cuh", "topk.cuh", "common.cuh", "infllmv2.cu"],
+    "attn_decode_cluster_kernel": ["attn_dec.cuh", "attn.cuh", "common.cuh", "infllmv2.cu"],
+}
+
+
+def source_sha(kernel: str) -> str:
+    """Hash of the CUDA sources `kernel` is built from: a DRAM-traffic figure counts only
+    when it was taken on exactly these sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "trainable_block_sparse_compress_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
 def dram_traffic(kernel: str, workload: str):
     """DRAM bytes (read + write) per launch from the committed ncu summary, if it was
-    taken on the current sources and the same workload (else None)."""
+    taken on the kernel's current sources and the same workload (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("source_sha") != source_sha():
-        return None
     e = d.get("kernels", {}).get(kernel, {})
-    if e.get("workload") != workload:
+    if e.get("source_sha") != source_sha(kernel) or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
