@@ -7,8 +7,8 @@
 // is n = 32 + 16 i (i >= 0) completes kernel i.  Its value is the mean of those 32 rows
 // with the arithmetic of compress_kernel: an fp64 sum (exact for bf16 inputs) rounded
 // once to bf16, so an appended cache holds the same kernels a full compression gives.
-// Bound by latency: 512 bytes written per (sequence, kv-head), plus 8 KB read and 256
-// bytes written when a kernel completes.
+// Bound by latency (a few dependent memory round trips): 512 bytes written per (sequence,
+// kv-head), plus 8 KB read and 256 bytes written when a kernel completes.
 #pragma once
 #include "common.cuh"
 
@@ -39,9 +39,14 @@ __global__ void __launch_bounds__(kHeadDim)
     k_cache[(bg * Lmax + pos) * kHeadDim + d] = kv;
     v_cache[(bg * Lmax + pos) * kHeadDim + d] = v_new[bg * kHeadDim + d];
     if (completes) {
+      // the 31 cached rows are loaded together (one round trip), then summed
       const __nv_bfloat16* rows = k_cache + (bg * Lmax + static_cast<size_t>(kStride) * ki) * kHeadDim + d;
+      __nv_bfloat16 r_[kKernel - 1];
+#pragma unroll
+      for (int r = 0; r < kKernel - 1; ++r) r_[r] = rows[r * kHeadDim];
       double s = 0.0;
-      for (int r = 0; r < kKernel - 1; ++r) s += static_cast<double>(__bfloat162float(rows[r * kHeadDim]));
+#pragma unroll
+      for (int r = 0; r < kKernel - 1; ++r) s += static_cast<double>(__bfloat162float(r_[r]));
       s += static_cast<double>(__bfloat162float(kv));  // the new row, from the input
       kc[(bg * NKmax + ki) * kHeadDim + d] = __double2bfloat16(s * (1.0 / kKernel));
     }
