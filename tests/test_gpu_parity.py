@@ -158,8 +158,11 @@ def test_attn_prefill_matches_oracle(B, L, Hq, Hkv, topk):
 
 
 @pytest.mark.parametrize("lens,Lmax,Hq,Hkv,topk", [([3000, 1, 31, 1500, 2049], 3000, 32, 2, 16),
+                                                  ([3000, 1, 31, 1500, 2049], 3000, 8, 2, 16),
                                                   ([9000, 8193, 64], 9000, 16, 1, 96)])
 def test_attn_decode_matches_oracle(lens, Lmax, Hq, Hkv, topk):
+    # 10 (sequence, kv-head) items take the cluster path (G = 16 and G = 4); 3 items the
+    # workspace split path
     B = len(lens)
     x = inputs(B, Lmax, Hq, Hkv, seed=500 + Lmax, mode="decode", lens=lens)
     p = ops.Params(B, Hq, Hkv, topk=topk)
