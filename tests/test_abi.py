@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from trainable_block_sparse_compress_b200 import _lib, build
 from trainable_block_sparse_compress_b200.ops import Params
@@ -131,3 +132,14 @@ def test_calls_reject_bad_arguments_before_launch(lib):
     # decode selection needs lens
     assert lib.infllmv2_select_blocks(cp(batch=4), 1, good, good, None, 1024, good, None, 0,
                                       None) == _lib.ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors_before_calling_the_library():
+    # the binding checks device, dtype and shape itself; nothing reaches the library
+    from trainable_block_sparse_compress_b200 import ops
+    p = ops.Params(batch=1, num_q_heads=16, num_kv_heads=1, topk=4)
+    k = torch.zeros((1, 1, 64, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.compress_keys(p, k)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.append_kv(p, k[:, :, 0], k[:, :, 0], k, k, torch.zeros(1, dtype=torch.int32), k)

@@ -1,13 +1,12 @@
-"""Python binding of the InfLLM v2 C ABI: the same four calls, taking torch tensors.
+"""Python binding of the InfLLM v2 C ABI: the same calls, taking torch tensors.
 
-PyTorch provides device memory and the current CUDA stream; the binding checks shapes
-and dtypes, allocates outputs and workspaces with the caching allocator, and passes raw
-pointers to the library.  No arithmetic of the method runs here.
+PyTorch provides device memory and the current CUDA stream; the binding checks shapes,
+dtypes and devices, allocates outputs and workspaces with the caching allocator, and
+passes raw pointers to the library.  No arithmetic of the method runs here.
 """
 from __future__ import annotations
 
 import ctypes
-import math
 from dataclasses import dataclass
 from typing import Optional, Tuple
 
@@ -71,6 +70,9 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 def _need(t: torch.Tensor, name: str, dtype, shape=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device: another device's pointer is not its memory
+        raise ValueError(f"{name} is on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
