@@ -322,6 +322,22 @@ def test_select_decode_equals_last_prefill_row():
     assert np.array_equal(idx_d[1, :, 0], idx_p[1, :, 1])
 
 
+def test_chunk_of_queries_equals_the_tail_rows_of_a_full_prefill():
+    # a chunk of the last Lq queries against the whole cache (the chunked-prefill case)
+    # selects the blocks, and gets the outputs, of the same rows of a full prefill
+    B, L, Hq, Hkv, Lq = 1, 700, 4, 2, 50
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=16)
+    p = oracle.Params(B, Hq, Hkv, topk=5)
+    kc = oracle.compress(p, as_u16(k))
+    rows = list(range(L - Lq, L))
+    idx_full = oracle.select(p, as_u16(q), kc, rows=rows)
+    idx_chunk = oracle.select(p, as_u16(q[:, L - Lq:]), kc, Lmax=L)
+    assert np.array_equal(idx_chunk, idx_full)
+    o_full, lse_full = oracle.attn(p, as_u16(q), as_u16(k), as_u16(v), idx_full, rows=rows)
+    o_chunk, lse_chunk = oracle.attn(p, as_u16(q[:, L - Lq:]), as_u16(k), as_u16(v), idx_chunk)
+    assert np.array_equal(o_chunk, o_full) and np.array_equal(lse_chunk, lse_full)
+
+
 def test_select_planted_needle_is_found():
     # make one far block's keys point along the group's mean query: it must be selected
     B, L, Hq, Hkv = 1, 2048, 8, 1
