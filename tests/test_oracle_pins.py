@@ -266,6 +266,35 @@ def test_select_invariants_random():
                     assert min(scores[b, g, r, j] for j in free) >= max(rest)
 
 
+@pytest.mark.parametrize("seed", [21, 22, 23])
+def test_select_top_k_is_the_best_subset_by_exhaustive_search(seed):
+    # brute force on tiny inputs: among all sets of k - |forced| eligible non-forced blocks,
+    # the oracle's choice has the largest total score, and among sets with that total the
+    # smallest indices (the tie rule; exact ties are pinned by the closed-form cases); odd
+    # seeds copy one block's keys into another, which brings two blocks' scores close
+    import itertools
+    B, L, Hq, Hkv = 1, 9 * 64, 4, 1
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=seed)
+    if seed % 2:
+        k[:, :, 64 * 3:64 * 4] = k[:, :, 64 * 5:64 * 6]  # blocks 3 and 5 hold the same keys
+    p = oracle.Params(B, Hq, Hkv, topk=5)
+    kc = oracle.compress(p, as_u16(k))
+    rows = np.array([L - 1, L - 30, 5 * 64 + 40])
+    idx, scores = oracle.select(p, as_u16(q), kc, rows=rows, want_scores=True)
+    for r, t in enumerate(rows):
+        cur = int(t) // 64
+        forced = {0} | {j for j in (cur - 1, cur) if j >= 0}
+        cand = [j for j in range(cur + 1) if j not in forced and scores[0, 0, r, j] >= 0]
+        m = min(p.topk - len(forced), len(cand))
+        best = None
+        for sub in itertools.combinations(cand, m):  # ascending tuples, enumerated in lexicographic order
+            tot = sum(scores[0, 0, r, j] for j in sub)
+            if best is None or tot > best[0] + 1e-12:
+                best = (tot, sub)
+        chosen = sorted(set(idx[0, 0, r][idx[0, 0, r] >= 0].tolist()) - forced)
+        assert tuple(chosen) == best[1], (t, chosen, best)
+
+
 def test_select_short_rows_keep_only_forced_blocks():
     q, k, v = rand_inputs(1, 96, 2, 1, seed=11)
     p = oracle.Params(1, 2, 1, topk=4)
