@@ -228,7 +228,9 @@ def run_ours(args, rank, world, device):
 
     sel_flops, attn_flops, gather_bytes = prefill_flops(p, L)
     comp_bytes = p.batch * p.num_kv_heads * (L + nk) * p.head_dim * 2
-    tc_peak = pk["bf16_tflops_sustained"]
+    # per-kernel event timings: the burst peak is the denominator (cuBLAS timed alone);
+    # the sustained figure (a seconds-long loop under the power cap) is given beside it
+    tc_peak = pk["bf16_tflops"]
     kern = {
         "compress": {"ms": kern_ms["compress"], "bound": "hbm", "algorithmic_bytes": comp_bytes,
                      "achieved": comp_bytes / kern_ms["compress"] / 1e6, "unit": "GB/s", "peak": pk["hbm_gbs"]},
@@ -240,6 +242,8 @@ def run_ours(args, rank, world, device):
     }
     for kv in kern.values():
         kv["frac"] = kv["achieved"] / kv["peak"]
+        if kv["bound"] == "tensor":
+            kv["frac_of_sustained"] = kv["achieved"] / pk["bf16_tflops_sustained"]
     top = max(kern, key=lambda n: kern[n]["ms"])
     tc = p.num_q_heads // p.num_kv_heads == 16  # the tensor-core (tcgen05) prefill kernels serve G = 16
     names = {"compress": "compress_kernel",
@@ -252,7 +256,7 @@ def run_ours(args, rank, world, device):
     roof = {"kernel": kname, "bound": kern[top]["bound"], "achieved": kern[top]["achieved"],
             "peak": kern[top]["peak"], "unit": kern[top]["unit"], "frac": kern[top]["frac"],
             "traffic": kern[top]["traffic"],
-            "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kern[top]['bound'] == 'tensor' else 'hbm_gbs'})"}
+            "peak_source": f"{peak_src} ({'bf16_tflops, burst' if kern[top]['bound'] == 'tensor' else 'hbm_gbs'})"}
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -275,7 +279,9 @@ def run_ours(args, rank, world, device):
     del q, k, v
     torch.cuda.empty_cache()
     if not args.no_decode:
-        result["decode"] = run_decode(args, rank, world, device, pk, peak_src)
+        result["decode"] = run_decode(args, args.decode_workload, rank, world, device, pk, peak_src)
+        if args.decode_workload_2:
+            result["decode_2"] = run_decode(args, args.decode_workload_2, rank, world, device, pk, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, wl, x)
     return result
@@ -345,12 +351,12 @@ def run_e2e(args, p, x, device):
             "overlap": "copies of neighbouring steps overlap the compute (two buffer sets, three streams)"}
 
 
-def run_decode(args, rank, world, device, pk, peak_src):
-    """One decode step (select -> attention) over filled ragged caches, L2 flushed before
-    every step (outside the timed events)."""
-    wl = WORKLOADS[args.decode_workload]
+def run_decode(args, workload, rank, world, device, pk, peak_src):
+    """One decode step (select -> attention) over filled caches, L2 flushed before every
+    step (outside the timed events).  Inputs: the same seed as the parity tests."""
+    wl = WORKLOADS[workload]
     p = ops.Params.from_workload(wl)
-    x = make_inputs(wl, seed=dist.rank_seed(args.seed + 1000, rank))
+    x = make_inputs(wl, seed=dist.rank_seed(args.seed, rank))
     Lmax = wl.seq_len
     q, k, v, lens = x.q.to(device), x.k.to(device), x.v.to(device), x.lens.to(device)
     kc = ops.compress_keys(p, k, lens=lens)  # cache maintenance, not timed
@@ -420,10 +426,10 @@ def run_decode(args, rank, world, device, pk, peak_src):
     att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
     sel_med, att_med = statistics.median(sel_us), statistics.median(att_us)
-    tr_s = dram_traffic("select_decode_kernel", args.decode_workload)
-    tr_a = dram_traffic(att_kernel, args.decode_workload)
+    tr_s = dram_traffic("select_decode_kernel", workload)
+    tr_a = dram_traffic(att_kernel, workload)
     return {
-        "workload": args.decode_workload, "value": us, "unit": "us/step", "higher_is_better": False,
+        "workload": workload, "value": us, "unit": "us/step", "higher_is_better": False,
         "batch": p.batch, "mean_len": float(x.lens.float().mean()), "steps": n,
         "l2": "flushed before every step (write then read a 2x L2 buffer, outside the timed events)",
         "roofline": {"bound": "hbm", "achieved": (sel_b + att_b) / us / 1e3, "peak": hbm, "unit": "GB/s",
@@ -514,6 +520,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_128k")
     ap.add_argument("--decode-workload", default="decode_ragged_128k")
+    ap.add_argument("--decode-workload-2", default="decode_32k", help="second decode line ('' for none)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

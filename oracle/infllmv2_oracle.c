@@ -23,7 +23,8 @@
  *       semantic kernel 32 tokens with stride 16, mean-pooled kernels, kernel-to-block
  *       max-pool, group-sum of scores, top-k including 1 initial + 2 local blocks.
  *
- * Readings taken where the pages are silent (numbered as in the design notes):
+ * Readings taken where the pages are silent (R1-R11; each is the plainest reading that
+ * the pages and the workload definition support):
  *  R1  a kernel is the arithmetic mean of its key rows; only complete kernels exist;
  *  R2  kernel i covers tokens [i*stride, i*stride + kernel_size);
  *  R3  per head, a softmax over every causally visible kernel; a block's score for the

@@ -6,6 +6,7 @@ path runs on the five benchmark workloads and is compared on sampled rows.
 """
 import json
 import os
+import warnings
 
 import numpy as np
 import pytest
@@ -260,6 +261,12 @@ def test_attn_decode_ignores_garbage_past_the_length():
 
 # ---------------------------------------------------------- whole path, workloads
 
+def report_ties(what, n_tie, n_rows):
+    """Makes the number of excused near-tie rows visible in the test log (warnings summary)."""
+    warnings.warn(f"{what}: {n_tie} of {n_rows} (sequence, kv-head, row) selections differ from the oracle's "
+                  f"only through an excused near-tie", UserWarning)
+
+
 def sample_rows(L):
     if L <= 4096:
         return np.arange(L)
@@ -283,14 +290,14 @@ def test_prefill_workload_end_to_end(name):
     idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
     idx_gr = idx_g[:, :, rows_t].cpu().numpy()
     same, n_tie = compare_selection(idx_gr, idx_o, sc, np.tile(rows, (wl.batch, 1)), p)
-    o_o, lse_o = oracle.attn(op, as_u16(x.q), as_u16(x.k), as_u16(x.v), idx_o, rows=rows)
+    report_ties(name, n_tie, same.size)
+    # every sampled row's output against the exact attention over the GPU's own block
+    # lists: rows whose list differs from the oracle's through an excused near-tie are
+    # checked too, on the list the GPU actually used
+    o_o, lse_o = oracle.attn(op, as_u16(x.q), as_u16(x.k), as_u16(x.v), idx_gr, rows=rows)
     o_gr = o_g[:, rows_t].float().cpu().numpy()  # [B, R, Hq, d]
     lse_gr = lse_g[:, :, rows_t].cpu().numpy()   # [B, Hq, R]
-    G = p.group
-    row_ok = np.repeat(same, G, axis=1)  # [B, Hq, R]
-    compare_attention(o_gr, o_o, mask=np.transpose(row_ok, (0, 2, 1)))
-    dl = np.abs(lse_gr - lse_o)[row_ok]
-    assert float(dl.max()) <= 1e-3
+    compare_attention(o_gr, o_o, lse_gr, lse_o)
 
 
 @pytest.mark.parametrize("name", ["decode_32k", "decode_ragged_128k"])
@@ -310,11 +317,12 @@ def test_decode_workload_end_to_end(name):
         nk = oracle.num_kernels(op, int(lens_np[b]))
         assert np.array_equal(kcg[b, :, :nk], kc_o[b, :, :nk]), b
     idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=wl.seq_len, want_scores=True)
-    same, _ = compare_selection(idx_g.cpu().numpy(), idx_o, sc, (lens_np - 1)[:, None], p)
-    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
-    row_ok = np.repeat(same[:, :, 0], p.group, axis=1)  # [B, Hq]
-    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], mask=row_ok)
-    assert float(np.abs(lse_g.cpu().numpy() - lse_o[:, :, 0])[row_ok].max()) <= 1e-3
+    idx_gn = idx_g.cpu().numpy()
+    same, n_tie = compare_selection(idx_gn, idx_o, sc, (lens_np - 1)[:, None], p)
+    report_ties(name, n_tie, same.size)
+    # all rows, each on the block list the GPU used (near-tie rows included)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_gn, lens=lens_np)
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
 
 
 # ------------------------------------------------------------ decode cache append

@@ -378,3 +378,52 @@ def test_select_planted_needle_is_found():
     p = oracle.Params(B, Hq, Hkv, topk=8)
     idx = oracle.select(p, as_u16(q), oracle.compress(p, as_u16(k)), rows=[t])
     assert needle in idx[0, 0, 0].tolist()
+
+
+def literal_block_scores(q, kc, t, g, G, scale):
+    """S(t, j) written out independently of the oracle: logits by a torch matrix product,
+    the per-head normaliser by torch.logsumexp, and each block's pool as the index window
+    of semantic kernels 4j-1 .. 4j+3 (kernel i spans tokens [16 i, 16 i + 32); with
+    64-token blocks the kernels that share a token with block j are exactly those),
+    cut to the kernels whose last token 16 i + 31 is <= t.  Returns {j: S(t, j)}."""
+    n_vis = (t - 31) // 16 + 1 if t >= 31 else 0
+    n_vis = min(n_vis, kc.shape[0])
+    if n_vis == 0:
+        return {}
+    logits = (q.double() @ kc[:n_vis].double().T) * scale  # [G, n_vis]
+    lse = torch.logsumexp(logits, dim=1)                    # [G]
+    scores = {}
+    for j in range(t // 64 + 1):
+        window = [i for i in range(4 * j - 1, 4 * j + 4) if 0 <= i < n_vis]
+        if not window:
+            continue
+        total = 0.0
+        for h in range(G):
+            best = max(float(logits[h, i]) for i in window)
+            total += math.exp(best - float(lse[h]))
+        scores[j] = total
+    return scores
+
+
+@pytest.mark.parametrize("G,Hkv,d,seed", [(1, 2, 128, 31), (4, 2, 128, 32), (4, 1, 32, 33)])
+def test_select_scores_match_an_independent_literal_scorer(G, Hkv, d, seed):
+    # random inputs, L <= 512, query rows across the whole sequence (before the first
+    # kernel completes, on block edges, in the middle of blocks, the last token)
+    B, L = 2, 512
+    q, k, v = rand_inputs(B, L, G * Hkv, Hkv, d=d, seed=seed)
+    p = oracle.Params(B, G * Hkv, Hkv, head_dim=d, topk=5)
+    kc = oracle.compress(p, as_u16(k))
+    rows = np.array([0, 30, 31, 47, 63, 64, 100, 191, 192, 255, 300, 383, 448, 500, 511])
+    _, scores = oracle.select(p, as_u16(q), kc, rows=rows, want_scores=True)
+    kc_t = f64(kc)
+    scale = 1.0 / math.sqrt(d)
+    for b in range(B):
+        for g in range(Hkv):
+            for r, t in enumerate(rows):
+                want = literal_block_scores(f64(as_u16(q[b, t, g * G:(g + 1) * G])), kc_t[b, g], int(t), g, G,
+                                            scale)
+                got = scores[b, g, r]
+                eligible = {j for j in range(len(got)) if got[j] >= 0}
+                assert eligible == set(want), (b, g, t)
+                for j, s in want.items():
+                    assert abs(got[j] - s) <= 1e-12 * abs(s), (b, g, t, j, got[j], s)

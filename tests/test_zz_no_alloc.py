@@ -4,17 +4,19 @@ Some callers cannot allocate device memory when they run attention -- an engine 
 whose execute step must not allocate, or a service that reserves its memory budget at
 start-up.  infllmv2_sparse_attn_decode_noalloc serves them from a fixed scratch array
 inside the library.  These tests call it through the C ABI and check that it gives the
-same result as the workspace-taking entry point, on two calls in a row (the second call
-reuses the scratch the first one left behind)."""
+same result as the workspace-taking entry point and as the CPU oracle's exact attention
+over the same block lists, on two calls in a row (the second call reuses the scratch the
+first one left behind)."""
 import ctypes
 
 import numpy as np
 import pytest
 import torch
 
-from parity import O_MAX_ABS, O_MEAN_ABS
+import oracle
+from parity import O_MAX_ABS, O_MEAN_ABS, compare_attention
 from trainable_block_sparse_compress_b200 import _lib, build, ops
-from trainable_block_sparse_compress_b200.synthetic import Workload, make_inputs
+from trainable_block_sparse_compress_b200.synthetic import Workload, as_u16, make_inputs
 
 
 def _check_noalloc_against_entry_point(wl, lens, seed):
@@ -28,6 +30,10 @@ def _check_noalloc_against_entry_point(wl, lens, seed):
     kc = ops.compress_keys(p, k, lens=lens)
     idx = ops.select_blocks_decode(p, q, kc, lens, wl.seq_len)
     o_ref, lse_ref = ops.sparse_attn_decode(p, q, k, v, lens, idx)
+    op = oracle.Params(p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.block_size, p.kernel_size,
+                       p.kernel_stride, p.topk, p.n_init, p.n_local, p.softmax_scale)
+    o_ora, lse_ora = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx.cpu().numpy(),
+                                 lens=np.array(lens.cpu().numpy(), np.int32))
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
         o = torch.full_like(q, float("nan"))
@@ -41,6 +47,7 @@ def _check_noalloc_against_entry_point(wl, lens, seed):
         assert torch.isfinite(o).all() and torch.isfinite(lse).all()
         assert float(diff.max()) <= O_MAX_ABS and float(diff.mean()) <= O_MEAN_ABS, call
         assert float((lse - lse_ref).abs().max()) <= 1e-3, call
+        compare_attention(o.float().cpu().numpy(), o_ora[:, 0], lse.cpu().numpy(), lse_ora[:, :, 0])
     assert ops.device_error(clear=True) == 0
 
 
