@@ -27,9 +27,10 @@
  *    infllmv2_device_error() reads.  The word is sticky: until its wait-timeout bit
  *    is cleared, later waits give up at once, so outputs of that call and of later
  *    calls are undefined.
- *  - Query positions: prefill queries are tokens 0..L-1 of a fresh sequence; a decode
- *    query is the last token of its sequence, at position lens[b]-1, and its own key
- *    and value are already in the cache.
+ *  - Query positions: prefill queries are tokens 0..L-1 of a fresh sequence; a chunk's
+ *    queries are the last q_lens[b] tokens of a cache of kv_lens[b] tokens; a decode
+ *    query is the last token of its sequence, at position lens[b]-1.  A query's own key
+ *    and value are always in the cache.
  *  - GQA: q-head h uses kv-head h / (num_q_heads / num_kv_heads).
  */
 #ifndef INFLLMV2_H_
@@ -156,6 +157,36 @@ INFLLMV2_API int infllmv2_select_blocks(const infllmv2_params* p, int mode, cons
 INFLLMV2_API int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const void* k,
                                  const void* v, const int32_t* block_idx, int32_t L, void* o,
                                  float* lse, void* ws, size_t ws_bytes, infllmv2_stream_t stream);
+
+/* Chunked / ragged-batch prefill: a chunk of queries against an existing cache ([S] s2.1:
+ * prefill of long contexts; s2.1.1-s2.1.2: every query token selects its own blocks;
+ * news page "Technical innovations in MinicPM4": dynamic context block selection).
+ * Sequence b's cache holds kv_lens[b] tokens (its keys, values and semantic kernels,
+ * e.g. from earlier chunks), and its chunk is the last q_lens[b] of them: query row r
+ * sits at position kv_lens[b] - q_lens[b] + r.  The selection and attention are those
+ * of infllmv2_select_blocks / infllmv2_sparse_attn_prefill at those positions; a fresh
+ * prefill is the case q_lens = kv_lens = NULL, Lq = Lmax = L.
+ *   q          bf16 [B, Lq, Hq, d]: rows 0..q_lens[b]-1 of sequence b are its chunk,
+ *              rows at or past q_lens[b] are padding
+ *   q_lens     int32 [B] device, or NULL (every chunk holds Lq queries)
+ *   kv_lens    int32 [B] device, or NULL (every cache holds Lmax tokens); values are
+ *              clamped on the GPU to kv_lens[b] in [0, Lmax], q_lens[b] in
+ *              [0, min(Lq, kv_lens[b])]
+ *   Lq, Lmax   1 <= Lq <= Lmax <= INFLLMV2_MAX_SEQ_LEN
+ *   kc         bf16 [B, Hkv, NK(Lmax), d] (infllmv2_compress_keys with lens = kv_lens)
+ *   block_idx  int32 [B, Hkv, Lq, topk] (output of the selection, input of the attention)
+ *   k, v       bf16 [B, Hkv, Lmax, d]
+ *   o          bf16 [B, Lq, Hq, d];  lse fp32 [B, Hq, Lq] or NULL
+ * Padding rows (r >= q_lens[b]) of block_idx, o and lse are not written.  No workspace
+ * (ws may be NULL).  INVALID_ARG for null / misaligned pointers or sizes out of range. */
+INFLLMV2_API int infllmv2_select_blocks_chunk(const infllmv2_params* p, const void* q, int32_t Lq, const void* kc,
+                                              const int32_t* q_lens, const int32_t* kv_lens, int32_t Lmax,
+                                              int32_t* block_idx, void* ws, size_t ws_bytes,
+                                              infllmv2_stream_t stream);
+INFLLMV2_API int infllmv2_sparse_attn_chunk(const infllmv2_params* p, const void* q, int32_t Lq, const void* k,
+                                            const void* v, const int32_t* q_lens, const int32_t* kv_lens,
+                                            int32_t Lmax, const int32_t* block_idx, void* o, float* lse, void* ws,
+                                            size_t ws_bytes, infllmv2_stream_t stream);
 
 /* Sparse attention for one decode token per sequence ([S] s2.1.3, prefill *and*
  * decode per s2.1 of the same page).  Split over the selected blocks across CTAs,

@@ -143,3 +143,26 @@ def test_binding_rejects_host_tensors_before_calling_the_library():
         ops.compress_keys(p, k)
     with pytest.raises(ValueError, match="CUDA tensor"):
         ops.append_kv(p, k[:, :, 0], k[:, :, 0], k, k, torch.zeros(1, dtype=torch.int32), k)
+
+
+def test_chunk_calls_reject_bad_arguments_before_launch(lib):
+    good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    sel = lib.infllmv2_select_blocks_chunk
+    att = lib.infllmv2_sparse_attn_chunk
+    # Lq in [1, Lmax], Lmax in [1, MAX_SEQ_LEN]
+    assert sel(cp(), good, 0, good, None, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(), good, 129, good, None, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(), good, 8, good, None, None, _lib.MAX_SEQ_LEN + 1, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    # pointers: q, block_idx (and kc once a kernel exists) 16-byte aligned; length arrays 4-byte aligned
+    assert sel(cp(), None, 8, good, None, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(), good, 8, None, None, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(), good, 8, good, good + 2, None, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(), good, 8, good, None, good + 1, 128, good, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert sel(cp(head_dim=64), good, 8, good, None, None, 128, good, None, 0, None) == _lib.ERR_UNSUPPORTED
+    assert att(cp(), good, 8, None, good, None, None, 128, good, good, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert att(cp(), good, 8, good, good, None, None, 128, good, None, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert att(cp(), good, 8, good, good, None, None, 128, good, good, good + 2, None, 0,
+               None) == _lib.ERR_INVALID_ARG
+    assert att(cp(), good, 200, good, good, None, None, 128, good, good, None, None, 0, None) == _lib.ERR_INVALID_ARG
+    assert att(cp(), good, 8, good, good, good + 3, None, 128, good, good, None, None, 0,
+               None) == _lib.ERR_INVALID_ARG

@@ -325,6 +325,79 @@ def test_decode_workload_end_to_end(name):
     compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
 
 
+# ------------------------------------------------------- chunked / ragged prefill
+
+def run_chunk_case(B, Lmax, Hq, Hkv, topk, kv_lens, q_lens, Lq, seed):
+    """Whole chunk path on the GPU (compress the caches, select, attend) against the oracle,
+    sequence by sequence.  Cache rows past kv_lens[b] and query rows past q_lens[b] hold
+    NaN: nothing of them may reach the outputs, and padding rows must stay unwritten."""
+    x = inputs(B, Lmax, Hq, Hkv, seed=seed)  # prefill-shaped: q [B, Lmax, Hq, d]
+    q = x.q[:, :Lq].clone()
+    k, v = x.k.clone(), x.v.clone()
+    for b in range(B):
+        k[b, :, kv_lens[b]:] = float("nan")
+        v[b, :, kv_lens[b]:] = float("nan")
+        q[b, q_lens[b]:] = float("nan")
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    ql = torch.tensor(q_lens, dtype=torch.int32).cuda()
+    kl = torch.tensor(kv_lens, dtype=torch.int32).cuda()
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    kc = ops.compress_keys(p, kd, lens=kl)
+    idx = torch.full((B, Hkv, Lq, topk), -7, dtype=torch.int32, device="cuda")
+    ops.select_blocks_chunk(p, qd, kc, Lmax, q_lens=ql, kv_lens=kl, out=idx)
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, Hq, Lq), 7.0, dtype=torch.float32, device="cuda")
+    ops.sparse_attn_chunk(p, qd, kd, vd, idx, q_lens=ql, kv_lens=kl, out=o, lse=lse)
+    torch.cuda.synchronize()
+    idx, o, lse = idx.cpu().numpy(), o.float().cpu().numpy(), lse.cpu().numpy()
+    op1 = oparams(ops.Params(1, Hq, Hkv, topk=topk))
+    n_tie = 0
+    for b in range(B):
+        n, m = kv_lens[b], q_lens[b]
+        assert np.all(idx[b, :, m:] == -7), "padding rows of block_idx written"
+        assert np.all(np.isnan(o[b, m:])) and np.all(lse[b, :, m:] == 7.0), "padding rows of o / lse written"
+        if m == 0:
+            continue
+        kb = as_u16(x.k[b:b + 1])  # the oracle reads only the first n rows
+        kc_o = oracle.compress(op1, kb, lens=np.array([n], np.int32))
+        idx_o, sc = oracle.select(op1, as_u16(x.q[b:b + 1, :m]), kc_o, lens=np.array([n], np.int32), Lmax=Lmax,
+                                  want_scores=True)
+        pos = np.arange(n - m, n)[None]
+        _, nt = compare_selection(idx[b:b + 1, :, :m], idx_o, sc, pos, p)
+        n_tie += nt
+        o_o, lse_o = oracle.attn(op1, as_u16(x.q[b:b + 1, :m]), kb, as_u16(x.v[b:b + 1]), idx[b:b + 1, :, :m],
+                                 lens=np.array([n], np.int32))
+        compare_attention(o[b:b + 1, :m], o_o, lse[b:b + 1, :, :m], lse_o)
+    report_ties(f"chunk B={B} G={Hq // Hkv}", n_tie, int(sum(q_lens)) * Hkv)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 2), (8, 1)])
+def test_chunk_against_a_longer_cache(Hq, Hkv):
+    # one sequence: a 700-query chunk at the end of a 5000-token cache (query row r at
+    # position 4300 + r), cache length not a multiple of 64
+    run_chunk_case(1, 5000, Hq, Hkv, 16, [5000], [700], 700, seed=1000 + Hq)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 2), (8, 1)])
+def test_chunk_ragged_batch(Hq, Hkv):
+    # ragged batch: chunk and cache lengths differ per sequence (a whole fresh prefill, a
+    # chunk ending mid-block, a short chunk, an empty chunk), padded to Lq = 1200
+    run_chunk_case(4, 3000, Hq, Hkv, 16, [3000, 1200, 100, 700], [500, 1200, 17, 0], 1200, seed=1100 + Hq)
+
+
+def test_chunk_rows_equal_the_same_rows_of_a_full_prefill():
+    # the last 300 queries as a chunk give bit-identical lists and outputs to the same rows
+    # of a full prefill of the sequence
+    B, L, Hq, Hkv, topk, m = 1, 4100, 32, 2, 16, 300
+    x = inputs(B, L, Hq, Hkv, seed=1200)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    q, k, v = x.q.cuda(), x.k.cuda(), x.v.cuda()
+    o_f, lse_f, idx_f, kc = ops.prefill(p, q, k, v)
+    o_c, lse_c, idx_c = ops.prefill_chunk(p, q[:, L - m:].contiguous(), k, v, kc)
+    assert torch.equal(idx_c, idx_f[:, :, L - m:])
+    assert torch.equal(o_c, o_f[:, L - m:]) and torch.equal(lse_c, lse_f[:, :, L - m:])
+
+
 # ------------------------------------------------------------ decode cache append
 
 def test_append_kv_matches_a_full_compression():

@@ -13,6 +13,9 @@ from .ops import (  # noqa: F401
     num_blocks,
     num_kernels,
     prefill,
+    prefill_chunk,
+    select_blocks_chunk,
+    sparse_attn_chunk,
     select_blocks_decode,
     select_blocks_prefill,
     sparse_attn_decode,

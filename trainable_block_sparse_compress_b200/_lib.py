@@ -59,7 +59,9 @@ SIGNATURES = {
     "infllmv2_num_kernels": (_i64, [_P, _i64]),
     "infllmv2_compress_keys": (_int, [_P, _vp, _vp, _i32, _vp, _vp]),
     "infllmv2_select_blocks": (_int, [_P, _int, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "infllmv2_select_blocks_chunk": (_int, [_P, _vp, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_prefill": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "infllmv2_sparse_attn_chunk": (_int, [_P, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode_noalloc": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "infllmv2_append_kv": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),

@@ -29,8 +29,10 @@ constexpr int kMaxTopk = 256;
 constexpr int kMergeRowFloats = kHeadDim + 4;
 
 struct AttnParams {
-  const int32_t* idx;   // [B, Hkv, Lq, topk]
-  const int32_t* lens;  // decode: [B] sequence lengths; prefill: nullptr
+  const int32_t* idx;      // [B, Hkv, Lq, topk]
+  const int32_t* lens;     // decode: [B] sequence lengths; prefill / chunk: nullptr
+  const int32_t* q_lens;   // chunk: [B] queries per sequence (<= Lq), or nullptr (= Lq)
+  const int32_t* kv_lens;  // chunk: [B] cached tokens per sequence (<= Lmax), or nullptr (= Lmax)
   int B, Hq, Hkv, G, Lq, Lmax, topk;
   int n_splits;          // decode: splits per (b, g); prefill: 1
   int blocks_per_split;  // decode: selected blocks per split
@@ -42,8 +44,13 @@ struct AttnParams {
   float* part_lse;   // decode: [B*Hkv, n_splits, 16] natural-log partial lse
 };
 
+// A work item: query row `row` of sequence b (its row in Q, O, lse and the block lists),
+// which sits at position t of the sequence; `valid` is false for padding rows of a
+// chunk (row >= q_lens[b]), which are skipped and not written.
 struct AttnItem {
-  int b, g, t, split, qrow;
+  int b, g, t, row, split, qrow;
+  int kv_len;  // cached tokens of sequence b: key rows at or past it are not the sequence's
+  bool valid;
   long long bg;
 };
 
@@ -53,20 +60,26 @@ __device__ __forceinline__ AttnItem attn_item(const AttnParams& p, long long ite
     // prefill: one (sequence, kv-head) after another, so the blocks in use at a time are
     // those of one K/V stream (64 MB at 128K, which L2 holds); latest tokens first
     it.bg = item / p.Lq;
-    it.t = p.Lq - 1 - static_cast<int>(item % p.Lq);
+    it.row = p.Lq - 1 - static_cast<int>(item % p.Lq);
     it.split = 0;
   } else {
     it.bg = item / p.n_splits;
     it.split = static_cast<int>(item % p.n_splits);
-    it.t = 0;
+    it.row = 0;
   }
   it.b = static_cast<int>(it.bg / p.Hkv);
   it.g = static_cast<int>(it.bg % p.Hkv);
   if (p.lens != nullptr) {
     it.t = min(p.lens[it.b], p.Lmax) - 1;  // -1 (no key) when lens[b] <= 0
+    it.kv_len = it.t + 1;
+    it.valid = true;
     it.qrow = it.b * p.Hq + it.g * p.G;
   } else {
-    it.qrow = (it.b * p.Lq + it.t) * p.Hq + it.g * p.G;
+    const ChunkLens c = chunk_lens(p.q_lens, p.kv_lens, it.b, p.Lq, p.Lmax);
+    it.kv_len = c.kv_len;
+    it.valid = it.row < c.q_len;
+    it.t = it.valid ? c.kv_len - c.q_len + it.row : -1;
+    it.qrow = (it.b * p.Lq + it.row) * p.Hq + it.g * p.G;
   }
   return it;
 }
@@ -225,14 +238,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (use > 0) mbar_wait(&S.qempty[slot], (use - 1) & 1, &S.abort);
       const AttnItem a = attn_item(p, item);
       const int cur = a.t >= 0 ? a.t / kBlock : -1;
-      const int32_t* row =
-          p.idx + ((a.bg * p.Lq + (p.lens ? 0 : a.t)) * static_cast<long long>(p.topk));
+      const int32_t* row = p.idx + ((a.bg * p.Lq + a.row) * static_cast<long long>(p.topk));
       const int lo = a.split * p.blocks_per_split;
       const int hi = p.lens ? lo + p.blocks_per_split : p.topk;
       int count = 0;
       for (int e0 = 0; e0 < p.topk; e0 += 32) {
         const int e = e0 + lane;
-        const int j = e < p.topk ? row[e] : -1;
+        const int j = (e < p.topk && a.valid) ? row[e] : -1;
         const bool ok = j >= 0 && j <= cur;
         const unsigned msk = __ballot_sync(0xffffffffu, ok);
         const int pos = count + __popc(msk & ((1u << lane) - 1u));
@@ -362,7 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         acc[3] += wts[w] * v.w;
       }
       const float lse_nat = L > 0.f ? (M + lg2(L)) * 0.6931471805599453f : -INFINITY;
-      if (r < p.G) {
+      if (r < p.G && a.valid) {
         if (p.lens == nullptr) {
           __nv_bfloat16* dst = p.o + (static_cast<long long>(a.qrow) + r) * kHeadDim + 4 * lane;
           uint2 pk;
@@ -370,7 +382,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           pk.y = pack_bf16(acc[2] * inv, acc[3] * inv);
           *reinterpret_cast<uint2*>(dst) = pk;
           if (p.lse != nullptr && lane == 0)
-            p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + r) * p.Lq + a.t] = lse_nat;
+            p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + r) * p.Lq + a.row] = lse_nat;
         } else {
           const long long prow = (a.bg * p.n_splits + a.split) * kGroupRows + r;
           *reinterpret_cast<float4*>(p.part_o + prow * kHeadDim + 4 * lane) =

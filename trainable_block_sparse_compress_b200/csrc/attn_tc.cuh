@@ -118,7 +118,8 @@ __device__ __forceinline__ void wg_reduce16(const float (&v)[16], float (&out)[1
   named_bar_sync(1 + wg, 128);  // S.red may be reused afterwards
 }
 
-// grid = min(items, SMs) persistent CTAs, block = 384.  Prefill only (p.lens == nullptr).
+// grid = min(items, SMs) persistent CTAs, block = 384.  Prefill and prefill chunks only
+// (p.lens == nullptr).
 __global__ void __launch_bounds__(kAtThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -176,12 +177,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int slot = it & 1, use = it >> 1;
       if (use > 0) mbar_wait(&S.q_empty[slot], (use - 1) & 1, &S.abort);
       const AttnItem a = attn_item(p, item);
-      const int cur = a.t / kBlock;
-      const int32_t* row = p.idx + ((a.bg * p.Lq + a.t) * static_cast<long long>(p.topk));
+      const int cur = a.t >= 0 ? a.t / kBlock : -1;
+      const int32_t* row = p.idx + ((a.bg * p.Lq + a.row) * static_cast<long long>(p.topk));
       int count = 0;
       for (int e0 = 0; e0 < p.topk; e0 += 32) {
         const int e = e0 + lane;
-        const int j = e < p.topk ? row[e] : -1;
+        const int j = (e < p.topk && a.valid) ? row[e] : -1;
         const bool ok = j >= 0 && j <= cur;
         const unsigned msk = __ballot_sync(0xffffffffu, ok);
         const int pos = count + __popc(msk & ((1u << lane) - 1u));
@@ -291,10 +292,28 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           }
           umma_commit(&S.q_empty[slot]);  // the item's query tile is no longer read
         } else {
+          const int n_blk = S.n_blocks[slot];
+          // key rows at or past the sequence's cached length (a chunk's cache may end inside
+          // the query's own block) hold arbitrary values: their V rows are zeroed in shared
+          // memory before the PV, so that they contribute exactly 0 (their P is 0)
+          const int kv_len = attn_item(p, item).kv_len;
           for (int i = 0; i < np; ++i) {
             const uint32_t pp = gp + i;
             mbar_wait(&S.p_full[pp % kAtBufs], (pp / kAtBufs) & 1, &S.abort);
             mbar_wait(&S.v_full[pp % kAtVStages], (pp / kAtVStages) & 1, &S.abort);
+            bool zeroed = false;
+            for (int hb = 0; hb < 2 && 2 * i + hb < n_blk; ++hb) {
+              const int r0 = kv_len - S.list[slot][2 * i + hb] * kBlock;  // first row past the cache
+              if (r0 >= kBlock) continue;
+              unsigned char* vs = vring + (pp % kAtVStages) * kAtSlotBytes + hb * (kKvTileBytes / 2);
+              for (int r = max(r0, 0); r < kBlock; ++r)
+                for (int c = 0; c < 8; ++c) {
+                  *reinterpret_cast<uint4*>(vs + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                  *reinterpret_cast<uint4*>(vs + kAtKHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+              zeroed = true;
+            }
+            if (zeroed) fence_proxy_async_smem();  // the generic writes before the MMA's reads
             tc_fence_after();
             const uint32_t obuf = tmem + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + (pp & 1)) * 16u;
             const uint32_t vb = smem_u32(vring + (pp % kAtVStages) * kAtSlotBytes);
@@ -454,13 +473,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
 #pragma unroll
       for (int h = 0; h < kGroupRows; ++h)
-        if (h < p.G) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(of[h]);
-      if (p.lse != nullptr && tid < p.G) {
+        if (h < p.G && a.valid) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(of[h]);
+      if (p.lse != nullptr && tid < p.G && a.valid) {
         float lv = -INFINITY;
 #pragma unroll
         for (int h = 0; h < kGroupRows; ++h)
           if (h == tid) lv = Lt[h] > 0.f ? (M[h] + lg2(Lt[h])) * 0.6931471805599453f : -INFINITY;
-        p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.t] = lv;
+        p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.row] = lv;
       }
     }
     tc_fence_before();

@@ -216,4 +216,19 @@ __device__ __forceinline__ int last_visible_kernel(int t) {
   return t >= kKernel - 1 ? (t - (kKernel - 1)) / kStride : -1;
 }
 
+// Queries and cache of sequence b in a prefill chunk: q_len queries, the last q_len of
+// kv_len cached tokens (so query row r sits at position kv_len - q_len + r).  Lengths
+// outside [0, Lq] and [0, Lmax] are clamped, and q_len to at most kv_len.
+struct ChunkLens {
+  int q_len, kv_len;
+};
+__device__ __forceinline__ ChunkLens chunk_lens(const int32_t* q_lens, const int32_t* kv_lens, int b, int Lq,
+                                                int Lmax) {
+  ChunkLens c;
+  c.kv_len = kv_lens ? min(max(kv_lens[b], 0), Lmax) : Lmax;
+  c.q_len = q_lens ? min(max(q_lens[b], 0), Lq) : Lq;
+  c.q_len = min(c.q_len, c.kv_len);
+  return c;
+}
+
 }  // namespace infllmv2

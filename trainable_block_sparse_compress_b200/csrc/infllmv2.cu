@@ -229,6 +229,144 @@ size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
   }
 }
 
+// Chunk arguments: Lq and Lmax in [1, INFLLMV2_MAX_SEQ_LEN], Lq <= Lmax, length arrays
+// 4-byte aligned (their values are read and clamped on the GPU).
+int check_chunk(int32_t Lq, const int32_t* q_lens, const int32_t* kv_lens, int32_t Lmax) {
+  if (check_len(Lq) != INFLLMV2_OK || check_len(Lmax) != INFLLMV2_OK || Lq > Lmax) return INFLLMV2_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q_lens) & 3u) || (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
+    return INFLLMV2_ERR_INVALID_ARG;
+  return INFLLMV2_OK;
+}
+
+// Prefill selection for Lq query rows per sequence against caches of Lmax tokens: a fresh
+// prefill (q_lens = kv_lens = NULL, Lq = Lmax = L) or a chunk of the last q_lens[b] of
+// kv_lens[b] cached tokens.
+int select_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const void* kc, const int32_t* q_lens,
+                   const int32_t* kv_lens, int32_t Lmax, int32_t* block_idx, cudaStream_t s) {
+  if (q == nullptr || block_idx == nullptr || !aligned16(q) || !aligned16(block_idx)) return INFLLMV2_ERR_INVALID_ARG;
+  const int64_t nk = num_kernels(Lmax);
+  if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
+  if (static_cast<uint64_t>(p->batch) * p->num_kv_heads * static_cast<uint64_t>(nk) > 0x7fffffffULL ||
+      static_cast<uint64_t>(p->batch) * Lq > 0x7fffffffULL)
+    return INFLLMV2_ERR_UNSUPPORTED;  // TMA coordinates are 32-bit
+  const int G = p->num_q_heads / p->num_kv_heads;
+  const int nblk_cap = round32(num_blocks(Lmax));
+  CUtensorMap tm_kc;
+  std::memset(&tm_kc, 0, sizeof tm_kc);
+  if (nk > 0) {
+    if (!make_map(&tm_kc, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kKcTile))
+      return INFLLMV2_ERR_CUDA;
+  } else {
+    // no complete kernel: every row keeps only its forced blocks; the kernel path runs
+    // with an empty score loop (no tile is loaded, so the map is never dereferenced)
+    if (!make_map(&tm_kc, q, kKcTile, kKcTile)) return INFLLMV2_ERR_CUDA;
+  }
+  SelPrefillParams a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.idx = block_idx;
+  a.q_lens = q_lens;
+  a.kv_lens = kv_lens;
+  a.B = p->batch;
+  a.Lq = Lq;
+  a.Lmax = Lmax;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = G;
+  a.NKmax = static_cast<int>(nk);
+  a.topk = p->topk;
+  a.n_init = p->n_init;
+  a.n_local = p->n_local;
+  a.nblk_cap = nblk_cap;
+  a.scale_log2 = scale_log2(p);
+  a.tiles_per_bg = (Lq + kSelWarps - 1) / kSelWarps;
+  const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
+  if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+  int st;
+  if (G == kGroupRows && nk > 0 && sel_tc_smem_bytes(nblk_cap) <= kMaxSmem) {
+    // tensor-core path: 8 tokens x 16 heads per 128-row UMMA tile
+    static_assert(kTcTokens == kSelWarps, "both prefill selection kernels tile 8 tokens");
+    CUtensorMap tm_q3, tm_kca, tm_kcb;
+    const uint64_t kc_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk;
+    if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * Lq, p->num_q_heads) ||
+        !make_map(&tm_kca, kc, kc_rows, kTcN) || !make_map(&tm_kcb, kc, kc_rows, kTcNB))
+      return INFLLMV2_ERR_CUDA;
+    const size_t smem = sel_tc_smem_bytes(nblk_cap);
+    if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_tc_kernel), smem)) != INFLLMV2_OK) return st;
+    select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kca, tm_kcb, a);
+    return launch_status();
+  }
+  const size_t smem = sel_prefill_smem_bytes(nblk_cap);
+  if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_kernel), smem)) != INFLLMV2_OK) return st;
+  select_prefill_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(tm_kc, a);
+  return launch_status();
+}
+
+int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
+                uint64_t kv_rows, AttnParams& a, cudaStream_t s);
+
+// Prefill attention for Lq query rows per sequence against caches of Lmax tokens (a fresh
+// prefill or a chunk, as for select_prefill).
+int attn_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const void* k, const void* v,
+                 const int32_t* q_lens, const int32_t* kv_lens, int32_t Lmax, const int32_t* block_idx, void* o,
+                 float* lse, cudaStream_t s) {
+  if (!q || !k || !v || !block_idx || !o) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_idx) || !aligned16(o))
+    return INFLLMV2_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * Lq * p->num_q_heads;
+  const uint64_t kv_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * Lmax;
+  if (q_rows > 0x7fffffffULL || kv_rows > 0x7fffffffULL) return INFLLMV2_ERR_UNSUPPORTED;  // 32-bit TMA rows
+  AttnParams a;
+  a.idx = block_idx;
+  a.lens = nullptr;
+  a.q_lens = q_lens;
+  a.kv_lens = kv_lens;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = p->num_q_heads / p->num_kv_heads;
+  a.Lq = Lq;
+  a.Lmax = Lmax;
+  a.topk = p->topk;
+  a.n_splits = 1;
+  a.blocks_per_split = p->topk;
+  a.scale_log2 = scale_log2(p);
+  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * Lq;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.part_o = nullptr;
+  a.part_lse = nullptr;
+  if (a.G == kGroupRows) {
+    // tensor-core path: per item, K/V block pairs against the group's 16 query rows
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
+        !make_map(&tv, v, kv_rows, kBlock))
+      return INFLLMV2_ERR_CUDA;
+    const size_t smem = attn_tc_smem_bytes();
+    int st = set_smem(reinterpret_cast<const void*>(attn_tc_kernel), smem);
+    if (st != INFLLMV2_OK) return st;
+    const long long grid = std::min<long long>(a.num_items, num_sms());
+    attn_tc_kernel<<<static_cast<unsigned>(grid), kAtThreads, smem, s>>>(tq, tk, tv, a);
+    return launch_status();
+  }
+  return launch_attn(p, q, q_rows, k, v, kv_rows, a, s);
+}
+
+int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
+                       uint64_t kv_rows, AttnParams& a, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
+      !make_map(&tv, v, kv_rows, kBlock))
+    return INFLLMV2_ERR_CUDA;
+  const size_t smem = attn_smem_bytes();
+  int st = set_smem(reinterpret_cast<const void*>(attn_kernel), smem);
+  if (st != INFLLMV2_OK) return st;
+  const long long grid = std::min<long long>(a.num_items, num_sms());
+  if (grid <= 0) return INFLLMV2_OK;
+  attn_kernel<<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -315,72 +453,26 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
   int st = check_params(p);
   if (st != INFLLMV2_OK) return st;
   if ((st = check_len(L)) != INFLLMV2_OK) return st;
+  if (mode == INFLLMV2_MODE_PREFILL) {
+    if (lens != nullptr) return INFLLMV2_ERR_INVALID_ARG;
+    return select_prefill(p, q, L, kc, nullptr, nullptr, L, block_idx, reinterpret_cast<cudaStream_t>(stream));
+  }
+  if (mode != INFLLMV2_MODE_DECODE) return INFLLMV2_ERR_INVALID_ARG;
+  (void)ws;  // decode selection needs no workspace
+  (void)ws_bytes;
   if (q == nullptr || block_idx == nullptr || !aligned16(q) || !aligned16(block_idx)) return INFLLMV2_ERR_INVALID_ARG;
+  if (lens == nullptr || (reinterpret_cast<uintptr_t>(lens) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
   const int64_t nk = num_kernels(L);
   if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
   if (static_cast<uint64_t>(p->batch) * p->num_kv_heads * static_cast<uint64_t>(nk) > 0x7fffffffULL)
     return INFLLMV2_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
-  if (mode == INFLLMV2_MODE_PREFILL) {
-    if (lens != nullptr) return INFLLMV2_ERR_INVALID_ARG;
-  } else if (mode == INFLLMV2_MODE_DECODE) {
-    if (lens == nullptr || (reinterpret_cast<uintptr_t>(lens) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
-    (void)ws;  // decode selection needs no workspace
-    (void)ws_bytes;
-  } else {
-    return INFLLMV2_ERR_INVALID_ARG;
-  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int G = p->num_q_heads / p->num_kv_heads;
-  const int nblk_cap = round32(num_blocks(L));
   CUtensorMap tm_kc;
   std::memset(&tm_kc, 0, sizeof tm_kc);
   // a map over a 1-row dummy extent is never dereferenced when there are no kernels
   if (nk > 0 && !make_map(&tm_kc, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kKcTile))
     return INFLLMV2_ERR_CUDA;
-
-  if (mode == INFLLMV2_MODE_PREFILL) {
-    if (nk == 0) {
-      // no complete kernel: every row keeps only its forced blocks; reuse the kernel
-      // path with an empty score loop (TA = TB = 0 never touches the map)
-      if (!make_map(&tm_kc, q, kKcTile, kKcTile)) return INFLLMV2_ERR_CUDA;
-    }
-    SelPrefillParams a;
-    a.q = static_cast<const __nv_bfloat16*>(q);
-    a.idx = block_idx;
-    a.B = p->batch;
-    a.L = L;
-    a.Hq = p->num_q_heads;
-    a.Hkv = p->num_kv_heads;
-    a.G = G;
-    a.NKmax = static_cast<int>(nk);
-    a.topk = p->topk;
-    a.n_init = p->n_init;
-    a.n_local = p->n_local;
-    a.nblk_cap = nblk_cap;
-    a.scale_log2 = scale_log2(p);
-    a.tiles_per_bg = (L + kSelWarps - 1) / kSelWarps;
-    if (G == kGroupRows && nk > 0 && sel_tc_smem_bytes(nblk_cap) <= kMaxSmem) {
-      // tensor-core path: 8 tokens x 16 heads per 128-row UMMA tile
-      static_assert(kTcTokens == kSelWarps, "both prefill selection kernels tile 8 tokens");
-      CUtensorMap tm_q3, tm_kca, tm_kcb;
-      const uint64_t kc_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk;
-      if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * L, p->num_q_heads) ||
-          !make_map(&tm_kca, kc, kc_rows, kTcN) || !make_map(&tm_kcb, kc, kc_rows, kTcNB))
-        return INFLLMV2_ERR_CUDA;
-      const size_t smem = sel_tc_smem_bytes(nblk_cap);
-      if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_tc_kernel), smem)) != INFLLMV2_OK) return st;
-      const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
-      if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
-      select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kca, tm_kcb, a);
-      return launch_status();
-    }
-    const size_t smem = sel_prefill_smem_bytes(nblk_cap);
-    if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_kernel), smem)) != INFLLMV2_OK) return st;
-    const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
-    if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
-    select_prefill_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(tm_kc, a);
-    return launch_status();
-  }
   SelDecodeParams a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.lens = lens;
@@ -404,19 +496,15 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
                         a);
 }
 
-static int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
-                       uint64_t kv_rows, AttnParams& a, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
-      !make_map(&tv, v, kv_rows, kBlock))
-    return INFLLMV2_ERR_CUDA;
-  const size_t smem = attn_smem_bytes();
-  int st = set_smem(reinterpret_cast<const void*>(attn_kernel), smem);
+int infllmv2_select_blocks_chunk(const infllmv2_params* p, const void* q, int32_t Lq, const void* kc,
+                                 const int32_t* q_lens, const int32_t* kv_lens, int32_t Lmax, int32_t* block_idx,
+                                 void* ws, size_t ws_bytes, infllmv2_stream_t stream) {
+  (void)ws;  // no workspace needed
+  (void)ws_bytes;
+  int st = check_params(p);
   if (st != INFLLMV2_OK) return st;
-  const long long grid = std::min<long long>(a.num_items, num_sms());
-  if (grid <= 0) return INFLLMV2_OK;
-  attn_kernel<<<static_cast<unsigned>(grid), kAttnThreads, smem, s>>>(tq, tk, tv, a);
-  return launch_status();
+  if ((st = check_chunk(Lq, q_lens, kv_lens, Lmax)) != INFLLMV2_OK) return st;
+  return select_prefill(p, q, Lq, kc, q_lens, kv_lens, Lmax, block_idx, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const void* k, const void* v,
@@ -427,44 +515,20 @@ int infllmv2_sparse_attn_prefill(const infllmv2_params* p, const void* q, const 
   int st = check_params(p);
   if (st != INFLLMV2_OK) return st;
   if ((st = check_len(L)) != INFLLMV2_OK) return st;
-  if (!q || !k || !v || !block_idx || !o) return INFLLMV2_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_idx) || !aligned16(o))
-    return INFLLMV2_ERR_INVALID_ARG;
-  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
-  AttnParams a;
-  a.idx = block_idx;
-  a.lens = nullptr;
-  a.B = p->batch;
-  a.Hq = p->num_q_heads;
-  a.Hkv = p->num_kv_heads;
-  a.G = p->num_q_heads / p->num_kv_heads;
-  a.Lq = L;
-  a.Lmax = L;
-  a.topk = p->topk;
-  a.n_splits = 1;
-  a.blocks_per_split = p->topk;
-  a.scale_log2 = scale_log2(p);
-  a.num_items = static_cast<long long>(p->batch) * p->num_kv_heads * L;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.lse = lse;
-  a.part_o = nullptr;
-  a.part_lse = nullptr;
-  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * L * p->num_q_heads;
-  const uint64_t kv_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * L;
-  if (a.G == kGroupRows) {
-    // tensor-core path: per item, K/V block pairs against the group's 16 query rows
-    CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
-        !make_map(&tv, v, kv_rows, kBlock))
-      return INFLLMV2_ERR_CUDA;
-    const size_t smem = attn_tc_smem_bytes();
-    if ((st = set_smem(reinterpret_cast<const void*>(attn_tc_kernel), smem)) != INFLLMV2_OK) return st;
-    const long long grid = std::min<long long>(a.num_items, num_sms());
-    attn_tc_kernel<<<static_cast<unsigned>(grid), kAtThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
-        tq, tk, tv, a);
-    return launch_status();
-  }
-  return launch_attn(p, q, q_rows, k, v, kv_rows, a, reinterpret_cast<cudaStream_t>(stream));
+  return attn_prefill(p, q, L, k, v, nullptr, nullptr, L, block_idx, o, lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_sparse_attn_chunk(const infllmv2_params* p, const void* q, int32_t Lq, const void* k, const void* v,
+                               const int32_t* q_lens, const int32_t* kv_lens, int32_t Lmax,
+                               const int32_t* block_idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                               infllmv2_stream_t stream) {
+  (void)ws;  // no workspace needed
+  (void)ws_bytes;
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_chunk(Lq, q_lens, kv_lens, Lmax)) != INFLLMV2_OK) return st;
+  return attn_prefill(p, q, Lq, k, v, q_lens, kv_lens, Lmax, block_idx, o, lse,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,
@@ -486,6 +550,8 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
   AttnParams a;
   a.idx = block_idx;
   a.lens = lens;
+  a.q_lens = nullptr;
+  a.kv_lens = nullptr;
   a.B = p->batch;
   a.Hq = p->num_q_heads;
   a.Hkv = p->num_kv_heads;

@@ -4,8 +4,9 @@
 // tokens and KV blocks is scored through semantic kernels, and the heads of a group
 // share one set of top blocks; s2.1.1: each token keeps its highest-scoring blocks.
 //
-// One CTA = 8 consecutive query tokens of one (sequence, kv-head); consumer warp w owns
-// token t0 + w and its 16 group heads (the MMA rows).  A producer warp streams 64-kernel
+// One CTA = 8 consecutive query rows of one (sequence, kv-head); consumer warp w owns
+// row t0 + w and its 16 group heads (the MMA rows).  A chunk's rows are the last q_len
+// tokens of a cache of kv_len tokens (a fresh prefill: q_len = kv_len = L).  A producer warp streams 64-kernel
 // tiles of Kc (64 x 128 bf16, TMA with 128-byte swizzle) through a 4-stage ring twice:
 //   pass A: logits x_h(i) = scale q_h . Kc_i, online log-sum-exp per head over the
 //           visible kernels;
@@ -26,12 +27,14 @@ constexpr int kKcTile = 64;
 constexpr int kKcTileBytes = kKcTile * kHeadDim * 2;
 
 struct SelPrefillParams {
-  const __nv_bfloat16* q;  // [B, L, Hq, d]
-  int32_t* idx;            // [B, Hkv, L, topk]
-  int B, L, Hq, Hkv, G, NKmax, topk, n_init, n_local;
-  int nblk_cap;  // score slots per token (>= number of blocks, multiple of 32)
+  const __nv_bfloat16* q;  // [B, Lq, Hq, d]
+  int32_t* idx;            // [B, Hkv, Lq, topk]
+  const int32_t* q_lens;   // [B] queries per sequence (<= Lq), or nullptr (= Lq)
+  const int32_t* kv_lens;  // [B] cached tokens per sequence (<= Lmax), or nullptr (= Lmax)
+  int B, Lq, Lmax, Hq, Hkv, G, NKmax, topk, n_init, n_local;
+  int nblk_cap;  // score slots per token (>= number of blocks in Lmax tokens, multiple of 32)
   float scale_log2;
-  int tiles_per_bg;  // ceil(L / 8)
+  int tiles_per_bg;  // ceil(Lq / 8)
 };
 
 struct SelSmem {
@@ -101,8 +104,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   const int tile = p.tiles_per_bg - 1 - static_cast<int>(blockIdx.x / nbg);
   const long long bg = blockIdx.x % nbg;
   const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int t0 = tile * kSelWarps;
-  const int imax_last = last_visible_kernel(min(t0 + kSelWarps - 1, p.L - 1));
+  const int t0 = tile * kSelWarps;  // first query row of the tile
+  const ChunkLens cl = chunk_lens(p.q_lens, p.kv_lens, b, p.Lq, p.Lmax);
+  if (t0 >= cl.q_len) return;  // padding rows only (uniform over the CTA)
+  const int off = cl.kv_len - cl.q_len;  // position of query row 0
+  const int imax_last = last_visible_kernel(off + min(t0 + kSelWarps - 1, cl.q_len - 1));
   const int TA = imax_last >= 0 ? imax_last / kKcTile + 1 : 0;
   const int TB = imax_last >= 0 ? (imax_last + 1) / kKcTile + 1 : 0;
 
@@ -136,15 +142,16 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 
   // ------------------------------------------------------------ consumer warp
   const int t_raw = t0 + warp;
-  const bool tok_ok = t_raw < p.L;
-  const int t = tok_ok ? t_raw : p.L - 1;
+  const bool tok_ok = t_raw < cl.q_len;
+  const int trow = tok_ok ? t_raw : cl.q_len - 1;  // query row (rows past q_len compute, write nothing)
+  const int t = off + trow;                        // its position in the sequence
   const int imax = last_visible_kernel(t);
   const int cur = t / kBlock;
   const int q4 = lane & 3, r0 = lane >> 2;
   const bool row0_ok = r0 < p.G, row1_ok = r0 + 8 < p.G;
 
   uint32_t qa[8][4];
-  load_q_frags(p.q + (static_cast<long long>(b * p.L + t) * p.Hq + g * p.G) * kHeadDim, p.G, qa);
+  load_q_frags(p.q + ((static_cast<long long>(b) * p.Lq + trow) * p.Hq + g * p.G) * kHeadDim, p.G, qa);
 
   // pass A: log-sum-exp over the visible kernels (base 2)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -243,7 +250,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   const int want = p.topk - forced_count(cur, p.n_init, p.n_local);
   const TopkThreshold th = warp_radix_threshold(keys, cur + 1, want, hist_all + warp * 256);
   if (tok_ok) {
-    int32_t* out = p.idx + ((bg * p.L + t) * static_cast<long long>(p.topk));
+    int32_t* out = p.idx + ((bg * p.Lq + trow) * static_cast<long long>(p.topk));
     warp_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out);
   }
 }

@@ -5,8 +5,9 @@
 // softmax over the visible semantic kernels, max-pool of the 5 kernels overlapping each
 // block, sum over the group's heads, top-k with forced initial/local blocks.
 //
-// One CTA = 8 consecutive query tokens of one (sequence, kv-head): 8 x 16 heads = the 128
-// rows (M) of a UMMA tile.  Warp roles (448 threads):
+// One CTA = 8 consecutive query rows of one (sequence, kv-head): 8 x 16 heads = the 128
+// rows (M) of a UMMA tile.  A chunk's rows are the last q_len tokens of a cache of kv_len
+// tokens (a fresh prefill: q_len = kv_len = L).  Warp roles (448 threads):
 //   warp 12 TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then Kc tiles
 //           through a 3-stage ring: pass A tiles of 128 kernels, pass B tiles of 144
 //           kernels that start 16 kernels early, so each pass-B tile also holds the
@@ -96,7 +97,7 @@ __device__ __forceinline__ float reduce_scatter16(const float (&v)[16]) {
 
 __device__ __forceinline__ float max4(float a, float b, float c, float d) { return fmaxf(fmaxf(a, b), fmaxf(c, d)); }
 
-// grid = B * Hkv * ceil(L / 8) (latest tiles first), block = 448.  Requires G == 16.
+// grid = B * Hkv * ceil(Lq / 8) (latest tiles first), block = 448.  Requires G == 16.
 __global__ void __launch_bounds__(kTcThreads, 1)
     select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q3, const __grid_constant__ CUtensorMap tm_kca,
                              const __grid_constant__ CUtensorMap tm_kcb, const SelPrefillParams p) {
@@ -113,8 +114,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int tile = p.tiles_per_bg - 1 - static_cast<int>(blockIdx.x / nbg);
   const long long bg = blockIdx.x % nbg;
   const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int t0 = tile * kTcTokens;
-  const int imax_last = last_visible_kernel(min(t0 + kTcTokens - 1, p.L - 1));
+  const int t0 = tile * kTcTokens;  // first query row of the tile
+  const ChunkLens cl = chunk_lens(p.q_lens, p.kv_lens, b, p.Lq, p.Lmax);
+  if (t0 >= cl.q_len) return;  // padding rows only (uniform over the CTA, before any set-up)
+  const int off = cl.kv_len - cl.q_len;  // position of query row 0
+  const int imax_last = last_visible_kernel(off + min(t0 + kTcTokens - 1, cl.q_len - 1));
   const int TA = imax_last >= 0 ? imax_last / kTcN + 1 : 0;
   const int TB = imax_last >= 0 ? (imax_last + 1) / kTcN + 1 : 0;
   const int T = TA + TB;
@@ -149,8 +153,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       prefetch_tmap(&tm_kca);
       prefetch_tmap(&tm_kcb);
       mbar_arrive_expect_tx(&S.qbar, kTcQBytes);
-      tma_load_3d(qs, &tm_q3, &S.qbar, 0, g * kGroupRows, b * p.L + t0);
-      tma_load_3d(qs + kTcQBytes / 2, &tm_q3, &S.qbar, 64, g * kGroupRows, b * p.L + t0);
+      tma_load_3d(qs, &tm_q3, &S.qbar, 0, g * kGroupRows, b * p.Lq + t0);
+      tma_load_3d(qs + kTcQBytes / 2, &tm_q3, &S.qbar, 64, g * kGroupRows, b * p.Lq + t0);
       const int row0 = static_cast<int>(bg * p.NKmax);
       for (int n = 0; n < T; ++n) {
         const int st = n % kTcStages, u = n / kTcStages;
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int wq = warp & 3;    // TMEM lane quarter
   const int row = 32 * wq + lane;
   const int tok = row >> 4;
-  const int t = min(t0 + tok, p.L - 1);  // rows of tokens past L compute but write nothing
+  const int t = off + min(t0 + tok, cl.q_len - 1);  // position; rows past q_len compute, write nothing
   const int imax = last_visible_kernel(t);
   const int cur = t / kBlock;
   const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
@@ -260,7 +264,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   // zero the key row of token `warp` (blocks 0..cur) while the warpgroups meet
   if (warp < kTcTokens) {
-    const int tz = min(t0 + warp, p.L - 1);
+    const int tz = off + min(t0 + warp, cl.q_len - 1);
     uint32_t* kz = keys_all + warp * p.nblk_cap;
     for (int j = lane; j <= tz / kBlock; j += 32) kz[j] = 0u;
   }
@@ -334,12 +338,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   named_bar_sync(2, 32 * kTcEpiWarps);        // all keys written
 
   // top-k of token `warp`
-  const int tr = t0 + warp;
-  if (warp < kTcTokens && tr < p.L) {
-    const int cu = tr / kBlock;
+  const int tr = t0 + warp;  // query row
+  if (warp < kTcTokens && tr < cl.q_len) {
+    const int cu = (off + tr) / kBlock;
     const uint32_t* kt = keys_all + warp * p.nblk_cap;
     const int want = p.topk - forced_count(cu, p.n_init, p.n_local);
-    int32_t* out = p.idx + ((bg * p.L + tr) * static_cast<long long>(p.topk));
+    int32_t* out = p.idx + ((bg * p.Lq + tr) * static_cast<long long>(p.topk));
     if (cu + 1 <= 32 * kTopkRegKeys) {
       warp_topk_select(kt, cu + 1, want, cu, p.n_init, p.n_local, p.topk, hist_all + warp * 256, out);
     } else {

@@ -121,6 +121,28 @@ def select_blocks_prefill(p: Params, q: torch.Tensor, kc: torch.Tensor,
     return out
 
 
+def select_blocks_chunk(p: Params, q: torch.Tensor, kc: torch.Tensor, Lmax: int,
+                        q_lens: Optional[torch.Tensor] = None, kv_lens: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Selection for a chunk of queries against existing caches.  q bf16 [B, Lq, Hq, d]: rows
+    0..q_lens[b]-1 are the last q_lens[b] of kv_lens[b] cached tokens of sequence b (None:
+    Lq and Lmax); kc [B, Hkv, NK(Lmax), d] -> block_idx int32 [B, Hkv, Lq, topk] (padding
+    rows are not written)."""
+    B, Lq, Hq, d = q.shape
+    _need(q, "q", torch.bfloat16, (p.batch, Lq, p.num_q_heads, p.head_dim))
+    _need(kc, "kc", torch.bfloat16, (p.batch, p.num_kv_heads, num_kernels(p, Lmax), p.head_dim))
+    for t, name in ((q_lens, "q_lens"), (kv_lens, "kv_lens")):
+        if t is not None:
+            _need(t, name, torch.int32, (p.batch,))
+    if out is None:
+        out = torch.empty((B, p.num_kv_heads, Lq, p.topk), dtype=torch.int32, device=q.device)
+    _need(out, "block_idx", torch.int32, (B, p.num_kv_heads, Lq, p.topk))
+    st = _lib.load().infllmv2_select_blocks_chunk(ctypes.byref(p.c()), _ptr(q), Lq, _ptr(kc), _ptr(q_lens),
+                                                  _ptr(kv_lens), Lmax, _ptr(out), None, 0, _stream())
+    _lib.check("infllmv2_select_blocks_chunk", st)
+    return out
+
+
 def select_blocks_decode(p: Params, q: torch.Tensor, kc: torch.Tensor, lens: torch.Tensor, Lmax: int,
                          out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """q bf16 [B, Hq, d], kc [B, Hkv, NK(Lmax), d], lens int32 [B] -> int32 [B, Hkv, 1, topk]."""
@@ -157,6 +179,35 @@ def sparse_attn_prefill(p: Params, q: torch.Tensor, k: torch.Tensor, v: torch.Te
     st = _lib.load().infllmv2_sparse_attn_prefill(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(block_idx),
                                                   L, _ptr(out), _ptr(lse), None, 0, _stream())
     _lib.check("infllmv2_sparse_attn_prefill", st)
+    return out, lse
+
+
+def sparse_attn_chunk(p: Params, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_idx: torch.Tensor,
+                      q_lens: Optional[torch.Tensor] = None, kv_lens: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      want_lse: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Attention of a chunk of queries (as select_blocks_chunk) over caches k, v bf16
+    [B, Hkv, Lmax, d]: O bf16 [B, Lq, Hq, d], lse fp32 [B, Hq, Lq] (padding rows not written)."""
+    B, Lq, Hq, d = q.shape
+    Lmax = k.shape[2]
+    _need(q, "q", torch.bfloat16, (p.batch, Lq, p.num_q_heads, p.head_dim))
+    _need(k, "k", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(v, "v", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(block_idx, "block_idx", torch.int32, (p.batch, p.num_kv_heads, Lq, p.topk))
+    for t, name in ((q_lens, "q_lens"), (kv_lens, "kv_lens")):
+        if t is not None:
+            _need(t, name, torch.int32, (p.batch,))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "o", torch.bfloat16, tuple(q.shape))
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq, Lq))
+    st = _lib.load().infllmv2_sparse_attn_chunk(ctypes.byref(p.c()), _ptr(q), Lq, _ptr(k), _ptr(v), _ptr(q_lens),
+                                                _ptr(kv_lens), Lmax, _ptr(block_idx), _ptr(out), _ptr(lse), None, 0,
+                                                _stream())
+    _lib.check("infllmv2_sparse_attn_chunk", st)
     return out, lse
 
 
@@ -239,6 +290,15 @@ def prefill(p: Params, q, k, v):
     idx = select_blocks_prefill(p, q, kc)
     o, lse = sparse_attn_prefill(p, q, k, v, idx)
     return o, lse, idx, kc
+
+
+def prefill_chunk(p: Params, q, k_cache, v_cache, kc, q_lens=None, kv_lens=None):
+    """A chunk of queries against filled caches (keys, values and semantic kernels of
+    kv_lens[b] tokens each): select -> sparse attention.  Returns (o, lse, idx)."""
+    Lmax = k_cache.shape[2]
+    idx = select_blocks_chunk(p, q, kc, Lmax, q_lens=q_lens, kv_lens=kv_lens)
+    o, lse = sparse_attn_chunk(p, q, k_cache, v_cache, idx, q_lens=q_lens, kv_lens=kv_lens)
+    return o, lse, idx
 
 
 def decode(p: Params, q, k_cache, v_cache, kc, lens, Lmax):
