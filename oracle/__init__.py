@@ -35,6 +35,8 @@ class _Params(ctypes.Structure):
         ("n_init", ctypes.c_int32),
         ("n_local", ctypes.c_int32),
         ("softmax_scale", ctypes.c_double),
+        ("score_mode", ctypes.c_int32),
+        ("pool_mode", ctypes.c_int32),
     ]
 
 
@@ -51,11 +53,14 @@ class Params:
     n_init: int = 1
     n_local: int = 2
     softmax_scale: float = 0.0
+    score_mode: int = 0  # 0 softmax-sum, 1 logit-sum
+    pool_mode: int = 0   # 0 overlapping kernels, 1 kernels inside the block
 
     def _c(self) -> _Params:
         return _Params(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim,
                        self.block_size, self.kernel_size, self.kernel_stride, self.topk,
-                       self.n_init, self.n_local, float(self.softmax_scale))
+                       self.n_init, self.n_local, float(self.softmax_scale), int(self.score_mode),
+                       int(self.pool_mode))
 
 
 def build(force: bool = False) -> str:
@@ -144,7 +149,7 @@ def select(p: Params, q, kc, lens=None, Lmax=None, rows=None, want_scores=False)
 
     Queries are the last Lq tokens of each sequence (lens[b] tokens, or Lmax when lens is
     None).  Returns idx [B,Hkv,R,topk] int32 and, if asked, scores [B,Hkv,R,nblk] float64
-    (-1 marks an ineligible block)."""
+    (-inf marks an ineligible block)."""
     q = _u16(q)
     kc = _u16(kc)
     B, Lq, Hq, d = q.shape

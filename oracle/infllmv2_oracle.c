@@ -41,6 +41,12 @@
  *  R11 bf16 inputs; kernels stored as bf16 (round to nearest even); scores and
  *      attention in double precision here.
  *
+ * Variants of the selection reading (the pages leave the score and the pooling open;
+ * [S] s2.1.3 lists hyper-parameter choices without values):
+ *  V1  logit-sum scoring: a block's score is the sum over the group's heads of the
+ *      block's max scaled logit, with no per-head softmax (one pass, no lse);
+ *  V2  inside pooling: a block's kernels are only those lying entirely inside it.
+ *
  * Layouts (row-major, innermost last; bf16 passed as raw uint16 bit patterns):
  *   Q   [B][Lq][Hq][d]      queries are the last Lq tokens of each sequence
  *   K,V [B][Hkv][Lmax][d]
@@ -60,6 +66,8 @@ typedef struct {
   int32_t block_size, kernel_size, kernel_stride;
   int32_t topk, n_init, n_local;
   double softmax_scale; /* <= 0 selects 1/sqrt(head_dim) (R10) */
+  int32_t score_mode;   /* 0: softmax-sum (R3); 1: logit-sum (V1) */
+  int32_t pool_mode;    /* 0: overlapping kernels (R4); 1: kernels inside the block (V2) */
 } oracle_params;
 
 /* ---------------------------------------------------------------- bf16 numbers */
@@ -118,10 +126,12 @@ static int kernel_visible(const oracle_params* p, int64_t i, int64_t t) {
   return i * p->kernel_stride + p->kernel_size - 1 <= t;
 }
 
-/* R4: kernel i overlaps block j iff their token ranges intersect. */
-static int kernel_overlaps_block(const oracle_params* p, int64_t i, int64_t j) {
+/* Kernel i pools into block j.  R4: their token ranges intersect; V2 (pool_mode 1): the
+ * kernel's range lies inside the block's. */
+static int kernel_pools_into_block(const oracle_params* p, int64_t i, int64_t j) {
   int64_t k0 = i * p->kernel_stride, k1 = k0 + p->kernel_size; /* [k0, k1) */
   int64_t b0 = j * p->block_size, b1 = b0 + p->block_size;     /* [b0, b1) */
+  if (p->pool_mode == 1) return b0 <= k0 && k1 <= b1;
   return k0 < b1 && b0 < k1;
 }
 
@@ -192,14 +202,15 @@ static int candidate_order(const void* a, const void* b) {
  * position t = n_b - Lq + rows[r]):
  *   x_h(i)  = scale * <q_h, Kc_i>              for each head h of group g, visible i
  *   lse_h   = log sum_i exp(x_h(i))            (R3, R5)
- *   m_h(j)  = max over visible kernels i overlapping block j of x_h(i)   (R4)
+ *   m_h(j)  = max over visible kernels i pooling into block j of x_h(i)  (R4 or V2)
  *   S(j)    = sum over heads h of group g of exp(m_h(j) - lse_h)        (R3, s2.1.2)
- * Blocks with no visible overlapping kernel are ineligible.  Forced blocks (R6) are
- * taken first; the remaining topk - |forced| slots go to eligible blocks by (R7).
- * The selection is written ascending and padded with -1 (R8).
+ *             or, with logit-sum scoring, of m_h(j)                     (V1)
+ * Blocks with no visible pooling kernel are ineligible.  Forced blocks (R6) are taken
+ * first; the remaining topk - |forced| slots go to eligible blocks by (R7).  The
+ * selection is written ascending and padded with -1 (R8).
  *
  * scores (optional, may be NULL): [B][Hkv][R][nblk_max] doubles, S(j) for eligible
- * blocks, -1 for ineligible or non-existing ones.
+ * blocks, -infinity for ineligible or non-existing ones (a logit-sum may be negative).
  * Returns 0, or -1 when a row's position falls outside its sequence. */
 int oracle_select(const oracle_params* p, const uint16_t* q, int64_t Lq, const uint16_t* kc,
                   int64_t NKmax, const int32_t* lens, int64_t Lmax, const int64_t* rows,
@@ -217,7 +228,7 @@ int oracle_select(const oracle_params* p, const uint16_t* q, int64_t Lq, const u
         int32_t* out = idx + ((b * H + g) * n_rows + r) * topk;
         double* srow = scores ? scores + ((b * H + g) * n_rows + r) * nblk_max : NULL;
         if (srow)
-          for (int64_t j = 0; j < nblk_max; ++j) srow[j] = -1.0;
+          for (int64_t j = 0; j < nblk_max; ++j) srow[j] = -INFINITY;
         for (int64_t s = 0; s < topk; ++s) out[s] = -1;
         if (t < 0 || t >= n || n > Lmax) {
           bad = 1;
@@ -245,16 +256,19 @@ int oracle_select(const oracle_params* p, const uint16_t* q, int64_t Lq, const u
             if (x[i] > xmax) xmax = x[i];
           }
           if (nvis == 0) continue; /* no kernel is complete yet: nothing to score */
-          double sum = 0.0;
-          for (int64_t i = 0; i < nvis; ++i) sum += exp(x[i] - xmax);
-          double lse = xmax + log(sum);
+          double lse = 0.0;
+          if (p->score_mode == 0) {
+            double sum = 0.0;
+            for (int64_t i = 0; i < nvis; ++i) sum += exp(x[i] - xmax);
+            lse = xmax + log(sum);
+          }
           for (int64_t j = 0; j < nblk; ++j) {
             double m = -INFINITY;
             for (int64_t i = 0; i < nvis; ++i)
-              if (kernel_overlaps_block(p, i, j) && x[i] > m) m = x[i];
+              if (kernel_pools_into_block(p, i, j) && x[i] > m) m = x[i];
             if (m == -INFINITY) continue;
             eligible[j] = 1;
-            S[j] += exp(m - lse);
+            S[j] += (p->score_mode == 0) ? exp(m - lse) : m;
           }
         }
 

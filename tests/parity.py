@@ -6,7 +6,7 @@ import torch
 
 # Tolerances.  Block indices: bit-exact, except where the oracle's score at the last
 # taken slot and the first left-out candidate differ by less than REL_TIE relative
-# (the GPU scores in fp32, the oracle in fp64).  Attention outputs (bf16 inputs, fp32
+# (the GPU scores in fp32, the oracle in fp64).  Ineligible blocks carry score -inf.  Attention outputs (bf16 inputs, fp32
 # accumulation, bf16 output): max-abs 2e-2 and mean-abs 2e-3 against the fp64 oracle.
 REL_TIE = 1e-5
 O_MAX_ABS = 2e-2
@@ -52,7 +52,7 @@ def check_row_selection(gpu_row, ora_row, scores, t, topk, n_init, n_local):
         return f"forced blocks {sorted(F - set(gs))} missing"
     if len(gs) != len([x for x in o if x >= 0]):
         return f"count {len(gs)} != {len([x for x in o if x >= 0])}"
-    cand = [(scores[j], j) for j in range(len(scores)) if scores[j] >= 0 and j not in F and j <= t // 64]
+    cand = [(scores[j], j) for j in range(len(scores)) if np.isfinite(scores[j]) and j not in F and j <= t // 64]
     cand.sort(key=lambda sj: (-sj[0], sj[1]))
     m = topk - len(F)
     if m <= 0 or len(cand) <= m:
@@ -61,10 +61,11 @@ def check_row_selection(gpu_row, ora_row, scores, t, topk, n_init, n_local):
     if not (sigma - nxt <= REL_TIE * max(abs(sigma), 1e-300)):
         return f"sets differ at a clear gap ({sigma:.9g} vs {nxt:.9g}): gpu {gs} oracle {o}"
     chosen = set(gs) - F
+    band = REL_TIE * abs(sigma)  # scores may be negative (logit-sum scoring)
     for s, j in cand:
-        if s > sigma * (1 + REL_TIE) and j not in chosen:
+        if s > sigma + band and j not in chosen:
             return f"block {j} (score {s:.9g}) above the tie band is missing"
-        if j in chosen and s < sigma * (1 - REL_TIE):
+        if j in chosen and s < sigma - band:
             return f"block {j} (score {s:.9g}) below the tie band was taken"
     return "tie"
 

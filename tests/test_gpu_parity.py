@@ -386,8 +386,10 @@ def test_chunk_ragged_batch(Hq, Hkv):
 
 
 def test_chunk_rows_equal_the_same_rows_of_a_full_prefill():
-    # the last 300 queries as a chunk give bit-identical lists and outputs to the same rows
-    # of a full prefill of the sequence
+    # the last 300 queries as a chunk give bit-identical block lists, and the same outputs
+    # up to the fp32 summation order, as the same rows of a full prefill of the sequence
+    # (a persistent CTA splits an item's block pairs between its two softmax warpgroups by
+    # the parity of its running pair count, which depends on the items it ran before)
     B, L, Hq, Hkv, topk, m = 1, 4100, 32, 2, 16, 300
     x = inputs(B, L, Hq, Hkv, seed=1200)
     p = ops.Params(B, Hq, Hkv, topk=topk)
@@ -395,7 +397,8 @@ def test_chunk_rows_equal_the_same_rows_of_a_full_prefill():
     o_f, lse_f, idx_f, kc = ops.prefill(p, q, k, v)
     o_c, lse_c, idx_c = ops.prefill_chunk(p, q[:, L - m:].contiguous(), k, v, kc)
     assert torch.equal(idx_c, idx_f[:, :, L - m:])
-    assert torch.equal(o_c, o_f[:, L - m:]) and torch.equal(lse_c, lse_f[:, :, L - m:])
+    assert float((o_c.float() - o_f[:, L - m:].float()).abs().max()) <= 1e-2
+    assert float((lse_c - lse_f[:, :, L - m:]).abs().max()) <= 1e-5
 
 
 # ------------------------------------------------------------ decode cache append

@@ -210,6 +210,7 @@ def golden_inputs(case):
     L, Hq = case["seq_len"], case["num_q_heads"]
     k = torch.zeros((1, 1, L, 128))
     for comp, key in ((0, "u"), (1, "w")):
+        k[0, 0, :, comp] = case.get(key + "_default", 0.0)
         for j, val in case[key].items():
             k[0, 0, int(j) * 64:(int(j) + 1) * 64, comp] = val
     q = torch.zeros((1, L, Hq, 128))
@@ -219,12 +220,16 @@ def golden_inputs(case):
     return bf16(q), bf16(k)
 
 
-@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "select_closed_form.json")))["cases"],
-                         ids=lambda c: c["name"])
+GOLDEN_CASES = [c for f in ("select_closed_form.json", "select_variants.json")
+                for c in json.load(open(os.path.join(GOLDEN, f)))["cases"]]
+
+
+@pytest.mark.parametrize("case", GOLDEN_CASES, ids=lambda c: c["name"])
 def test_select_closed_form_cases(case):
     q, k = golden_inputs(case)
     p = oracle.Params(1, case["num_q_heads"], case["num_kv_heads"], topk=case["topk"],
-                      n_init=case["n_init"], n_local=case["n_local"], softmax_scale=0.125)
+                      n_init=case["n_init"], n_local=case["n_local"], softmax_scale=0.125,
+                      score_mode=case.get("score_mode", 0), pool_mode=case.get("pool_mode", 0))
     kc = oracle.compress(p, as_u16(k))
     idx = oracle.select(p, as_u16(q), kc, rows=[case["query_pos"]])
     assert idx[0, 0, 0].tolist() == case["expected"]
@@ -261,7 +266,7 @@ def test_select_invariants_random():
                 sel = set(idx[b, g, r][idx[b, g, r] >= 0].tolist())
                 forced = {0, cur, cur - 1}
                 free = [j for j in sel if j not in forced]
-                rest = [scores[b, g, r, j] for j in range(cur + 1) if j not in sel and scores[b, g, r, j] >= 0]
+                rest = [scores[b, g, r, j] for j in range(cur + 1) if j not in sel and np.isfinite(scores[b, g, r, j])]
                 if free and rest:
                     assert min(scores[b, g, r, j] for j in free) >= max(rest)
 
@@ -284,7 +289,7 @@ def test_select_top_k_is_the_best_subset_by_exhaustive_search(seed):
     for r, t in enumerate(rows):
         cur = int(t) // 64
         forced = {0} | {j for j in (cur - 1, cur) if j >= 0}
-        cand = [j for j in range(cur + 1) if j not in forced and scores[0, 0, r, j] >= 0]
+        cand = [j for j in range(cur + 1) if j not in forced and np.isfinite(scores[0, 0, r, j])]
         m = min(p.topk - len(forced), len(cand))
         best = None
         for sub in itertools.combinations(cand, m):  # ascending tuples, enumerated in lexicographic order
@@ -316,7 +321,7 @@ def test_select_identical_heads_scale_scores():
     i1, s1 = oracle.select(p1, as_u16(q), kc, rows=rows, want_scores=True)
     i4, s4 = oracle.select(p4, as_u16(q.repeat(1, 1, 4, 1)), kc, rows=rows, want_scores=True)
     assert np.array_equal(i1, i4)
-    el = s1 >= 0
+    el = np.isfinite(s1)
     assert np.allclose(s4[el], 4 * s1[el], rtol=1e-13)
 
 
@@ -380,12 +385,14 @@ def test_select_planted_needle_is_found():
     assert needle in idx[0, 0, 0].tolist()
 
 
-def literal_block_scores(q, kc, t, g, G, scale):
+def literal_block_scores(q, kc, t, g, G, scale, score_mode=0, pool_mode=0):
     """S(t, j) written out independently of the oracle: logits by a torch matrix product,
     the per-head normaliser by torch.logsumexp, and each block's pool as the index window
     of semantic kernels 4j-1 .. 4j+3 (kernel i spans tokens [16 i, 16 i + 32); with
-    64-token blocks the kernels that share a token with block j are exactly those),
-    cut to the kernels whose last token 16 i + 31 is <= t.  Returns {j: S(t, j)}."""
+    64-token blocks the kernels that share a token with block j are exactly those), or
+    4j .. 4j+2 for the kernels inside the block (pool_mode 1), cut to the kernels whose
+    last token 16 i + 31 is <= t.  score_mode 1 sums the heads' max logits instead of
+    exp(max - lse).  Returns {j: S(t, j)}."""
     n_vis = (t - 31) // 16 + 1 if t >= 31 else 0
     n_vis = min(n_vis, kc.shape[0])
     if n_vis == 0:
@@ -394,24 +401,28 @@ def literal_block_scores(q, kc, t, g, G, scale):
     lse = torch.logsumexp(logits, dim=1)                    # [G]
     scores = {}
     for j in range(t // 64 + 1):
-        window = [i for i in range(4 * j - 1, 4 * j + 4) if 0 <= i < n_vis]
+        lo, hi = (4 * j, 4 * j + 3) if pool_mode == 1 else (4 * j - 1, 4 * j + 4)
+        window = [i for i in range(lo, hi) if 0 <= i < n_vis]
         if not window:
             continue
         total = 0.0
         for h in range(G):
             best = max(float(logits[h, i]) for i in window)
-            total += math.exp(best - float(lse[h]))
+            total += best if score_mode == 1 else math.exp(best - float(lse[h]))
         scores[j] = total
     return scores
 
 
-@pytest.mark.parametrize("G,Hkv,d,seed", [(1, 2, 128, 31), (4, 2, 128, 32), (4, 1, 32, 33)])
-def test_select_scores_match_an_independent_literal_scorer(G, Hkv, d, seed):
+@pytest.mark.parametrize("G,Hkv,d,seed,score_mode,pool_mode", [
+    (1, 2, 128, 31, 0, 0), (4, 2, 128, 32, 0, 0), (4, 1, 32, 33, 0, 0),
+    (4, 2, 64, 34, 1, 0), (4, 2, 64, 35, 0, 1), (2, 1, 64, 36, 1, 1)])
+def test_select_scores_match_an_independent_literal_scorer(G, Hkv, d, seed, score_mode, pool_mode):
     # random inputs, L <= 512, query rows across the whole sequence (before the first
-    # kernel completes, on block edges, in the middle of blocks, the last token)
+    # kernel completes, on block edges, in the middle of blocks, the last token), for the
+    # softmax-sum / logit-sum scores and the overlap / inside pooling
     B, L = 2, 512
     q, k, v = rand_inputs(B, L, G * Hkv, Hkv, d=d, seed=seed)
-    p = oracle.Params(B, G * Hkv, Hkv, head_dim=d, topk=5)
+    p = oracle.Params(B, G * Hkv, Hkv, head_dim=d, topk=5, score_mode=score_mode, pool_mode=pool_mode)
     kc = oracle.compress(p, as_u16(k))
     rows = np.array([0, 30, 31, 47, 63, 64, 100, 191, 192, 255, 300, 383, 448, 500, 511])
     _, scores = oracle.select(p, as_u16(q), kc, rows=rows, want_scores=True)
@@ -421,9 +432,9 @@ def test_select_scores_match_an_independent_literal_scorer(G, Hkv, d, seed):
         for g in range(Hkv):
             for r, t in enumerate(rows):
                 want = literal_block_scores(f64(as_u16(q[b, t, g * G:(g + 1) * G])), kc_t[b, g], int(t), g, G,
-                                            scale)
+                                            scale, score_mode, pool_mode)
                 got = scores[b, g, r]
-                eligible = {j for j in range(len(got)) if got[j] >= 0}
+                eligible = {j for j in range(len(got)) if np.isfinite(got[j])}
                 assert eligible == set(want), (b, g, t)
                 for j, s in want.items():
-                    assert abs(got[j] - s) <= 1e-12 * abs(s), (b, g, t, j, got[j], s)
+                    assert abs(got[j] - s) <= 1e-12 * max(abs(s), 1.0), (b, g, t, j, got[j], s)
