@@ -90,13 +90,30 @@ enum {
  *   n_init         initial blocks always selected (blocks 0..n_init-1), >= 0
  *   n_local        local blocks always selected (the query's block and the
  *                  n_local-1 blocks before it), >= 0; n_init + n_local <= topk
- *   softmax_scale  scale of q.k in scoring and attention; <= 0 means 1/sqrt(d)      */
+ *   softmax_scale  scale of q.k in scoring and attention; <= 0 means 1/sqrt(d)
+ *   score_mode     block score (INFLLMV2_SCORE_*); 0 = softmax-sum
+ *   pool_mode      kernel-to-block pooling (INFLLMV2_POOL_*); 0 = overlapping kernels
+ * A zero-initialised struct with the sizes filled in selects the default reading.    */
 typedef struct {
   int32_t batch, num_q_heads, num_kv_heads, head_dim;
   int32_t block_size, kernel_size, kernel_stride;
   int32_t topk, n_init, n_local;
   float softmax_scale;
+  int32_t score_mode, pool_mode;
 } infllmv2_params;
+
+/* Variants of the block score and of the pooling ([S] s2.1.2 names the relevance score
+ * through fine-grained semantic kernels without a formula; s2.1.3 lists hyper-parameter
+ * choices without values).  With m_h(j) the max scaled logit of head h over the
+ * kernels pooled into block j:
+ *   INFLLMV2_SCORE_SOFTMAX_SUM  S(j) = sum_h exp(m_h(j) - lse_h), lse_h over every visible
+ *                               kernel (two passes over the kernels)
+ *   INFLLMV2_SCORE_LOGIT_SUM    S(j) = sum_h m_h(j) (one pass, no lse; may be negative)
+ *   INFLLMV2_POOL_OVERLAP       block j pools every kernel overlapping it (4j-1 .. 4j+3)
+ *   INFLLMV2_POOL_INSIDE        block j pools the kernels inside it (4j .. 4j+2); a block
+ *                               is eligible once kernel 4j is visible                  */
+enum { INFLLMV2_SCORE_SOFTMAX_SUM = 0, INFLLMV2_SCORE_LOGIT_SUM = 1 };
+enum { INFLLMV2_POOL_OVERLAP = 0, INFLLMV2_POOL_INSIDE = 1 };
 
 /* Largest sequence length (prefill L or decode Lmax) the kernels accept. */
 #define INFLLMV2_MAX_SEQ_LEN 262144
@@ -124,8 +141,9 @@ INFLLMV2_API int infllmv2_compress_keys(const infllmv2_params* p, const void* k,
  *            token is <= t;
  *   lse_h  = log sum_i exp(x_h(i));
  *   m_h(j) = max of x_h(i) over the visible kernels overlapping block j (kernels
- *            4j-1 .. 4j+3);
- *   S(j)   = sum over the group's heads of exp(m_h(j) - lse_h).
+ *            4j-1 .. 4j+3; with INFLLMV2_POOL_INSIDE, 4j .. 4j+2);
+ *   S(j)   = sum over the group's heads of exp(m_h(j) - lse_h) (with
+ *            INFLLMV2_SCORE_LOGIT_SUM, of m_h(j)).
  * Forced blocks (0..n_init-1 and cur-n_local+1..cur, cur = t / 64) are always taken;
  * the other topk - |forced| slots go to the eligible blocks with the highest S, lower
  * block index first on equal S.  Each row of block_idx is written ascending and

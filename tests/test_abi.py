@@ -166,3 +166,12 @@ def test_chunk_calls_reject_bad_arguments_before_launch(lib):
     assert att(cp(), good, 200, good, good, None, None, 128, good, good, None, None, 0, None) == _lib.ERR_INVALID_ARG
     assert att(cp(), good, 8, good, good, good + 3, None, 128, good, good, None, None, 0,
                None) == _lib.ERR_INVALID_ARG
+
+
+def test_score_and_pool_modes_are_checked(lib):
+    f = lib.infllmv2_check_params
+    for s, pm in ((0, 0), (1, 0), (0, 1), (1, 1)):
+        assert f(cp(score_mode=s, pool_mode=pm)) == _lib.OK
+    assert f(cp(score_mode=2)) == _lib.ERR_INVALID_ARG
+    assert f(cp(pool_mode=-1)) == _lib.ERR_INVALID_ARG
+    assert ctypes.sizeof(_lib.CParams) == 13 * 4  # the C struct: 10 int32, a float, 2 int32

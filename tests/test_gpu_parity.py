@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from parity import (bf16_to_f64, bf16_ulp_diff, compare_attention, compare_selection, u16)
+from parity import (bf16_to_f64, bf16_ulp_diff, check_row_selection, compare_attention, compare_selection,
+                    u16)
 from trainable_block_sparse_compress_b200 import build, ops
 from trainable_block_sparse_compress_b200.synthetic import WORKLOADS, Workload, as_u16, make_inputs
 
@@ -32,7 +33,7 @@ def cuda_library():
 
 def oparams(p: ops.Params) -> oracle.Params:
     return oracle.Params(p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.block_size, p.kernel_size,
-                         p.kernel_stride, p.topk, p.n_init, p.n_local, p.softmax_scale)
+                         p.kernel_stride, p.topk, p.n_init, p.n_local, p.softmax_scale, p.score_mode, p.pool_mode)
 
 
 def inputs(B, L, Hq, Hkv, seed, mode="prefill", lens=None):
@@ -72,12 +73,17 @@ def test_compress_closed_form_exact():
 
 # -------------------------------------------------------------------- selection
 
-@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "select_closed_form.json")))["cases"],
-                         ids=lambda c: c["name"])
-def test_select_closed_form_cases(case):
+GOLDEN_CASES = [c for f in ("select_closed_form.json", "select_variants.json")
+                for c in json.load(open(os.path.join(GOLDEN, f)))["cases"]]
+
+
+@pytest.mark.parametrize("case", GOLDEN_CASES, ids=lambda c: c["name"])
+@pytest.mark.parametrize("mode", ["prefill", "decode"])
+def test_select_closed_form_cases(case, mode):
     L, Hq = case["seq_len"], case["num_q_heads"]
     k = torch.zeros((1, 1, L, 128))
     for comp, key in ((0, "u"), (1, "w")):
+        k[0, 0, :, comp] = case.get(key + "_default", 0.0)
         for j, val in case[key].items():
             k[0, 0, int(j) * 64:(int(j) + 1) * 64, comp] = val
     q = torch.zeros((1, L, Hq, 128))
@@ -85,10 +91,17 @@ def test_select_closed_form_cases(case):
         for h in range(Hq):
             q[0, :, h, h] = 8.0
     p = ops.Params(1, Hq, 1, topk=case["topk"], n_init=case["n_init"], n_local=case["n_local"],
-                   softmax_scale=0.125)
-    kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda())
-    idx = ops.select_blocks_prefill(p, q.to(torch.bfloat16).cuda(), kc).cpu().numpy()
-    assert idx[0, 0, case["query_pos"]].tolist() == case["expected"]
+                   softmax_scale=0.125, score_mode=case.get("score_mode", 0), pool_mode=case.get("pool_mode", 0))
+    t = case["query_pos"]
+    if mode == "prefill":
+        kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda())
+        idx = ops.select_blocks_prefill(p, q.to(torch.bfloat16).cuda(), kc).cpu().numpy()
+        assert idx[0, 0, t].tolist() == case["expected"]
+    else:  # the same row as a decode query over a cache of t + 1 tokens
+        lens = torch.tensor([t + 1], dtype=torch.int32).cuda()
+        kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda(), lens=lens)
+        idx = ops.select_blocks_decode(p, q[:, t].to(torch.bfloat16).contiguous().cuda(), kc, lens, L)
+        assert idx.cpu().numpy()[0, 0, 0].tolist() == case["expected"]
 
 
 SELECT_CASES = [
@@ -119,6 +132,75 @@ def test_select_prefill_matches_oracle(B, L, Hq, Hkv, topk, ni, nl):
     rows = prefill_rows(L)
     idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
     compare_selection(idx_g[:, :, rows], idx_o, sc, np.tile(rows, (B, 1)), p)
+
+
+# score / pool variants: (score_mode, pool_mode); (0, 0) is the default reading above
+VARIANTS = [(1, 0), (0, 1), (1, 1)]
+
+
+@pytest.mark.parametrize("score_mode,pool_mode", VARIANTS)
+@pytest.mark.parametrize("B,L,Hq,Hkv,topk", [(1, 3000, 32, 2, 16), (2, 1000, 8, 1, 6)])
+def test_select_prefill_variants_match_oracle(B, L, Hq, Hkv, topk, score_mode, pool_mode):
+    # G = 16 (tcgen05 kernel) and G = 8 (m16n8k16 kernel), rows across the sequence
+    x = inputs(B, L, Hq, Hkv, seed=250 + L + 7 * score_mode + pool_mode)
+    p = ops.Params(B, Hq, Hkv, topk=topk, score_mode=score_mode, pool_mode=pool_mode)
+    op = oparams(p)
+    kc_o = oracle.compress(op, as_u16(x.k))
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_prefill(p, x.q.cuda(), kc_t).cpu().numpy()
+    rows = prefill_rows(L)
+    idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
+    _, n_tie = compare_selection(idx_g[:, :, rows], idx_o, sc, np.tile(rows, (B, 1)), p)
+    report_ties(f"prefill variant s{score_mode} p{pool_mode} G={Hq // Hkv}", n_tie, B * Hkv * len(rows))
+
+
+@pytest.mark.parametrize("score_mode,pool_mode", VARIANTS)
+def test_select_decode_variants_match_oracle(score_mode, pool_mode):
+    lens, Lmax, Hq, Hkv, topk = [9000, 1, 31, 1500, 2049, 64, 65], 9000, 32, 2, 16
+    B = len(lens)
+    x = inputs(B, Lmax, Hq, Hkv, seed=350 + 7 * score_mode + pool_mode, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk, score_mode=score_mode, pool_mode=pool_mode)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_decode(p, x.q.cuda(), kc_t, x.lens.cuda(), Lmax).cpu().numpy()
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    compare_selection(idx_g, idx_o, sc, (lens_np - 1)[:, None], p)
+
+
+@pytest.mark.parametrize("mode", ["prefill", "decode"])
+def test_logit_sum_with_negative_scores(mode):
+    # keys shifted by -2 in every component and queries made positive: nearly every logit,
+    # and so every block's logit sum, is negative; the top-k order must still follow the
+    # values (order-preserving keys over all 32 bits)
+    B, L, Hq, Hkv, topk = 1, 3000, 32, 2, 16
+    x = inputs(B, L, Hq, Hkv, seed=450)
+    q = x.q.float().abs().to(torch.bfloat16)
+    k = (x.k.float() - 2.0).to(torch.bfloat16)
+    p = ops.Params(B, Hq, Hkv, topk=topk, score_mode=1)
+    op = oparams(p)
+    kc_o = oracle.compress(op, as_u16(k))
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    rows = prefill_rows(L)
+    idx_o, sc = oracle.select(op, as_u16(q), kc_o, rows=rows, want_scores=True)
+    fin = sc[np.isfinite(sc)]
+    assert (fin < 0).mean() > 0.99
+    if mode == "prefill":
+        idx_g = ops.select_blocks_prefill(p, q.cuda(), kc_t).cpu().numpy()[:, :, rows]
+        compare_selection(idx_g, idx_o, sc, np.tile(rows, (B, 1)), p)
+    else:  # each sampled row as a decode query over the cache up to it
+        lens_np = (rows[-40:] + 1).astype(np.int32)
+        pd = ops.Params(len(lens_np), Hq, Hkv, topk=topk, score_mode=1)
+        kd = k.expand(len(lens_np), -1, -1, -1).contiguous().cuda()
+        lens_t = torch.from_numpy(lens_np).cuda()
+        kc_d = ops.compress_keys(pd, kd, lens=lens_t)
+        idx_g = ops.select_blocks_decode(pd, q[0, rows[-40:]].contiguous().cuda(), kc_d, lens_t, L).cpu().numpy()
+        for r in range(len(lens_np)):
+            for g in range(Hkv):
+                res = check_row_selection(idx_g[r, g, 0], idx_o[0, g, len(rows) - 40 + r],
+                                          sc[0, g, len(rows) - 40 + r], int(lens_np[r] - 1), topk, 1, 2)
+                assert res in ("exact", "tie"), res
 
 
 @pytest.mark.parametrize("lens,Lmax,Hq,Hkv,topk", [([3000, 1, 31, 1500, 2049], 3000, 32, 2, 16),

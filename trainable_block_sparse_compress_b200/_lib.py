@@ -21,6 +21,11 @@ ERR_CUDA = -4
 MODE_PREFILL = 0
 MODE_DECODE = 1
 
+SCORE_SOFTMAX_SUM = 0
+SCORE_LOGIT_SUM = 1
+POOL_OVERLAP = 0
+POOL_INSIDE = 1
+
 OP_COMPRESS = 0
 OP_SELECT_PREFILL = 1
 OP_SELECT_DECODE = 2
@@ -51,6 +56,8 @@ class CParams(ctypes.Structure):
         ("n_init", ctypes.c_int32),
         ("n_local", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float),
+        ("score_mode", ctypes.c_int32),
+        ("pool_mode", ctypes.c_int32),
     ]
 
 

@@ -209,6 +209,35 @@ __device__ __forceinline__ unsigned char* align_smem(unsigned char* p, uint32_t 
   return p + (r - a);
 }
 
+// Order-preserving image of a float in uint32 (a < b exactly when enc(a) < enc(b)), so
+// that integer atomicMax computes a float max.  Never 0 for a non-NaN float.
+__device__ __forceinline__ uint32_t ord_enc(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_dec(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Block-score variants of the selection (the pages leave the score and the pooling
+// open): softmax-sum (sum over heads of exp(block max - lse)) or logit-sum (sum over
+// heads of the block max logit, no lse); overlapping kernels 4j-1 .. 4j+3 or the kernels
+// inside the block 4j .. 4j+2.
+constexpr int kScoreSoftmaxSum = 0, kScoreLogitSum = 1;
+constexpr int kPoolOverlap = 0, kPoolInside = 1;
+
+// Top-k key of a candidate block's score: a larger score gives a larger key, and 0 is
+// left for non-candidates.  Softmax-sum scores are >= 0: their bit patterns + 1; logit
+// sums may be negative: the order-preserving image.
+__device__ __forceinline__ uint32_t score_key(float s, int score_mode) {
+  return score_mode == kScoreLogitSum ? ord_enc(s) : __float_as_uint(s) + 1u;
+}
+
+// Block j has a visible pooled kernel for a query whose last visible kernel is imax.
+__device__ __forceinline__ bool block_eligible(int j, int imax, int pool_mode) {
+  return (pool_mode == kPoolInside ? 4 * j : max(4 * j - 1, 0)) <= imax;
+}
+
 // Semantic-kernel arithmetic for block 64 / kernel 32 / stride 16: kernel i covers
 // tokens [16 i, 16 i + 32) and is visible to the query at t iff 16 i + 31 <= t.
 // Highest visible kernel index for position t (-1 when none).

@@ -29,7 +29,7 @@ using namespace infllmv2;
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -41,6 +41,9 @@ int check_params(const infllmv2_params* p) {
   if (p->topk < 1 || p->n_init < 0 || p->n_local < 0) return INFLLMV2_ERR_INVALID_ARG;
   if (static_cast<long long>(p->n_init) + p->n_local > p->topk) return INFLLMV2_ERR_INVALID_ARG;
   if (!(p->softmax_scale <= 0.f || std::isfinite(p->softmax_scale))) return INFLLMV2_ERR_INVALID_ARG;
+  if ((p->score_mode != INFLLMV2_SCORE_SOFTMAX_SUM && p->score_mode != INFLLMV2_SCORE_LOGIT_SUM) ||
+      (p->pool_mode != INFLLMV2_POOL_OVERLAP && p->pool_mode != INFLLMV2_POOL_INSIDE))
+    return INFLLMV2_ERR_INVALID_ARG;
   const int G = p->num_q_heads / p->num_kv_heads;
   if (p->head_dim != kHeadDim || p->block_size != kBlock || p->kernel_size != kKernel ||
       p->kernel_stride != kStride)
@@ -276,6 +279,8 @@ int select_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const vo
   a.topk = p->topk;
   a.n_init = p->n_init;
   a.n_local = p->n_local;
+  a.score_mode = p->score_mode;
+  a.pool_mode = p->pool_mode;
   a.nblk_cap = nblk_cap;
   a.scale_log2 = scale_log2(p);
   a.tiles_per_bg = (Lq + kSelWarps - 1) / kSelWarps;
@@ -486,6 +491,8 @@ int infllmv2_select_blocks(const infllmv2_params* p, int mode, const void* q, co
   a.topk = p->topk;
   a.n_init = p->n_init;
   a.n_local = p->n_local;
+  a.score_mode = p->score_mode;
+  a.pool_mode = p->pool_mode;
   a.scale_log2 = scale_log2(p);
   if (nk == 0 && !make_map(&tm_kc, q, kKcTile, kKcTile)) return INFLLMV2_ERR_CUDA;  // never read: no tiles
   const int C = select_cluster(p, nk);

@@ -13,7 +13,8 @@
 //   2. after a cluster barrier each CTA forms lse_h from the C partial states and takes
 //      the previous CTA's carry into its first block (both read through distributed
 //      shared memory, all loads in parallel), computes S(j) = sum_h exp(m_h(j) - lse_h)
-//      for its blocks and stores the keys into CTA 0;
+//      (or, with logit-sum scoring, sum_h m_h(j)) for its blocks and stores the keys into
+//      CTA 0 (with inside pooling block j pools kernels 4j .. 4j+2 only, and no carry);
 //   3. CTA 0 finds the k-th largest key by a 32-way radix search (lane l of every warp
 //      counts the keys at or above candidate digit l; once the digit's bucket holds at
 //      most 32 keys they are ranked directly) and all its threads write the ascending
@@ -48,6 +49,7 @@ struct SelDecodeParams {
   const int32_t* lens;     // [B]
   int32_t* idx;            // [B, Hkv, 1, topk]
   int B, Hq, Hkv, G, Lmax, NKmax, topk, n_init, n_local;
+  int score_mode, pool_mode;  // kScore*, kPool*
   float scale_log2;
 };
 
@@ -73,16 +75,6 @@ constexpr size_t sel_decode_smem_bytes() {
          sizeof(SdSmem);
 }
 
-// Order-preserving image of a float in uint32 (a < b exactly when enc(a) < enc(b)), so
-// that integer atomicMax computes a float max.
-__device__ __forceinline__ uint32_t ord_enc(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float ord_dec(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
 // For each lane l: how many of this warp's keys (thread i takes keys i + kSdThreads s,
 // s < R) are >= T | l << shift, where the bits of T below shift + w are zero and l < 2^w
 // (lanes l >= 2^w count the keys at or above T + 2^(shift + w), the bucket's upper end).
@@ -92,14 +84,15 @@ __device__ __forceinline__ float ord_dec(uint32_t k) {
 __device__ __forceinline__ int warp_count_digits(const uint32_t* keys, int n, int R, uint32_t T, int shift, int w,
                                                  bool first) {
   const int lane = threadIdx.x & 31;
-  const uint32_t hT = T >> (shift + w);
+  const bool top = shift + w >= 32;  // the digit holds the key's top bits (a shift by 32 is undefined)
+  const uint32_t hT = top ? 0u : T >> (shift + w);
   const uint32_t dmask = (1u << w) - 1u;
   int cnt = 0;
 #pragma unroll 2
   for (int s = 0; s < R; ++s) {
     const int j = static_cast<int>(threadIdx.x) + kSdThreads * s;
     const uint32_t k = j < n ? keys[j] : 0u;
-    const uint32_t hk = k >> (shift + w);
+    const uint32_t hk = top ? 0u : k >> (shift + w);
     const bool in = hk == hT;
     const uint32_t d = (k >> shift) & dmask;
     const unsigned A = __ballot_sync(0xffffffffu, hk > hT);
@@ -125,8 +118,8 @@ __device__ __forceinline__ int warp_count_digits(const uint32_t* keys, int n, in
 }
 
 // k-th largest of the n keys in shared memory by all kSdThreads threads; same result as
-// warp_radix_threshold.  Radix search on the 31 key bits in digits of 5 (the last one
-// 1): lane l of every warp counts the keys >= T | l << shift (warp_count_digits), the
+// warp_radix_threshold.  Radix search on the 32 key bits in digits of 5 (the last one
+// 2): lane l of every warp counts the keys >= T | l << shift (warp_count_digits), the
 // counts meet in S.cnt (double-buffered: one barrier per digit) and the largest digit
 // with at least `want` keys at or above it is taken.  As soon as the chosen digit's
 // bucket holds at most 32 keys, they are gathered and ranked directly.
@@ -150,15 +143,15 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     buf ^= 1;
     return tot;
   };
-  // first digit (bits 30..26); lane 0 counts the candidates (keys >= 1): bucket 0 is [1, 2^26)
-  int tot = count_ge(0u, 26, 5, true);
+  // first digit (bits 31..27); lane 0 counts the candidates (keys >= 1): bucket 0 is [1, 2^27)
+  int tot = count_ge(0u, 27, 5, true);
   if (__shfl_sync(0xffffffffu, tot, 0) <= want) {  // at most `want` candidates: take them all
     r.key = 0;
     r.ties = 0;
     return r;
   }
   uint32_t T = 0;
-  int shift = 26, above = 0, inb = 0;  // bucket [max(T, 1), T + 2^shift): `inb` keys, `above` keys above it
+  int shift = 27, above = 0, inb = 0;  // bucket [max(T, 1), T + 2^shift): `inb` keys, `above` keys above it
   for (;;) {
     const unsigned ok = __ballot_sync(0xffffffffu, tot >= want);  // lane 0 always qualifies
     const int l = 31 - __clz(ok);
@@ -167,7 +160,7 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     inb = __shfl_sync(0xffffffffu, tot, l) - above;
     T |= static_cast<uint32_t>(l) << shift;
     if (inb <= 32 || shift == 0) break;
-    const int w = shift > 5 ? 5 : 1;  // 26, 21, 16, 11, 6, 1 (5 bits each), then bit 0
+    const int w = shift >= 7 ? 5 : shift;  // 27, 22, 17, 12, 7, 2 (5 bits each), then bits 1..0
     shift -= w;
     tot = count_ge(T, shift, w, false);
   }
@@ -398,19 +391,25 @@ __global__ void __launch_bounds__(kSdThreads)
           }
         }
         // quad q (lanes q4 = 0, 2 of n-tile nt: quads 2 nt, 2 nt + 1 of the warp's four):
-        // its max feeds block q, its last kernel block q + 1
+        // its max feeds block q, its last kernel block q + 1 (overlap pooling); with inside
+        // pooling only kernels 4q .. 4q+2 feed block q and the last kernel no block
+        const bool inside = p.pool_mode == kPoolInside;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const float pm0 = fmaxf(s[nt][0], s[nt][1]), pm1 = fmaxf(s[nt][2], s[nt][3]);
+          const bool drop_last = inside && (q4 & 1);  // this lane's second kernel is 4q+3
+          const float pm0 = drop_last ? s[nt][0] : fmaxf(s[nt][0], s[nt][1]);
+          const float pm1 = drop_last ? s[nt][2] : fmaxf(s[nt][2], s[nt][3]);
           const float om0 = __shfl_xor_sync(0xffffffffu, pm0, 1), om1 = __shfl_xor_sync(0xffffffffu, pm1, 1);
           const float la0 = __shfl_xor_sync(0xffffffffu, s[nt][1], 1);
           const float la1 = __shfl_xor_sync(0xffffffffu, s[nt][3], 1);
           if ((q4 & 1) == 0) {
             const int qd = (i * kKcTile + kofs + 8 * nt + 4 * (q4 >> 1)) >> 2;
             atomicMax(&bm[r0 * kSdBStride + qd], ord_enc(fmaxf(pm0, om0)));
-            atomicMax(&bm[r0 * kSdBStride + qd + 1], ord_enc(la0));
             atomicMax(&bm[(r0 + 8) * kSdBStride + qd], ord_enc(fmaxf(pm1, om1)));
-            atomicMax(&bm[(r0 + 8) * kSdBStride + qd + 1], ord_enc(la1));
+            if (!inside) {
+              atomicMax(&bm[r0 * kSdBStride + qd + 1], ord_enc(la0));
+              atomicMax(&bm[(r0 + 8) * kSdBStride + qd + 1], ord_enc(la1));
+            }
           }
         }
         // online (max, sum of exp2) per head
@@ -490,17 +489,17 @@ __global__ void __launch_bounds__(kSdThreads)
     const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
     for (int j = jb0 + threadIdx.x; j < jb1; j += kSdThreads) {
       const int ql = j - jb0;  // <= nq, since cur + 1 <= ceil(nk / 4) + 1 <= C nq + 1
-      const bool eligible = max(4 * j - 1, 0) < nk;
+      const bool eligible = block_eligible(j, nk - 1, p.pool_mode);
       const bool forced = j < p.n_init || j > cur - p.n_local;
       uint32_t key = 0u;
       if (eligible && !forced && ql <= nq) {
         float sc = 0.f;
         for (int h = 0; h < p.G; ++h) {
           float mb = ord_dec(bm[h * kSdBStride + ql]);
-          if (ql == 0) mb = fmaxf(mb, S.carry[h]);
-          sc += ex2(mb - S.lse2[h]);
+          if (ql == 0 && p.pool_mode == kPoolOverlap) mb = fmaxf(mb, S.carry[h]);
+          sc += p.score_mode == kScoreLogitSum ? mb : ex2(mb - S.lse2[h]);
         }
-        key = __float_as_uint(sc) + 1u;
+        key = score_key(sc, p.score_mode);
       }
       keys0[j] = key;
     }

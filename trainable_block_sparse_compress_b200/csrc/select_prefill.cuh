@@ -13,6 +13,8 @@
 //   pass B: the logits again; per head the max over the 5 kernels 4j-1..4j+3 that
 //           overlap block j, p_h(j) = exp(m_h(j) - lse_h), summed over the 16 heads
 //           with warp shuffles, giving the block score S(j) kept in shared memory.
+// Variants: logit-sum scoring sums m_h(j) itself and skips pass A; inside pooling takes
+// the max over kernels 4j..4j+2 only.
 // Finally each warp radix-selects its token's top blocks and writes them ascending.
 #pragma once
 #include "common.cuh"
@@ -32,6 +34,7 @@ struct SelPrefillParams {
   const int32_t* q_lens;   // [B] queries per sequence (<= Lq), or nullptr (= Lq)
   const int32_t* kv_lens;  // [B] cached tokens per sequence (<= Lmax), or nullptr (= Lmax)
   int B, Lq, Lmax, Hq, Hkv, G, NKmax, topk, n_init, n_local;
+  int score_mode, pool_mode;  // kScore*, kPool*
   int nblk_cap;  // score slots per token (>= number of blocks in Lmax tokens, multiple of 32)
   float scale_log2;
   int tiles_per_bg;  // ceil(Lq / 8)
@@ -109,7 +112,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (t0 >= cl.q_len) return;  // padding rows only (uniform over the CTA)
   const int off = cl.kv_len - cl.q_len;  // position of query row 0
   const int imax_last = last_visible_kernel(off + min(t0 + kSelWarps - 1, cl.q_len - 1));
-  const int TA = imax_last >= 0 ? imax_last / kKcTile + 1 : 0;
+  // pass A (the per-head lse) only for softmax-sum scoring
+  const int TA = (imax_last >= 0 && p.score_mode == kScoreSoftmaxSum) ? imax_last / kKcTile + 1 : 0;
   const int TB = imax_last >= 0 ? (imax_last + 1) / kKcTile + 1 : 0;
 
   if (threadIdx.x == 0) {
@@ -203,6 +207,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   __syncwarp();
 
   // pass B: block scores
+  const bool inside = p.pool_mode == kPoolInside, logit = p.score_mode == kScoreLogitSum;
   float carry0 = -INFINITY, carry1 = -INFINITY;
   const int base4 = lane & ~3;
   for (int n = TA; n < TA + TB; ++n) {
@@ -220,28 +225,33 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         s[nt][e] = ok ? s[nt][e] * p.scale_log2 : -INFINITY;
         s[nt][2 + e] = ok ? s[nt][2 + e] * p.scale_log2 : -INFINITY;
       }
-      // group of 4 kernels: cols 0-3 (lanes q4 0,1) or 4-7 (lanes q4 2,3) of this n-tile
-      float g0 = fmaxf(s[nt][0], s[nt][1]), g1 = fmaxf(s[nt][2], s[nt][3]);
+      // group of 4 kernels: cols 0-3 (lanes q4 0,1) or 4-7 (lanes q4 2,3) of this n-tile;
+      // with inside pooling the group's last kernel (4j + 3, this lane's second column on
+      // odd q4) leaves the block's pool
+      const bool drop_last = inside && (q4 & 1);
+      float g0 = drop_last ? s[nt][0] : fmaxf(s[nt][0], s[nt][1]);
+      float g1 = drop_last ? s[nt][2] : fmaxf(s[nt][2], s[nt][3]);
       g0 = fmaxf(g0, __shfl_xor_sync(0xffffffffu, g0, 1));
       g1 = fmaxf(g1, __shfl_xor_sync(0xffffffffu, g1, 1));
-      // the kernel before each group (4j - 1) straddles blocks j-1 and j
+      // the kernel before each group (4j - 1) straddles blocks j-1 and j (overlap pooling)
       const float lastA0 = __shfl_sync(0xffffffffu, s[nt][1], base4 | 1);
       const float lastA1 = __shfl_sync(0xffffffffu, s[nt][3], base4 | 1);
       const float lastB0 = __shfl_sync(0xffffffffu, s[nt][1], base4 | 3);
       const float lastB1 = __shfl_sync(0xffffffffu, s[nt][3], base4 | 3);
-      const float mb0 = fmaxf(g0, q4 < 2 ? carry0 : lastA0);
-      const float mb1 = fmaxf(g1, q4 < 2 ? carry1 : lastA1);
+      const float mb0 = inside ? g0 : fmaxf(g0, q4 < 2 ? carry0 : lastA0);
+      const float mb1 = inside ? g1 : fmaxf(g1, q4 < 2 ? carry1 : lastA1);
       carry0 = lastB0;
       carry1 = lastB1;
-      float pr = (row0_ok ? ex2(mb0 - lse0) : 0.f) + (row1_ok ? ex2(mb1 - lse1) : 0.f);
+      float pr = logit ? ((row0_ok ? mb0 : 0.f) + (row1_ok ? mb1 : 0.f))
+                       : ((row0_ok ? ex2(mb0 - lse0) : 0.f) + (row1_ok ? ex2(mb1 - lse1) : 0.f));
       pr += __shfl_xor_sync(0xffffffffu, pr, 4);
       pr += __shfl_xor_sync(0xffffffffu, pr, 8);
       pr += __shfl_xor_sync(0xffffffffu, pr, 16);
       const int j = c * 16 + 2 * nt + (q4 >> 1);
       if ((lane == 0 || lane == 2) && j <= cur) {
-        const bool eligible = max(4 * j - 1, 0) <= imax;
+        const bool eligible = block_eligible(j, imax, p.pool_mode);
         const bool forced = j < p.n_init || j > cur - p.n_local;
-        if (eligible && !forced) keys[j] = __float_as_uint(pr) + 1u;
+        if (eligible && !forced) keys[j] = score_key(pr, p.score_mode);
       }
     }
   }

@@ -3,7 +3,8 @@
 //
 // Same rule as select_prefill.cuh (MiniCPM4 summary page s2.1.1 / s2.1.2): per head a
 // softmax over the visible semantic kernels, max-pool of the 5 kernels overlapping each
-// block, sum over the group's heads, top-k with forced initial/local blocks.
+// block, sum over the group's heads, top-k with forced initial/local blocks (and the
+// same variants: logit-sum scoring without pass A, inside pooling).
 //
 // One CTA = 8 consecutive query rows of one (sequence, kv-head): 8 x 16 heads = the 128
 // rows (M) of a UMMA tile.  A chunk's rows are the last q_len tokens of a cache of kv_len
@@ -119,7 +120,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (t0 >= cl.q_len) return;  // padding rows only (uniform over the CTA, before any set-up)
   const int off = cl.kv_len - cl.q_len;  // position of query row 0
   const int imax_last = last_visible_kernel(off + min(t0 + kTcTokens - 1, cl.q_len - 1));
-  const int TA = imax_last >= 0 ? imax_last / kTcN + 1 : 0;
+  // pass A (the per-head lse) only for softmax-sum scoring
+  const int TA = (imax_last >= 0 && p.score_mode == kScoreSoftmaxSum) ? imax_last / kTcN + 1 : 0;
   const int TB = imax_last >= 0 ? (imax_last + 1) / kTcN + 1 : 0;
   const int T = TA + TB;
 
@@ -283,7 +285,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     lse = L > 0.f ? M + lg2(L) : INFINITY;
   }
 
-  // pass B: block maxima along the row, p = exp(m - lse), group sum over the 16 heads
+  // pass B: block maxima along the row, p = exp(m - lse) (or m itself for logit-sum
+  // scoring), group sum over the 16 heads
+  const bool inside = p.pool_mode == kPoolInside, logit = p.score_mode == kScoreLogitSum;
   uint32_t* keys = keys_all + tok * p.nblk_cap;
   int nb = TA;
   while (nb % kTcEpiWGs != wg) ++nb;
@@ -316,17 +320,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
 #pragma unroll
         for (int gq = 0; gq < 8; ++gq) {
-          const float mb = fmaxf(max4(x[4 * gq], x[4 * gq + 1], x[4 * gq + 2], x[4 * gq + 3]), carry);
-          pb[8 * q2 + gq] = ex2(fmaf(mb, sl2, -lse));
+          // overlap: kernels 4j-1 (the carry) .. 4j+3; inside: 4j .. 4j+2 (raw logits)
+          const float mb = inside ? fmaxf(fmaxf(x[4 * gq], x[4 * gq + 1]), x[4 * gq + 2])
+                                  : fmaxf(max4(x[4 * gq], x[4 * gq + 1], x[4 * gq + 2], x[4 * gq + 3]), carry);
+          pb[8 * q2 + gq] = logit ? mb : ex2(fmaf(mb, sl2, -lse));  // a logit sum ranks like a scaled one
           carry = x[4 * gq + 3];
         }
       }
       const float sum = reduce_scatter16(pb);
       const int j = 32 * c + 16 * half + (lane & 15);
       if (j <= cur) {
-        const bool eligible = max(4 * j - 1, 0) <= imax;
+        const bool eligible = block_eligible(j, imax, p.pool_mode);
         const bool forced = j < p.n_init || j > cur - p.n_local;
-        keys[j] = (eligible && !forced) ? __float_as_uint(sum) + 1u : 0u;
+        keys[j] = (eligible && !forced) ? score_key(sum, p.score_mode) : 0u;
       }
     }
     tc_fence_before();

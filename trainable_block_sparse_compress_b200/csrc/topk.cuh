@@ -3,8 +3,8 @@
 //
 // Ordering rule (MiniCPM4 summary page s2.1.1: each query token keeps its highest
 // scoring blocks): higher score first, lower block index first among equal scores.
-// Scores are non-negative fp32 group sums, so their IEEE bit patterns order like the
-// values.  A candidate's key is bits(score) + 1 and a non-candidate's key is 0.
+// A candidate's key is a nonzero uint32 that orders like its score (score_key) and a
+// non-candidate's key is 0; all 32 key bits may be in use.
 // The k-th largest key T is found either by sorting a prefiltered candidate set
 // (warp_topk_select) or by bisection on the key bits with warp-wide counts; the list is
 // then written in ascending block order with forced blocks first-class members and
@@ -30,7 +30,7 @@ __device__ __forceinline__ bool topk_simple(const TopkThreshold& th) {
 __device__ __forceinline__ uint32_t take_from(const TopkThreshold& th) { return th.key == 0u ? 1u : th.key; }
 
 // One warp.  keys[0..n) in shared memory; `want` keys to take.  Finds the want-th
-// largest key T by bisection on its bits, most significant first: T >= c exactly when
+// largest key T by bisection on its 32 bits, most significant first: T >= c exactly when
 // at least `want` keys are >= c.  Each lane holds up to kTopkRegKeys keys in registers
 // (n <= 32 * kTopkRegKeys); larger n re-reads shared memory each step.  No atomics.
 constexpr int kTopkRegKeys = 64;
@@ -75,7 +75,7 @@ __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* ke
       return r;
     }
 #pragma unroll 1
-    for (int bit = 30; bit >= 0; --bit) {
+    for (int bit = 31; bit >= 0; --bit) {
       const uint32_t c = T | (1u << bit);
       if (warp_count_ge_regs(kr, c) >= want) T = c;
     }
@@ -89,7 +89,7 @@ __device__ __forceinline__ TopkThreshold warp_radix_threshold(const uint32_t* ke
     return r;
   }
 #pragma unroll 1
-  for (int bit = 30; bit >= 0; --bit) {
+  for (int bit = 31; bit >= 0; --bit) {
     const uint32_t c = T | (1u << bit);
     if (warp_count_ge_smem(keys, n, c) >= want) T = c;
   }
@@ -276,7 +276,7 @@ __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, in
       } else {
         uint32_t T = 0;
 #pragma unroll 1
-        for (int bit = 30; bit >= 0; --bit) {
+        for (int bit = 31; bit >= 0; --bit) {
           const uint32_t c = T | (1u << bit);
           if (warp_count_ge_regs(kr, c) >= want) T = c;
         }

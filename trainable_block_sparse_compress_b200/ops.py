@@ -28,6 +28,8 @@ class Params:
     n_init: int = 1
     n_local: int = 2
     softmax_scale: float = 0.0
+    score_mode: int = 0  # 0 softmax-sum, 1 logit-sum (the block score)
+    pool_mode: int = 0   # 0 overlapping kernels, 1 kernels inside the block (the pooling)
 
     @property
     def group(self) -> int:
@@ -36,7 +38,7 @@ class Params:
     def c(self) -> _lib.CParams:
         return _lib.CParams(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
                             self.kernel_size, self.kernel_stride, self.topk, self.n_init, self.n_local,
-                            float(self.softmax_scale))
+                            float(self.softmax_scale), int(self.score_mode), int(self.pool_mode))
 
     @staticmethod
     def from_workload(wl, batch: Optional[int] = None) -> "Params":
