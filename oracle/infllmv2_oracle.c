@@ -46,6 +46,8 @@
  *  V1  logit-sum scoring: a block's score is the sum over the group's heads of the
  *      block's max scaled logit, with no per-head softmax (one pass, no lse);
  *  V2  inside pooling: a block's kernels are only those lying entirely inside it.
+ *  V3  backward: gradients flow to q, k and v through the attention over the selected
+ *      blocks; the top-k selection itself passes no gradient.
  *
  * Layouts (row-major, innermost last; bf16 passed as raw uint16 bit patterns):
  *   Q   [B][Lq][Hq][d]      queries are the last Lq tokens of each sequence
@@ -384,6 +386,117 @@ int64_t oracle_attn(const oracle_params* p, const uint16_t* q, int64_t Lq, const
           if (lse) lse[(b * Hq + h) * n_rows + r] = mx + log(den);
         }
         free(logit);
+        free(pos);
+        free(use);
+      }
+    }
+  }
+  if (bad_row) return -1;
+  return bad_idx;
+}
+
+/* --------------------------------------- step 6: backward of the sparse attention */
+
+/* Gradients of the sparse attention of oracle_attn with respect to q, k and v, for a
+ * given upstream gradient d_o ([S] s2.1 and s2.1.3: the attention is trained, so it is
+ * differentiated; the block selection is a top-k choice, constant almost everywhere, so
+ * no gradient flows through it -- the block lists are fixed inputs here (V3)).
+ *
+ * For batch b, q-head h (kv-head g = h / G) and query row r at position t, with J the
+ * keys of the selected blocks cut at t and P_u = softmax_u(scale * <q, K_u>) over J:
+ *   dV_u  += P_u d_o                          (u in J)
+ *   dP_u   = <d_o, V_u>
+ *   dS_u   = P_u (dP_u - sum_w P_w dP_w)
+ *   dq     = scale * sum_u dS_u K_u
+ *   dK_u  += scale * dS_u q
+ * Every query row of the Lq rows is evaluated (queries are the last Lq tokens of each
+ * sequence, as in oracle_attn); idx is [B][Hkv][Lq][topk].
+ *   d_o [B][Lq][Hq][d] bf16; dq [B][Lq][Hq][d] doubles; dk, dv [B][Hkv][Lmax][d]
+ *   doubles (rows a sequence does not reach stay 0).
+ * Returns 0, the count of block indices outside [0, t / block] (skipped), or -1 when a
+ * row's position lies outside its sequence.  Parallel over (b, kv-head) only, so the
+ * sums into dk and dv run in a fixed order. */
+int64_t oracle_attn_backward(const oracle_params* p, const uint16_t* q, int64_t Lq, const uint16_t* k,
+                             const uint16_t* v, const int32_t* lens, int64_t Lmax, const int32_t* idx,
+                             const uint16_t* d_o, double* dq, double* dk, double* dv) {
+  const int64_t B = p->batch, Hq = p->num_q_heads, H = p->num_kv_heads, d = p->head_dim;
+  const int64_t G = Hq / H, topk = p->topk, bs = p->block_size;
+  const double scale = scale_of(p);
+  int64_t bad_idx = 0;
+  int bad_row = 0;
+  memset(dq, 0, sizeof(double) * (size_t)(B * Lq * Hq * d));
+  memset(dk, 0, sizeof(double) * (size_t)(B * H * Lmax * d));
+  memset(dv, 0, sizeof(double) * (size_t)(B * H * Lmax * d));
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(+ : bad_idx) reduction(| : bad_row)
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t g = 0; g < H; ++g) {
+      int64_t n = lens ? lens[b] : Lmax;
+      const uint16_t* kbase = k + (b * H + g) * Lmax * d;
+      const uint16_t* vbase = v + (b * H + g) * Lmax * d;
+      double* dkb = dk + (b * H + g) * Lmax * d;
+      double* dvb = dv + (b * H + g) * Lmax * d;
+      for (int64_t r = 0; r < Lq; ++r) {
+        int64_t t = n - Lq + r;
+        if (t < 0 || t >= n || n > Lmax) {
+          bad_row = 1;
+          continue;
+        }
+        int64_t cur = t / bs;
+        const int32_t* sel = idx + ((b * H + g) * Lq + r) * topk;
+        char* use = (char*)calloc((size_t)(cur + 1), 1);
+        for (int64_t s = 0; s < topk; ++s) {
+          if (sel[s] < 0) continue;
+          if (sel[s] > cur) {
+            ++bad_idx;
+            continue;
+          }
+          use[sel[s]] = 1;
+        }
+        int64_t nkeys = 0;
+        for (int64_t j = 0; j <= cur; ++j)
+          if (use[j]) nkeys += (j == cur) ? (t - j * bs + 1) : bs;
+        int64_t* pos = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nkeys > 0 ? nkeys : 1));
+        double* pr = (double*)malloc(sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 1));
+        double* dp = (double*)malloc(sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 1));
+        int64_t u = 0;
+        for (int64_t j = 0; j <= cur; ++j)
+          if (use[j])
+            for (int64_t key = j * bs; key < (j + 1) * bs && key <= t; ++key) pos[u++] = key;
+        for (int64_t hh = 0; hh < G && nkeys > 0; ++hh) {
+          int64_t h = g * G + hh; /* R9 */
+          const uint16_t* qv = q + ((b * Lq + r) * Hq + h) * d;
+          const uint16_t* gv = d_o + ((b * Lq + r) * Hq + h) * d;
+          double* dqv = dq + ((b * Lq + r) * Hq + h) * d;
+          /* probabilities */
+          double mx = -INFINITY;
+          for (u = 0; u < nkeys; ++u) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += bf16_to_double(qv[c]) * bf16_to_double(kbase[pos[u] * d + c]);
+            pr[u] = scale * dot;
+            if (pr[u] > mx) mx = pr[u];
+          }
+          double den = 0.0;
+          for (u = 0; u < nkeys; ++u) den += exp(pr[u] - mx);
+          for (u = 0; u < nkeys; ++u) pr[u] = exp(pr[u] - mx) / den;
+          /* dP_u = <d_o, V_u>, and the row's sum_u P_u dP_u */
+          double pdp = 0.0;
+          for (u = 0; u < nkeys; ++u) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += bf16_to_double(gv[c]) * bf16_to_double(vbase[pos[u] * d + c]);
+            dp[u] = dot;
+            pdp += pr[u] * dot;
+          }
+          for (u = 0; u < nkeys; ++u) {
+            const double ds = pr[u] * (dp[u] - pdp);
+            for (int64_t c = 0; c < d; ++c) {
+              dqv[c] += scale * ds * bf16_to_double(kbase[pos[u] * d + c]);
+              dkb[pos[u] * d + c] += scale * ds * bf16_to_double(qv[c]);
+              dvb[pos[u] * d + c] += pr[u] * bf16_to_double(gv[c]);
+            }
+          }
+        }
+        free(dp);
+        free(pr);
         free(pos);
         free(use);
       }

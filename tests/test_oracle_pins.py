@@ -438,3 +438,85 @@ def test_select_scores_match_an_independent_literal_scorer(G, Hkv, d, seed, scor
                 assert eligible == set(want), (b, g, t)
                 for j, s in want.items():
                     assert abs(got[j] - s) <= 1e-12 * max(abs(s), 1.0), (b, g, t, j, got[j], s)
+
+
+# --------------------------------------------------------------------- backward
+
+def masked_sdpa_grads(q, k, v, d_o, allow, scale):
+    """Reference gradients by torch autograd through dense SDPA in float64.
+    q, d_o [B, L, Hq, d]; k, v [B, Hkv, L, d]; allow [B, Hkv, L, L] boolean (query row,
+    key).  K and V are repeated over each group's heads, so the group sum of their
+    gradients is autograd's own."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    qq = q.double().permute(0, 2, 1, 3).clone().requires_grad_(True)  # [B, Hq, L, d]
+    kk = k.double().clone().requires_grad_(True)
+    vv = v.double().clone().requires_grad_(True)
+    mask = allow.repeat_interleave(G, 1)
+    o = F.scaled_dot_product_attention(qq, kk.repeat_interleave(G, 1), vv.repeat_interleave(G, 1),
+                                       attn_mask=mask, scale=scale)
+    o.backward(d_o.double().permute(0, 2, 1, 3))
+    return qq.grad.permute(0, 2, 1, 3).numpy(), kk.grad.numpy(), vv.grad.numpy()
+
+
+def block_mask(idx, L, block=64):
+    """allow[b, g, t, u]: key u lies in a block listed for row t and u <= t."""
+    B, H, R, _ = idx.shape
+    allow = torch.zeros((B, H, R, L), dtype=torch.bool)
+    keys = torch.arange(L)
+    for b in range(B):
+        for g in range(H):
+            for t in range(R):
+                sel = torch.tensor([j for j in idx[b, g, t] if j >= 0], dtype=torch.long)
+                inb = torch.zeros(L, dtype=torch.bool)
+                if len(sel):
+                    inb = (keys[:, None] // block == sel[None, :]).any(1)
+                allow[b, g, t] = inb & (keys <= t)
+    return allow
+
+
+@pytest.mark.parametrize("Hq,Hkv,all_blocks,seed", [(4, 2, True, 40), (6, 2, False, 41), (16, 1, False, 42)])
+def test_attn_backward_equals_autograd_of_masked_sdpa(Hq, Hkv, all_blocks, seed):
+    # every visible block (dense causal attention) or a random subset of each row's
+    # blocks (the block set always includes the row's own block, as the forced local
+    # block does, so every row attends to at least itself)
+    B, L, topk = 2, 300, 8
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=seed)
+    g = torch.Generator().manual_seed(seed + 100)
+    d_o = bf16(torch.randn((B, L, Hq, 128), generator=g))
+    rng = np.random.default_rng(seed)
+    idx = np.full((B, Hkv, L, topk), -1, np.int32)
+    for b in range(B):
+        for gg in range(Hkv):
+            for t in range(L):
+                cur = t // 64
+                if all_blocks:
+                    sel = np.arange(cur + 1)
+                else:
+                    others = rng.permutation(cur)[: rng.integers(0, cur + 1)]
+                    sel = np.sort(np.concatenate([others, [cur]]))
+                idx[b, gg, t, :len(sel)] = sel
+    p = oracle.Params(B, Hq, Hkv, topk=topk)
+    dq, dk, dv = oracle.attn_backward(p, as_u16(q), as_u16(k), as_u16(v), idx, as_u16(d_o))
+    rq, rk, rv = masked_sdpa_grads(q, k, v, d_o, block_mask(idx, L), 1 / math.sqrt(128))
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert np.allclose(got, ref, atol=1e-10, rtol=1e-9), float(np.abs(got - ref).max())
+
+
+def test_attn_backward_of_a_chunk_against_a_longer_cache():
+    # the last 70 rows as a chunk (queries at positions 230..299 of a 300-token cache):
+    # dq equals the full backward's rows, dk / dv the full backward's with only those rows'
+    # upstream gradient
+    B, L, Hq, Hkv, topk, m = 1, 300, 4, 2, 5, 70
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=43)
+    g = torch.Generator().manual_seed(143)
+    d_o = bf16(torch.randn((B, L, Hq, 128), generator=g))
+    d_o[:, :L - m] = 0
+    p = oracle.Params(B, Hq, Hkv, topk=topk)
+    idx = oracle.select(p, as_u16(q), oracle.compress(p, as_u16(k)))
+    dq_f, dk_f, dv_f = oracle.attn_backward(p, as_u16(q), as_u16(k), as_u16(v), idx, as_u16(d_o))
+    dq_c, dk_c, dv_c = oracle.attn_backward(p, as_u16(q[:, L - m:]), as_u16(k), as_u16(v), idx[:, :, L - m:],
+                                            as_u16(d_o[:, L - m:]), lens=np.array([L], np.int32))
+    assert np.allclose(dq_c, dq_f[:, L - m:], atol=1e-12)
+    assert np.allclose(dk_c, dk_f, atol=1e-12) and np.allclose(dv_c, dv_f, atol=1e-12)
