@@ -75,7 +75,8 @@ enum {
   INFLLMV2_OP_SELECT_PREFILL = 1,
   INFLLMV2_OP_SELECT_DECODE = 2,
   INFLLMV2_OP_ATTN_PREFILL = 3,
-  INFLLMV2_OP_ATTN_DECODE = 4
+  INFLLMV2_OP_ATTN_DECODE = 4,
+  INFLLMV2_OP_ATTN_BACKWARD = 5
 };
 
 /* Problem description shared by all calls.
@@ -220,6 +221,30 @@ INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const voi
                                 const void* v_cache, const int32_t* lens, int32_t Lmax,
                                 const int32_t* block_idx, void* o, float* lse, void* ws,
                                 size_t ws_bytes, infllmv2_stream_t stream);
+
+/* Backward of the prefill sparse attention over fixed block lists ([S] s2.1, s2.1.3:
+ * the sparse attention is trained; the top-k block choice is constant almost
+ * everywhere, so the gradients reach q, k and v through the attention only and the block
+ * lists are inputs).  With P = softmax(scale q K_J^T) over the keys J of a row's blocks
+ * cut at its position t, D = sum_d dO O:
+ *   dq = scale sum_u P_u (dO.V_u - D) K_u,  dK_u += scale P_u (dO.V_u - D) q,
+ *   dV_u += P_u dO.
+ *   q, o, d_o  bf16 [B, L, Hq, d] (o and lse from infllmv2_sparse_attn_prefill on the
+ *              same inputs; P is recomputed from lse)
+ *   k, v       bf16 [B, Hkv, L, d];  lse fp32 [B, Hq, L]
+ *   block_idx  int32 [B, Hkv, L, topk] as for the forward (unique entries per row)
+ *   dq         bf16 [B, L, Hq, d];  dk, dv bf16 [B, Hkv, L, d] (outputs)
+ *   ws         at least infllmv2_workspace_size(p, INFLLMV2_OP_ATTN_BACKWARD, L) bytes
+ *              (contents on entry do not matter; about 8 bytes x (topk / 2 + 2 d) per
+ *              (token, kv-head)).
+ * dq is deterministic; dk and dv are summed over a block's query rows by several CTAs
+ * with fp32 atomics, so their rounding may differ between runs.  Fresh sequences only
+ * (query t at position t).  WORKSPACE for a missing or short workspace, INVALID_ARG for
+ * null / misaligned pointers. */
+INFLLMV2_API int infllmv2_sparse_attn_backward(const infllmv2_params* p, const void* q, const void* k,
+                                               const void* v, const void* o, const float* lse, const void* d_o,
+                                               const int32_t* block_idx, int32_t L, void* dq, void* dk, void* dv,
+                                               void* ws, size_t ws_bytes, infllmv2_stream_t stream);
 
 /* Decode sparse attention that allocates nothing and takes no workspace.  The paper has
  * no counterpart to this entry point: it exists for callers that cannot allocate device

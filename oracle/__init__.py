@@ -91,7 +91,7 @@ def _load():
         lib.oracle_select.restype = ctypes.c_int
         lib.oracle_attn.argtypes = [P, vp, i64, vp, vp, vp, i64, vp, vp, i64, vp, vp]
         lib.oracle_attn.restype = i64
-        lib.oracle_attn_backward.argtypes = [P, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
+        lib.oracle_attn_backward.argtypes = [P, vp, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp]
         lib.oracle_attn_backward.restype = i64
         _lib = lib
     return _lib
@@ -194,10 +194,11 @@ def attn(p: Params, q, k, v, idx, lens=None, rows=None):
     return o, lse
 
 
-def attn_backward(p: Params, q, k, v, idx, d_o, lens=None):
+def attn_backward(p: Params, q, k, v, idx, d_o, lens=None, o=None):
     """Gradients of the sparse attention (block lists fixed).  q, d_o [B,Lq,Hq,d]; k, v
-    [B,Hkv,Lmax,d] (bf16 as uint16); idx [B,Hkv,Lq,topk] for every query row.  Returns
-    dq [B,Lq,Hq,d], dk and dv [B,Hkv,Lmax,d] as float64."""
+    [B,Hkv,Lmax,d] (bf16 as uint16); idx [B,Hkv,Lq,topk] for every query row; o: the
+    forward output [B,Lq,Hq,d] (float64) when the backward takes it as an input, else
+    None (exact).  Returns dq [B,Lq,Hq,d], dk and dv [B,Hkv,Lmax,d] as float64."""
     q = _u16(q)
     k = _u16(k)
     v = _u16(v)
@@ -208,11 +209,14 @@ def attn_backward(p: Params, q, k, v, idx, d_o, lens=None):
     assert idx.shape == (B, p.num_kv_heads, Lq, p.topk), idx.shape
     assert d_o.shape == q.shape
     lens_a = None if lens is None else np.ascontiguousarray(lens, dtype=np.int32)
+    o_a = None if o is None else np.ascontiguousarray(o, dtype=np.float64)
+    if o_a is not None:
+        assert o_a.shape == q.shape, o_a.shape
     dq = np.empty((B, Lq, Hq, d), dtype=np.float64)
     dk = np.empty(k.shape, dtype=np.float64)
     dv = np.empty(v.shape, dtype=np.float64)
     rc = _load().oracle_attn_backward(ctypes.byref(p._c()), _ptr(q), Lq, _ptr(k), _ptr(v), _ptr(lens_a), Lmax,
-                                      _ptr(idx), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv))
+                                      _ptr(idx), _ptr(d_o), _ptr(o_a), _ptr(dq), _ptr(dk), _ptr(dv))
     if rc < 0:
         raise ValueError("oracle_attn_backward: a query position lies outside its sequence")
     if rc > 0:

@@ -413,12 +413,14 @@ int64_t oracle_attn(const oracle_params* p, const uint16_t* q, int64_t Lq, const
  * sequence, as in oracle_attn); idx is [B][Hkv][Lq][topk].
  *   d_o [B][Lq][Hq][d] bf16; dq [B][Lq][Hq][d] doubles; dk, dv [B][Hkv][Lmax][d]
  *   doubles (rows a sequence does not reach stay 0).
+ *   o   [B][Lq][Hq][d] doubles or NULL: the forward output, when the backward takes it as
+ *       an input; then sum_w P_w dP_w is computed as <d_o, o> (equal for the exact o).
  * Returns 0, the count of block indices outside [0, t / block] (skipped), or -1 when a
  * row's position lies outside its sequence.  Parallel over (b, kv-head) only, so the
  * sums into dk and dv run in a fixed order. */
 int64_t oracle_attn_backward(const oracle_params* p, const uint16_t* q, int64_t Lq, const uint16_t* k,
                              const uint16_t* v, const int32_t* lens, int64_t Lmax, const int32_t* idx,
-                             const uint16_t* d_o, double* dq, double* dk, double* dv) {
+                             const uint16_t* d_o, const double* o, double* dq, double* dk, double* dv) {
   const int64_t B = p->batch, Hq = p->num_q_heads, H = p->num_kv_heads, d = p->head_dim;
   const int64_t G = Hq / H, topk = p->topk, bs = p->block_size;
   const double scale = scale_of(p);
@@ -485,6 +487,11 @@ int64_t oracle_attn_backward(const oracle_params* p, const uint16_t* q, int64_t 
             for (int64_t c = 0; c < d; ++c) dot += bf16_to_double(gv[c]) * bf16_to_double(vbase[pos[u] * d + c]);
             dp[u] = dot;
             pdp += pr[u] * dot;
+          }
+          if (o) { /* the forward output as given: sum_w P_w dP_w = <d_o, o> */
+            const double* ov = o + ((b * Lq + r) * Hq + h) * d;
+            pdp = 0.0;
+            for (int64_t c = 0; c < d; ++c) pdp += bf16_to_double(gv[c]) * ov[c];
           }
           for (u = 0; u < nkeys; ++u) {
             const double ds = pr[u] * (dp[u] - pdp);

@@ -103,3 +103,33 @@ def compare_attention(o_gpu: np.ndarray, o_ora: np.ndarray, lse_gpu=None, lse_or
         assert np.all(np.isfinite(lse_gpu)[finite])
         assert float(dl[finite].max()) <= LSE_MAX_ABS, f"lse max abs error {float(dl[finite].max())}"
     return mx, mean
+
+
+# Gradients of the backward pass: every error source is a bf16 rounding (of P and dS as
+# MMA operands, of the forward's O inside D = dO.O, and of the bf16 outputs), 2^-8
+# relative to the terms it rounds.  The terms' scale differs by orders of magnitude from
+# row to row (a query row that attends to 2 keys has a dq ~ 20x that of one attending to
+# a thousand; a key attended by every row has a larger dK than one attended by few), so
+# errors are measured against the RMS of their own gradient row (128 values: one (token,
+# head) of dq, one key of dK / dV), with a floor of 1e-3 x the tensor's RMS for rows whose
+# exact gradient is (nearly) zero.  A row's largest element is ~3 RMS, so the roundings
+# leave ~2^-8 x 6 RMS = 2.3e-2 RMS at most and ~2^-8 / 2 RMS on average.  Bars: max 5e-2,
+# mean 5e-3 (of the row RMS).
+GRAD_MAX_ROW_RMS = 5e-2
+GRAD_MEAN_ROW_RMS = 5e-3
+
+
+def compare_grad(g, ref, what=""):
+    """g: GPU gradient (torch, any float dtype); ref: fp64 oracle gradient (numpy); the
+    last axis is the row of 128 values.  Returns (max, mean) error over the row RMS."""
+    g = g.detach().float().cpu().numpy().astype(np.float64)
+    assert g.shape == ref.shape, (what, g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), what
+    rms_all = float(np.sqrt(np.mean(ref * ref)))
+    assert rms_all > 0, what
+    row_rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    rel = np.abs(g - ref) / np.maximum(row_rms, 1e-3 * rms_all)
+    mx, mean = float(rel.max()), float(rel.mean())
+    assert mx <= GRAD_MAX_ROW_RMS, f"{what}: max abs error {mx:.3g} x its row's RMS"
+    assert mean <= GRAD_MEAN_ROW_RMS, f"{what}: mean abs error {mean:.3g} x its row's RMS"
+    return mx, mean

@@ -175,3 +175,22 @@ def test_score_and_pool_modes_are_checked(lib):
     assert f(cp(score_mode=2)) == _lib.ERR_INVALID_ARG
     assert f(cp(pool_mode=-1)) == _lib.ERR_INVALID_ARG
     assert ctypes.sizeof(_lib.CParams) == 13 * 4  # the C struct: 10 int32, a float, 2 int32
+
+
+def test_backward_rejects_bad_arguments_before_launch(lib):
+    good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    f = lib.infllmv2_sparse_attn_backward
+    need = lib.infllmv2_workspace_size(cp(), _lib.OP_ATTN_BACKWARD, 1024)
+    assert need > 0
+    args = [good] * 7 + [1024] + [good] * 3
+    assert f(cp(), *args, None, 0, None) == _lib.ERR_WORKSPACE
+    assert f(cp(), *args, good, need - 1, None) == _lib.ERR_WORKSPACE
+    bad = list(args)
+    bad[4] = good + 2  # lse must be 4-byte aligned
+    assert f(cp(), *bad, good, need, None) == _lib.ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = None
+    assert f(cp(), *bad, good, need, None) == _lib.ERR_INVALID_ARG
+    bad = list(args)
+    bad[7] = 0
+    assert f(cp(), *bad, good, need, None) == _lib.ERR_INVALID_ARG

@@ -520,3 +520,23 @@ def test_attn_backward_of_a_chunk_against_a_longer_cache():
                                             as_u16(d_o[:, L - m:]), lens=np.array([L], np.int32))
     assert np.allclose(dq_c, dq_f[:, L - m:], atol=1e-12)
     assert np.allclose(dk_c, dk_f, atol=1e-12) and np.allclose(dv_c, dv_f, atol=1e-12)
+
+
+def test_attn_backward_with_the_exact_output_given_equals_the_exact_backward():
+    # the backward that takes the forward output as an input forms sum_u P_u dP_u as
+    # <d_o, o>; with the exact o it is the exact backward
+    B, L, Hq, Hkv, topk = 1, 400, 4, 2, 5
+    q, k, v = rand_inputs(B, L, Hq, Hkv, seed=44)
+    g = torch.Generator().manual_seed(144)
+    d_o = bf16(torch.randn((B, L, Hq, 128), generator=g))
+    p = oracle.Params(B, Hq, Hkv, topk=topk)
+    idx = oracle.select(p, as_u16(q), oracle.compress(p, as_u16(k)))
+    o, _ = oracle.attn(p, as_u16(q), as_u16(k), as_u16(v), idx)
+    exact = oracle.attn_backward(p, as_u16(q), as_u16(k), as_u16(v), idx, as_u16(d_o))
+    given = oracle.attn_backward(p, as_u16(q), as_u16(k), as_u16(v), idx, as_u16(d_o), o=o)
+    for a, b in zip(exact, given):
+        assert np.allclose(a, b, atol=1e-11, rtol=1e-9)
+    # and a perturbed o changes dq and dk but not dv (dV_u = sum P_u d_o has no D)
+    worse = oracle.attn_backward(p, as_u16(q), as_u16(k), as_u16(v), idx, as_u16(d_o), o=o * 1.01)
+    assert not np.allclose(worse[0], exact[0]) and not np.allclose(worse[1], exact[1])
+    assert np.array_equal(worse[2], exact[2])

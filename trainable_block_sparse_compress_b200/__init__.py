@@ -15,6 +15,7 @@ from .ops import (  # noqa: F401
     prefill,
     prefill_chunk,
     select_blocks_chunk,
+    sparse_attn_backward,
     sparse_attn_chunk,
     select_blocks_decode,
     select_blocks_prefill,

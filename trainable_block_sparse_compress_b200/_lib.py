@@ -31,6 +31,7 @@ OP_SELECT_PREFILL = 1
 OP_SELECT_DECODE = 2
 OP_ATTN_PREFILL = 3
 OP_ATTN_DECODE = 4
+OP_ATTN_BACKWARD = 5
 
 MAX_SEQ_LEN = 262144
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -70,6 +71,8 @@ SIGNATURES = {
     "infllmv2_sparse_attn_prefill": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_chunk": (_int, [_P, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "infllmv2_sparse_attn_decode": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "infllmv2_sparse_attn_backward": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz,
+                                              _vp]),
     "infllmv2_sparse_attn_decode_noalloc": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "infllmv2_append_kv": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
     "infllmv2_workspace_size": (_sz, [_P, _int, _i32]),

@@ -16,6 +16,7 @@
 #include "../../include/infllmv2.h"
 #include "append.cuh"
 #include "attn.cuh"
+#include "attn_bwd.cuh"
 #include "attn_dec.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -212,6 +213,30 @@ int select_cluster(const infllmv2_params* p, int64_t nk) {
   return c;
 }
 
+// Workspace of the backward pass, in order (each part 256-byte aligned): D [B, Hq, L]
+// fp32; cnt, cursor, off [n] and segoff [n + 1] int32 (n = B * Hkv * blocks); the row
+// lists [B * Hkv * L * topk] int32; dK and dV accumulators [B, Hkv, L, d] fp32.
+struct BwdLayout {
+  size_t delta, cnt, cursor, off, segoff, list, dk, dv, total;
+  long long n;
+};
+BwdLayout bwd_layout(const infllmv2_params* p, int32_t L) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  BwdLayout w;
+  const size_t B = p->batch, Hq = p->num_q_heads, Hkv = p->num_kv_heads;
+  w.n = static_cast<long long>(B * Hkv * num_blocks(L));
+  w.delta = 0;
+  w.cnt = up(w.delta + B * Hq * L * 4);
+  w.cursor = up(w.cnt + w.n * 4);
+  w.off = up(w.cursor + w.n * 4);
+  w.segoff = up(w.off + w.n * 4);
+  w.list = up(w.segoff + (w.n + 1) * 4);
+  w.dk = up(w.list + B * Hkv * static_cast<size_t>(L) * p->topk * 4);
+  w.dv = up(w.dk + B * Hkv * static_cast<size_t>(L) * kHeadDim * 4);
+  w.total = up(w.dv + B * Hkv * static_cast<size_t>(L) * kHeadDim * 4);
+  return w;
+}
+
 size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
   if (check_params(p) != INFLLMV2_OK || check_len(L) != INFLLMV2_OK) return static_cast<size_t>(-1);
   switch (op) {
@@ -221,6 +246,8 @@ size_t ws_size(const infllmv2_params* p, int op, int32_t L) {
       return 0;
     case INFLLMV2_OP_SELECT_DECODE:
       return 0;
+    case INFLLMV2_OP_ATTN_BACKWARD:
+      return bwd_layout(p, L).total;
     case INFLLMV2_OP_ATTN_DECODE: {
       const DecodePlan d = decode_plan(p);
       if (d.cluster > 0) return 0;
@@ -536,6 +563,77 @@ int infllmv2_sparse_attn_chunk(const infllmv2_params* p, const void* q, int32_t 
   if ((st = check_chunk(Lq, q_lens, kv_lens, Lmax)) != INFLLMV2_OK) return st;
   return attn_prefill(p, q, Lq, k, v, q_lens, kv_lens, Lmax, block_idx, o, lse,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_sparse_attn_backward(const infllmv2_params* p, const void* q, const void* k, const void* v,
+                                  const void* o, const float* lse, const void* d_o, const int32_t* block_idx, int32_t L,
+                                  void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(L)) != INFLLMV2_OK) return st;
+  if (!q || !k || !v || !o || !lse || !d_o || !block_idx || !dq || !dk || !dv) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(block_idx) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return INFLLMV2_ERR_INVALID_ARG;
+  const BwdLayout w = bwd_layout(p, L);
+  if (ws == nullptr || ws_bytes < w.total || !aligned16(ws)) return INFLLMV2_ERR_WORKSPACE;
+  const long long rows = static_cast<long long>(p->batch) * p->num_kv_heads * L;
+  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * L * p->num_q_heads;
+  if (rows * p->topk > 0x7fffffffLL || q_rows > 0x7fffffffULL || w.n + 1 > 0x7fffffffLL)
+    return INFLLMV2_ERR_UNSUPPORTED;  // 32-bit row lists and TMA rows
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* wb = static_cast<unsigned char*>(ws);
+  BwdParams a;
+  a.idx = block_idx;
+  a.lse = lse;
+  a.delta = reinterpret_cast<float*>(wb + w.delta);
+  a.cnt = reinterpret_cast<int32_t*>(wb + w.cnt);
+  a.off = reinterpret_cast<int32_t*>(wb + w.off);
+  a.segoff = reinterpret_cast<int32_t*>(wb + w.segoff);
+  a.list = reinterpret_cast<int32_t*>(wb + w.list);
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = p->num_q_heads / p->num_kv_heads;
+  a.L = L;
+  a.topk = p->topk;
+  a.nblk = static_cast<int>(num_blocks(L));
+  a.scale_log2 = scale_log2(p);
+  a.scale = a.scale_log2 / 1.4426950408889634f;
+  a.num_items = rows;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk32 = reinterpret_cast<float*>(wb + w.dk);
+  a.dv32 = reinterpret_cast<float*>(wb + w.dv);
+  CUtensorMap tq, tdo, tk, tv;
+  if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tdo, d_o, q_rows, kGroupRows) ||
+      !make_map(&tk, k, static_cast<uint64_t>(rows), kBlock) || !make_map(&tv, v, static_cast<uint64_t>(rows), kBlock))
+    return INFLLMV2_ERR_CUDA;
+  // counters and the fp32 accumulators start at zero
+  if (cudaMemsetAsync(wb + w.cnt, 0, w.off - w.cnt, s) != cudaSuccess ||
+      cudaMemsetAsync(wb + w.dk, 0, w.total - w.dk, s) != cudaSuccess)
+    return INFLLMV2_ERR_CUDA;
+  const int n = static_cast<int>(w.n);
+  bwd_delta_kernel<<<static_cast<unsigned>((q_rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(d_o), static_cast<const __nv_bfloat16*>(o), p->batch, L, p->num_q_heads,
+      const_cast<float*>(a.delta));
+  const unsigned rgrid = static_cast<unsigned>((rows + 255) / 256);
+  bwd_count_kernel<<<rgrid, 256, 0, s>>>(block_idx, static_cast<int>(rows), L, p->topk, a.nblk,
+                                         const_cast<int32_t*>(a.cnt));
+  bwd_scan_kernel<<<1, 1024, 0, s>>>(a.cnt, n, const_cast<int32_t*>(a.off), const_cast<int32_t*>(a.segoff));
+  bwd_fill_kernel<<<rgrid, 256, 0, s>>>(block_idx, static_cast<int>(rows), L, p->topk, a.nblk, a.off,
+                                        reinterpret_cast<int32_t*>(wb + w.cursor), const_cast<int32_t*>(a.list));
+  if ((st = launch_status()) != INFLLMV2_OK) return st;
+  const size_t smem_q = bwd_dq_smem_bytes(), smem_kv = bwd_dkdv_smem_bytes();
+  if ((st = set_smem(reinterpret_cast<const void*>(bwd_dq_kernel), smem_q)) != INFLLMV2_OK) return st;
+  if ((st = set_smem(reinterpret_cast<const void*>(bwd_dkdv_kernel), smem_kv)) != INFLLMV2_OK) return st;
+  bwd_dq_kernel<<<static_cast<unsigned>(std::min<long long>(rows, num_sms())), kBwdThreads, smem_q, s>>>(tq, tdo, tk,
+                                                                                                        tv, a);
+  bwd_dkdv_kernel<<<static_cast<unsigned>(num_sms()), kBwdThreads, smem_kv, s>>>(tq, tdo, tk, tv, a);
+  const long long n4 = rows * kHeadDim / 4;
+  bwd_cast_kernel<<<static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 8LL * num_sms())), 256, 0, s>>>(
+      reinterpret_cast<const float4*>(a.dk32), reinterpret_cast<const float4*>(a.dv32), n4, static_cast<uint2*>(dk),
+      static_cast<uint2*>(dv));
+  return launch_status();
 }
 
 int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,

@@ -213,6 +213,31 @@ def sparse_attn_chunk(p: Params, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     return out, lse
 
 
+def sparse_attn_backward(p: Params, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                         lse: torch.Tensor, d_o: torch.Tensor, block_idx: torch.Tensor,
+                         ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients of the prefill sparse attention with the block lists fixed: q, o, d_o bf16
+    [B, L, Hq, d], k, v bf16 [B, Hkv, L, d], lse fp32 [B, Hq, L] from the forward ->
+    dq [B, L, Hq, d], dk, dv [B, Hkv, L, d] (bf16)."""
+    B, L, Hq, d = q.shape
+    for t, name in ((q, "q"), (o, "o"), (d_o, "d_o")):
+        _need(t, name, torch.bfloat16, (p.batch, L, p.num_q_heads, p.head_dim))
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, name, torch.bfloat16, (p.batch, p.num_kv_heads, L, p.head_dim))
+    _need(lse, "lse", torch.float32, (p.batch, p.num_q_heads, L))
+    _need(block_idx, "block_idx", torch.int32, (p.batch, p.num_kv_heads, L, p.topk))
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws = _workspace(p, _lib.OP_ATTN_BACKWARD, L, ws, q.device)
+    nbytes = ws.numel() * ws.element_size()
+    st = _lib.load().infllmv2_sparse_attn_backward(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                                   _ptr(d_o), _ptr(block_idx), L, _ptr(dq), _ptr(dk), _ptr(dv),
+                                                   _ptr(ws), nbytes, _stream())
+    _lib.check("infllmv2_sparse_attn_backward", st)
+    return dq, dk, dv
+
+
 def sparse_attn_decode(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                        lens: torch.Tensor, block_idx: torch.Tensor, out: Optional[torch.Tensor] = None,
                        lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
