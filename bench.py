@@ -14,6 +14,7 @@ sequence: weak scaling, no collective on the data path.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -282,6 +283,12 @@ def run_ours(args, rank, world, device):
         result["decode"] = run_decode(args, args.decode_workload, rank, world, device, pk, peak_src)
         if args.decode_workload_2:
             result["decode_2"] = run_decode(args, args.decode_workload_2, rank, world, device, pk, peak_src)
+    if rank == 0 and not args.no_extras:
+        try:
+            result["extras"] = run_extras(args, device, pk, peak_src)
+        except Exception as e:  # the extra timings never cost the main line
+            result["extras"] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, wl, x)
     return result
@@ -450,6 +457,95 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     }
 
 
+# ------------------------------------------------- chunks, variants, backward
+
+def _time_ms(fn, reps, stream):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    fn()
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        fn()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    return ev[0].elapsed_time(ev[1]) / reps
+
+
+def run_extras(args, device, pk, peak_src):
+    """The other calls of the library, each timed with CUDA events on its own (rank 0):
+    a prefill chunk against a 128K cache, the selection variants at 128K, and the
+    backward pass at 32K.  Inputs are the seeded workloads of the parity tests."""
+    stream = torch.cuda.current_stream()
+    reps = max(3, min(args.steps, 10))
+    tc_peak = pk["bf16_tflops"]
+    out = {"peak_source": f"{peak_src} (bf16_tflops, burst)"}
+
+    wl = WORKLOADS["prefill_128k"]
+    p = ops.Params.from_workload(wl)
+    L = wl.seq_len
+    x = make_inputs(wl, seed=args.seed)
+    q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
+    del x
+    kc = ops.compress_keys(p, k)
+
+    # a chunk of the last m queries against the whole cache (positions L-m .. L-1)
+    m = 8192
+    qc = q[:, L - m:].contiguous()
+    idx_c = torch.empty((p.batch, p.num_kv_heads, m, p.topk), dtype=torch.int32, device=device)
+    o_c = torch.empty_like(qc)
+
+    def chunk_step():
+        ops.select_blocks_chunk(p, qc, kc, L, out=idx_c)
+        ops.sparse_attn_chunk(p, qc, k, v, idx_c, out=o_c, want_lse=False)
+    ms_chunk = _time_ms(chunk_step, reps, stream)
+    ms_attn_c = _time_ms(lambda: ops.sparse_attn_chunk(p, qc, k, v, idx_c, out=o_c, want_lse=False), reps, stream)
+    t = np.arange(L - m, L, dtype=np.int64)
+    cur = t // 64
+    keys = 64 * (np.minimum(p.topk, cur + 1) - 1) + (t - 64 * cur + 1)
+    fl = 4 * p.head_dim * p.num_q_heads * int(keys.sum())
+    out["chunk"] = {"workload": f"prefill_128k cache, chunk of the last {m} queries", "ms": ms_chunk,
+                    "tokens_per_s": m / (ms_chunk / 1e3), "attn_ms": ms_attn_c,
+                    "attn_tflops": fl / ms_attn_c / 1e9, "attn_frac": fl / ms_attn_c / 1e9 / tc_peak}
+    del qc, idx_c, o_c
+
+    # selection variants over the whole 128K prefill
+    idx = torch.empty((p.batch, p.num_kv_heads, L, p.topk), dtype=torch.int32, device=device)
+    sel_flops, _, _ = prefill_flops(p, L)
+    var = {}
+    for sm, pm in ((0, 0), (1, 0), (0, 1), (1, 1)):
+        pv = dataclasses.replace(p, score_mode=sm, pool_mode=pm)
+        ms_sel = _time_ms(lambda: ops.select_blocks_prefill(pv, q, kc, out=idx), reps, stream)
+        flops = sel_flops if sm == 0 else sel_flops // 2  # logit-sum: one pass over the kernels
+        var[f"score{sm}_pool{pm}"] = {"ms": ms_sel, "tflops": flops / ms_sel / 1e9,
+                                      "frac": flops / ms_sel / 1e9 / tc_peak}
+    out["select_variants_128k"] = var
+    del q, k, v, kc, idx
+    torch.cuda.empty_cache()
+
+    # backward at 32K: the forward once, then the backward timed alone
+    wl = WORKLOADS["prefill_32k"]
+    p = ops.Params.from_workload(wl)
+    L = wl.seq_len
+    x = make_inputs(wl, seed=args.seed)
+    q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
+    g = torch.Generator().manual_seed(args.seed + 7)
+    d_o = torch.randn(x.q.shape, generator=g).to(torch.bfloat16).to(device)
+    del x
+    o, lse, idx, kc = ops.prefill(p, q, k, v)
+    ws = torch.empty(ops.workspace_size(p, 5, L), dtype=torch.uint8, device=device)
+    ms_bwd = _time_ms(lambda: ops.sparse_attn_backward(p, q, k, v, o, lse, d_o, idx, ws=ws), reps, stream)
+    _, attn_flops, _ = prefill_flops(p, L)
+    bwd_flops = attn_flops * 5 // 2  # recompute S, dP, dV, dK, dQ: 5 products of the forward's 2
+    out["backward_32k"] = {"workload": "prefill_32k (B=1, L=32768, 32/2 heads, top-96)", "ms": ms_bwd,
+                           "tflops": bwd_flops / ms_bwd / 1e9, "frac": bwd_flops / ms_bwd / 1e9 / tc_peak,
+                           "algorithmic_flops": bwd_flops,
+                           "note": "kernels run 7 products (S and dP are recomputed in both passes), "
+                                   "on m16n8k16 tensor-core MMAs"}
+    del q, k, v, d_o, o, lse, idx, kc, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_rows_time(wl, x, rows):
@@ -510,6 +606,25 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_run(name, device):
+    """The hot path of one workload, twice (a warm-up and one more run), for single-kernel
+    profiler captures on small cases: prefill (compress, select, attend) or a decode step
+    (compress the caches, select, attend).  Prints nothing."""
+    wl = WORKLOADS[name]
+    p = ops.Params.from_workload(wl)
+    x = make_inputs(wl, seed=0)
+    q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
+    for _ in range(2):
+        if wl.mode == "prefill":
+            ops.prefill(p, q, k, v)
+        else:
+            lens = x.lens.to(device)
+            kc = ops.compress_keys(p, k, lens=lens)
+            ops.decode(p, q, k, v, kc, lens, wl.seq_len)
+    torch.cuda.synchronize()
+    assert ops.device_error(clear=True) == 0
+
+
 # ---------------------------------------------------------------------- main
 
 def main():
@@ -523,11 +638,18 @@ def main():
     ap.add_argument("--decode-workload-2", default="decode_32k", help="second decode line ('' for none)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the chunk / variant / backward timings")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-rows", type=int, default=96)
+    ap.add_argument("--profile-run", default=None, metavar="WORKLOAD",
+                    help="run WORKLOAD's hot path twice and exit (for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.profile_run:
+        lib_build.build()
+        profile_run(args.profile_run, torch.device("cuda", 0))
+        return
 
     ri = dist.rank_info()
     rank, world, local = ri.rank, ri.world, ri.local
