@@ -26,6 +26,10 @@
 //          states are merged (thread = output column d) and O and the log-sum-exp are
 //          written;
 //   warp 8 also loads the query tile and compacts the block list of each item.
+// In a prefill chunk the cache may end inside the query's own block; key rows past the
+// cache end hold arbitrary values, so the V producer loads that one pair onto a barrier of
+// its own, zeroes those rows in shared memory and only then marks the pair loaded (their
+// P is 0, and 0 x anything stays 0 only when "anything" is finite).
 #pragma once
 #include "attn.cuh"
 #include "common.cuh"
@@ -51,7 +55,9 @@ constexpr uint32_t kAtTmemCols = kAtOCol + 64 <= 128 ? 128 : (kAtOCol + 64 <= 25
 struct AtSmem {
   uint64_t k_full[kAtKStages], k_empty[kAtKStages], v_full[kAtVStages], v_empty[kAtVStages], q_full[2], q_empty[2];
   uint64_t s_full[kAtBufs], p_full[kAtBufs], pv_done[kAtBufs], mma_done[2];
+  uint64_t vtail;   // the V producer's own barrier for the pair that straddles the cache end
   int n_blocks[2];
+  int tail_pos[2];  // list position of the block that straddles the cache end (-1: none)
   int list[2][kMaxTopk];
   float red[kAtSoftWGs][4][kGroupRows];
   float mstate[kAtSoftWGs][kGroupRows], lstate[kAtSoftWGs][kGroupRows];
@@ -65,6 +71,16 @@ constexpr size_t attn_tc_smem_bytes() {
          sizeof(AtSmem);
 }
 static_assert(attn_tc_smem_bytes() <= 227 * 1024, "shared memory of one CTA");
+
+// Zeroes V rows r0 .. 63 of the block whose 64 rows start at `vs` in a pair slot (both
+// 64-column halves).  Runs only for the block that straddles a cache end.
+__device__ __noinline__ void zero_v_rows(unsigned char* vs, int r0) {
+  for (int r = max(r0, 0); r < kBlock; ++r)
+    for (int c = 0; c < 8; ++c) {
+      *reinterpret_cast<uint4*>(vs + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(vs + kAtKHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+    }
+}
 
 // Per-lane result of a 32-lane max / sum over 16 values: lane L holds the total for
 // value index L >> 1 (lanes 2h and 2h+1 agree).  16 shuffles.
@@ -152,6 +168,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     mbar_init(&S.mma_done[0], 1);
     mbar_init(&S.mma_done[1], 1);
+    mbar_init(&S.vtail, 1);
     S.abort = 0;
     fence_mbar_init();
   }
@@ -173,13 +190,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     uint32_t gpair = 0;
     int it = 0;
+    long long k_last[kAtKStages];  // last pair loaded into each K stage (lane 0), for the drain
+    int q_last[2] = {-1, -1};      // last use of each query-tile slot
+    for (int st = 0; st < kAtKStages; ++st) k_last[st] = -1;
     for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
       const int slot = it & 1, use = it >> 1;
       if (use > 0) mbar_wait(&S.q_empty[slot], (use - 1) & 1, &S.abort);
       const AttnItem a = attn_item(p, item);
       const int cur = a.t >= 0 ? a.t / kBlock : -1;
       const int32_t* row = p.idx + ((a.bg * p.Lq + a.row) * static_cast<long long>(p.topk));
-      int count = 0;
+      const int tail_j = (a.kv_len % kBlock) != 0 ? a.kv_len / kBlock : -1;  // straddles the cache end
+      int count = 0, tail = -1;
       for (int e0 = 0; e0 < p.topk; e0 += 32) {
         const int e = e0 + lane;
         const int j = (e < p.topk && a.valid) ? row[e] : -1;
@@ -187,17 +208,25 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const unsigned msk = __ballot_sync(0xffffffffu, ok);
         const int pos = count + __popc(msk & ((1u << lane) - 1u));
         if (ok) S.list[slot][pos] = j;
+        const unsigned tm = __ballot_sync(0xffffffffu, ok && j == tail_j);
+        if (tm != 0u) tail = count + __popc(msk & ((1u << (__ffs(tm) - 1)) - 1u));
         count += __popc(msk);
       }
-      if (lane == 0) S.n_blocks[slot] = count;
+      if (lane == 0) {
+        S.n_blocks[slot] = count;
+        S.tail_pos[slot] = tail;
+      }
       __threadfence_block();
       __syncwarp();
       const int np = (count + 1) / 2;
       if (lane == 0) {
         unsigned char* qs = qtiles + slot * kQTileBytes;
-        mbar_arrive_expect_tx(&S.q_full[slot], kQTileBytes);
-        tma_load_2d(qs, &tm_q, &S.q_full[slot], 0, a.qrow);
-        tma_load_2d(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow);
+        if (!S.abort) {
+          mbar_arrive_expect_tx(&S.q_full[slot], kQTileBytes);
+          tma_load_2d(qs, &tm_q, &S.q_full[slot], 0, a.qrow);
+          tma_load_2d(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow);
+          q_last[slot] = use;
+        }
         const long long kvrow0 = a.bg * p.Lmax;
         for (int i = 0; i < np; ++i, ++gpair) {
           const int st = static_cast<int>(gpair % kAtKStages);
@@ -209,6 +238,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
           const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
           unsigned char* sk = kring + st * kAtSlotBytes;
+          k_last[st] = gpair;
           mbar_arrive_expect_tx(&S.k_full[st], kAtSlotBytes);
           // rows 0-63 of each 128-key half: block a; rows 64-127: block b (zeros when absent)
           tma_load_2d(sk, &tm_k, &S.k_full[st], 0, ra);
@@ -221,6 +251,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       gpair = __shfl_sync(0xffffffffu, gpair, 0);
     }
+    if (lane == 0 && S.abort) {  // let every copy this warp issued land before the CTA ends
+      for (int st = 0; st < kAtKStages; ++st)
+        if (k_last[st] >= 0) mbar_wait_drain(&S.k_full[st], static_cast<uint32_t>((k_last[st] / kAtKStages) & 1));
+      for (int sl = 0; sl < 2; ++sl)
+        if (q_last[sl] >= 0) mbar_wait_drain(&S.q_full[sl], static_cast<uint32_t>(q_last[sl] & 1));
+    }
     return;
   }
 
@@ -229,13 +265,16 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // V pairs are loaded through their own ring, so a V slot is held only until its PV,
     // and K slots recycle right after their QK.
     if (lane == 0) {
-      uint32_t gpair = 0;
+      uint32_t gpair = 0, n_tail = 0;
       int it = 0;
+      long long v_last[kAtVStages];  // last pair loaded into each V stage, for the drain
+      for (int st = 0; st < kAtVStages; ++st) v_last[st] = -1;
       for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
         const int slot = it & 1, use = it >> 1;
         mbar_wait(&S.q_full[slot], use & 1, &S.abort);  // the item's block list is ready
         const AttnItem a = attn_item(p, item);
         const int count = S.n_blocks[slot];
+        const int tail = S.tail_pos[slot];
         const int np = (count + 1) / 2;
         const long long kvrow0 = a.bg * p.Lmax;
         for (int i = 0; i < np; ++i, ++gpair) {
@@ -248,14 +287,33 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
           const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
           unsigned char* sv = vring + st * kAtSlotBytes;
-          mbar_arrive_expect_tx(&S.v_full[st], kAtSlotBytes);
-          tma_load_2d(sv, &tm_v, &S.v_full[st], 0, ra);
-          tma_load_2d(sv + kAtKHalf, &tm_v, &S.v_full[st], 64, ra);
-          tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.v_full[st], 0, rb);
-          tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.v_full[st], 64, rb);
+          v_last[st] = gpair;
+          if ((tail >> 1) != i) {  // (tail == -1: no straddling block in the item)
+            mbar_arrive_expect_tx(&S.v_full[st], kAtSlotBytes);
+            tma_load_2d(sv, &tm_v, &S.v_full[st], 0, ra);
+            tma_load_2d(sv + kAtKHalf, &tm_v, &S.v_full[st], 64, ra);
+            tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.v_full[st], 0, rb);
+            tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.v_full[st], 64, rb);
+          } else {
+            // the pair with the block that straddles the cache end: load it here, zero the
+            // rows past the end, then mark it loaded
+            mbar_arrive_expect_tx(&S.vtail, kAtSlotBytes);
+            tma_load_2d(sv, &tm_v, &S.vtail, 0, ra);
+            tma_load_2d(sv + kAtKHalf, &tm_v, &S.vtail, 64, ra);
+            tma_load_2d(sv + kKvTileBytes / 2, &tm_v, &S.vtail, 0, rb);
+            tma_load_2d(sv + kAtKHalf + kKvTileBytes / 2, &tm_v, &S.vtail, 64, rb);
+            mbar_wait_drain(&S.vtail, n_tail & 1);
+            ++n_tail;
+            zero_v_rows(sv + (tail & 1) * (kKvTileBytes / 2), a.kv_len - S.list[slot][tail] * kBlock);
+            fence_proxy_async_smem();  // the generic writes before the MMA's reads
+            mbar_arrive(&S.v_full[st]);
+          }
         }
         mbar_arrive(&S.q_empty[slot]);  // done with the item's block list
       }
+      if (S.abort)  // let every copy this thread issued land before the CTA ends
+        for (int st = 0; st < kAtVStages; ++st)
+          if (v_last[st] >= 0) mbar_wait_drain(&S.v_full[st], static_cast<uint32_t>((v_last[st] / kAtVStages) & 1));
     }
     return;
   }
@@ -292,28 +350,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           }
           umma_commit(&S.q_empty[slot]);  // the item's query tile is no longer read
         } else {
-          const int n_blk = S.n_blocks[slot];
-          // key rows at or past the sequence's cached length (a chunk's cache may end inside
-          // the query's own block) hold arbitrary values: their V rows are zeroed in shared
-          // memory before the PV, so that they contribute exactly 0 (their P is 0)
-          const int kv_len = attn_item(p, item).kv_len;
           for (int i = 0; i < np; ++i) {
             const uint32_t pp = gp + i;
             mbar_wait(&S.p_full[pp % kAtBufs], (pp / kAtBufs) & 1, &S.abort);
             mbar_wait(&S.v_full[pp % kAtVStages], (pp / kAtVStages) & 1, &S.abort);
-            bool zeroed = false;
-            for (int hb = 0; hb < 2 && 2 * i + hb < n_blk; ++hb) {
-              const int r0 = kv_len - S.list[slot][2 * i + hb] * kBlock;  // first row past the cache
-              if (r0 >= kBlock) continue;
-              unsigned char* vs = vring + (pp % kAtVStages) * kAtSlotBytes + hb * (kKvTileBytes / 2);
-              for (int r = max(r0, 0); r < kBlock; ++r)
-                for (int c = 0; c < 8; ++c) {
-                  *reinterpret_cast<uint4*>(vs + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                  *reinterpret_cast<uint4*>(vs + kAtKHalf + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                }
-              zeroed = true;
-            }
-            if (zeroed) fence_proxy_async_smem();  // the generic writes before the MMA's reads
             tc_fence_after();
             const uint32_t obuf = tmem + kAtOCol + static_cast<uint32_t>(2 * (it & 1) + (pp & 1)) * 16u;
             const uint32_t vb = smem_u32(vring + (pp % kAtVStages) * kAtSlotBytes);
