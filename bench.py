@@ -61,6 +61,8 @@ KERNEL_SOURCES = {
     "attn_kernel": ["attn.cuh", "common.cuh", "infllmv2.cu"],
     "select_decode_kernel": ["select_decode.cuh", "select_prefill.cuh", "topk.cuh", "common.cuh", "infllmv2.cu"],
     "attn_decode_cluster_kernel": ["attn_dec.cuh", "attn.cuh", "common.cuh", "infllmv2.cu"],
+    "decode_step_kernel": ["decode_step.cuh", "select_decode.cuh", "attn_dec.cuh", "select_prefill.cuh", "topk.cuh",
+                           "attn.cuh", "common.cuh", "infllmv2.cu"],
 }
 
 
@@ -359,8 +361,9 @@ def run_e2e(args, p, x, device):
 
 
 def run_decode(args, workload, rank, world, device, pk, peak_src):
-    """One decode step (select -> attention) over filled caches, L2 flushed before every
-    step (outside the timed events).  Inputs: the same seed as the parity tests."""
+    """One decode step (selection -> attention, fused in one launch) over filled caches, L2
+    flushed before every step (outside the timed events).  Inputs: the same seed as the
+    parity tests.  The two separate calls are timed too, for the per-kernel split."""
     wl = WORKLOADS[workload]
     p = ops.Params.from_workload(wl)
     x = make_inputs(wl, seed=dist.rank_seed(args.seed, rank))
@@ -376,8 +379,7 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     stream = torch.cuda.current_stream()
 
     def step():
-        ops.select_blocks_decode(p, q, kc, lens, Lmax, out=idx, ws=ws_s)
-        ops.sparse_attn_decode(p, q, k, v, lens, idx, out=o, lse=lse, ws=ws_a)
+        ops.decode_step(p, q, k, v, kc, lens, block_idx=idx, out=o, lse=lse)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -387,8 +389,6 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         flush.zero_()  # evict the caches' lines from L2 ...
         flush.view(torch.int32).sum()  # ... and leave it clean, so no write-back lands in the step
 
-    # the step: selection then attention back to back (the attention launch overlaps the
-    # end of the selection), events only around the pair
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
     for s in range(n):
         flush_l2()
@@ -397,10 +397,17 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         ev[s][1].record(stream)
     torch.cuda.synchronize()
     step_us = [ev[s][0].elapsed_time(ev[s][1]) * 1e3 for s in range(n)]
-    # per-kernel breakdown in a separate pass (an event between the two kernels keeps the
-    # attention from starting early, so these add up to a little more than the step)
+    # the two separate calls: the pair (the attention launch overlaps the end of the
+    # selection), then each kernel alone (an event between them keeps the attention from
+    # starting early)
+    evp = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
     for s in range(n):
+        flush_l2()
+        evp[s][0].record(stream)
+        ops.select_blocks_decode(p, q, kc, lens, Lmax, out=idx, ws=ws_s)
+        ops.sparse_attn_decode(p, q, k, v, lens, idx, out=o, lse=lse, ws=ws_a)
+        evp[s][1].record(stream)
         flush_l2()
         evk[s][0].record(stream)
         ops.select_blocks_decode(p, q, kc, lens, Lmax, out=idx, ws=ws_s)
@@ -408,6 +415,7 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         ops.sparse_attn_decode(p, q, k, v, lens, idx, out=o, lse=lse, ws=ws_a)
         evk[s][2].record(stream)
     torch.cuda.synchronize()
+    pair_us = [evp[s][0].elapsed_time(evp[s][1]) * 1e3 for s in range(n)]
     sel_us = [evk[s][0].elapsed_time(evk[s][1]) * 1e3 for s in range(n)]
     att_us = [evk[s][1].elapsed_time(evk[s][2]) * 1e3 for s in range(n)]
     us = statistics.median(step_us)
@@ -433,6 +441,7 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
     sel_med, att_med = statistics.median(sel_us), statistics.median(att_us)
+    tr_f = dram_traffic("decode_step_kernel", workload)
     tr_s = dram_traffic("select_decode_kernel", workload)
     tr_a = dram_traffic(att_kernel, workload)
     return {
@@ -441,17 +450,20 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         "l2": "flushed before every step (write then read a 2x L2 buffer, outside the timed events)",
         "roofline": {"bound": "hbm", "achieved": (sel_b + att_b) / us / 1e3, "peak": hbm, "unit": "GB/s",
                      "frac": (sel_b + att_b) / us / 1e3 / hbm, "algorithmic_bytes": sel_b + att_b,
-                     "traffic": tr_s + tr_a if tr_s is not None and tr_a is not None else None,
-                     "peak_source": f"{peak_src} (hbm_gbs)"},
+                     "traffic": tr_f, "peak_source": f"{peak_src} (hbm_gbs)"},
         "kernels": {
-            "select": {"kernel": "select_decode_kernel", "us": sel_med, "algorithmic_bytes": sel_b,
-                       "achieved_GBps": sel_b / sel_med / 1e3,
-                       "traffic": tr_s},
-            "attn": {"kernel": att_kernel, "us": att_med, "algorithmic_bytes": att_b,
-                     "achieved_GBps": att_b / att_med / 1e3,
-                     "traffic": tr_a},
+            "step": {"kernel": "decode_step_kernel", "us": us, "algorithmic_bytes": sel_b + att_b,
+                     "achieved_GBps": (sel_b + att_b) / us / 1e3, "traffic": tr_f},
         },
-        "gpu_launches_per_step": 2 if ws_a.numel() == 0 else 3,
+        "gpu_launches_per_step": 1,
+        "separate_calls": {
+            "note": "infllmv2_select_blocks(DECODE) then infllmv2_sparse_attn_decode on the same inputs",
+            "pair_us": statistics.median(pair_us),
+            "select": {"kernel": "select_decode_kernel", "us": sel_med, "algorithmic_bytes": sel_b,
+                       "achieved_GBps": sel_b / sel_med / 1e3, "traffic": tr_s},
+            "attn": {"kernel": att_kernel, "us": att_med, "algorithmic_bytes": att_b,
+                     "achieved_GBps": att_b / att_med / 1e3, "traffic": tr_a},
+        },
         "append": {"kernel": "append_kv_kernel", "us": app_us, "bytes_per_step": app_bytes,
                    "note": "cache maintenance of a decode step (new K/V rows, completed kernels), timed apart"},
     }

@@ -194,3 +194,31 @@ def test_backward_rejects_bad_arguments_before_launch(lib):
     bad = list(args)
     bad[7] = 0
     assert f(cp(), *bad, good, need, None) == _lib.ERR_INVALID_ARG
+
+
+def test_decode_step_rejects_bad_arguments_before_launch(lib):
+    good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    f = lib.infllmv2_decode_step
+    # q, k_cache, v_cache, kc, lens, Lmax, block_idx, o, lse
+    args = [good, good, good, good, good, 1024, good, good, None]
+    for i in (0, 1, 2, 4, 6, 7):  # required pointers
+        bad = list(args)
+        bad[i] = None
+        assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG, i
+    for i in (0, 1, 2, 3, 6, 7):  # 16-byte aligned
+        bad = list(args)
+        bad[i] = good + 8
+        assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG, i
+    bad = list(args)
+    bad[4] = good + 2  # lens 4-byte aligned
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(args)
+    bad[8] = good + 1  # lse 4-byte aligned
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(args)
+    bad[3] = None  # kc is needed once a semantic kernel exists
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(args)
+    bad[5] = 0
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    assert f(cp(head_dim=64), *args, None) == _lib.ERR_UNSUPPORTED

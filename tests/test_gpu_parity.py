@@ -283,6 +283,12 @@ def test_decode_at_the_maximum_length():
     o_g, lse_g = ops.sparse_attn_decode(p, q, k, v, ln, torch.from_numpy(idx_o).cuda())
     o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
     compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
+    # the fused step at the same lengths: the separate selection's lists, the exact
+    # attention over them
+    o_f, lse_f, idx_f = ops.decode_step(p, q, k, v, kc_t, ln)
+    assert np.array_equal(idx_f.cpu().numpy(), idx_g)
+    o_o2, lse_o2 = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_g, lens=lens_np)
+    compare_attention(o_f.float().cpu().numpy(), o_o2[:, 0], lse_f.cpu().numpy(), lse_o2[:, :, 0])
 
 
 def test_attn_decode_many_items_per_cta_is_deterministic():
@@ -339,6 +345,97 @@ def test_attn_decode_ignores_garbage_past_the_length():
     o_o, _ = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_o, lens=lens_np)
     assert torch.isfinite(o_g).all()
     compare_attention(o_g.float().cpu().numpy(), o_o[:, 0])
+
+
+# ------------------------------------------------------------- fused decode step
+
+def run_decode_step_case(lens, Lmax, Hq, Hkv, topk, seed, score_mode=0, pool_mode=0, nan_tail=False):
+    """The fused decode step (selection and attention in one launch) on the oracle's
+    kernels: its block lists are the separate selection's, bit for bit, and checked
+    against the oracle's; its outputs against the exact attention over those lists and
+    against the separate attention call.  With nan_tail the cache rows at or past lens[b]
+    hold NaN, which must not reach the outputs."""
+    B = len(lens)
+    x = inputs(B, Lmax, Hq, Hkv, seed=seed, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk, score_mode=score_mode, pool_mode=pool_mode)
+    op = oparams(p)
+    lens_np = np.array(lens, np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k), lens=lens_np)
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    k, v = x.k.clone(), x.v.clone()
+    if nan_tail:
+        for b, n in enumerate(lens):
+            k[b, :, n:] = float("nan")
+            v[b, :, n:] = float("nan")
+    q, kd, vd, ln = x.q.cuda(), k.cuda(), v.cuda(), x.lens.cuda()
+    o_g, lse_g, idx_g = ops.decode_step(p, q, kd, vd, kc_t, ln)
+    idx_s = ops.select_blocks_decode(p, q, kc_t, ln, Lmax)
+    o_s, lse_s = ops.sparse_attn_decode(p, q, kd, vd, ln, idx_s)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_g, idx_s)
+    assert torch.isfinite(o_g).all()
+    idx_gn = idx_g.cpu().numpy()
+    idx_o, sc = oracle.select(op, as_u16(x.q)[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    _, n_tie = compare_selection(idx_gn, idx_o, sc, (lens_np - 1)[:, None], p)
+    o_o, lse_o = oracle.attn(op, as_u16(x.q)[:, None], as_u16(x.k), as_u16(x.v), idx_gn, lens=lens_np)
+    compare_attention(o_g.float().cpu().numpy(), o_o[:, 0], lse_g.cpu().numpy(), lse_o[:, :, 0])
+    # the separate attention may split the list over CTAs differently: last bits only
+    assert (o_g.float() - o_s.float()).abs().max().item() <= 1e-2
+    assert (lse_g - lse_s).abs().max().item() <= 1e-4
+    return n_tie
+
+
+@pytest.mark.parametrize("lens,Lmax,Hq,Hkv,topk", [([3000, 1, 31, 1500, 2049], 3000, 32, 2, 16),
+                                                  ([70, 64, 65, 128], 128, 8, 1, 3),
+                                                  ([9000, 8193, 64], 9000, 16, 1, 96),
+                                                  ([9000, 8193], 9000, 4, 4, 100),
+                                                  ([20000, 4097, 12345, 600, 19999, 33], 20000, 32, 2, 96)])
+def test_decode_step_matches_oracle(lens, Lmax, Hq, Hkv, topk):
+    # 3 to 12 items: clusters of 16 CTAs
+    run_decode_step_case(lens, Lmax, Hq, Hkv, topk, seed=900 + Lmax)
+
+
+@pytest.mark.parametrize("B", [40, 80])
+def test_decode_step_small_clusters(B):
+    # 80 and 160 (sequence, kv-head) items: clusters of 2 CTAs and of 1
+    lens = np.random.default_rng(B).integers(1, 4001, size=B).tolist()
+    run_decode_step_case(lens, 4000, 32, 2, 16, seed=980 + B)
+
+
+@pytest.mark.parametrize("score_mode,pool_mode", VARIANTS)
+def test_decode_step_variants_match_oracle(score_mode, pool_mode):
+    run_decode_step_case([5000, 4999, 64, 1000], 5000, 32, 2, 24, seed=950, score_mode=score_mode,
+                         pool_mode=pool_mode)
+
+
+def test_decode_step_ignores_garbage_past_the_length():
+    run_decode_step_case([100, 64, 65, 3001], 3072, 16, 1, 8, seed=960, nan_tail=True)
+
+
+def test_decode_step_empty_sequence_and_determinism():
+    # lens[b] = 0: no query, the list is all -1, o is 0 and lse is -inf; the other rows
+    # are unaffected, and repeated steps agree bit for bit
+    lens, Lmax, Hq, Hkv, topk = [0, 3000, 5, 2500], 3000, 32, 2, 16
+    B = len(lens)
+    x = inputs(B, Lmax, Hq, Hkv, seed=970, mode="decode", lens=lens)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    q, k, v, ln = x.q.cuda(), x.k.cuda(), x.v.cuda(), x.lens.cuda()
+    kc = ops.compress_keys(p, k, lens=ln)
+    o_ref, lse_ref, idx_ref = ops.decode_step(p, q, k, v, kc, ln)
+    assert torch.all(idx_ref[0] == -1)
+    assert torch.all(o_ref[0] == 0) and torch.all(torch.isneginf(lse_ref[0]))
+    for _ in range(3):
+        o_g, lse_g, idx_g = ops.decode_step(p, q, k, v, kc, ln)
+        assert torch.equal(idx_g, idx_ref) and torch.equal(o_g, o_ref) and torch.equal(lse_g, lse_ref)
+    # rows 1..3 against the oracle
+    op = oparams(ops.Params(B - 1, Hq, Hkv, topk=topk))
+    lens_np = np.array(lens[1:], np.int32)
+    kc_o = oracle.compress(op, as_u16(x.k[1:]), lens=lens_np)
+    idx_o, sc = oracle.select(op, as_u16(x.q[1:])[:, None], kc_o, lens=lens_np, Lmax=Lmax, want_scores=True)
+    idx_gn = idx_ref[1:].cpu().numpy()
+    compare_selection(idx_gn, idx_o, sc, (lens_np - 1)[:, None], ops.Params(B - 1, Hq, Hkv, topk=topk))
+    o_o, lse_o = oracle.attn(op, as_u16(x.q[1:])[:, None], as_u16(x.k[1:]), as_u16(x.v[1:]), idx_gn, lens=lens_np)
+    compare_attention(o_ref[1:].float().cpu().numpy(), o_o[:, 0], lse_ref[1:].cpu().numpy(), lse_o[:, :, 0])
 
 
 # ---------------------------------------------------------- whole path, workloads

@@ -1,4 +1,7 @@
-// attn.cuh -- exact attention over the selected KV blocks (prefill and decode).
+// attn.cuh -- exact attention over the selected KV blocks on m16n8k16 tensor-core
+// MMAs: the split decode path (few sequences), and the work-item mapping, parameters
+// and per-block update shared with the other attention kernels.  Prefill and prefill
+// chunks run on attn_tc_kernel (attn_tc.cuh) for every group size.
 //
 // MiniCPM4 summary page (端设备上的超高效大型语言模型) s2.1.3: each token attends only to
 // its most relevant KV blocks; s2.1.2: the query heads of one group share those blocks,

@@ -43,64 +43,30 @@ constexpr size_t attn_dec_smem_bytes() {
   return 1024 + static_cast<size_t>(kAdStages) * kAttnStageBytes + kQTileBytes + sizeof(AdSmem);
 }
 
-// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.  C divides 16.
-__global__ void __launch_bounds__(kAdThreads)
-    attn_decode_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* ring = align_smem(smem_raw, 1024);
-  unsigned char* qtile = ring + kAdStages * kAttnStageBytes;
-  AdSmem& S = *reinterpret_cast<AdSmem*>(qtile + kQTileBytes);
-  float* part = reinterpret_cast<float*>(ring);      // [4 warps][16][kMergeRowFloats], once the ring drained
-  float* comb = part + kAttnConsumers * kAdWarpRows;  // [16][kMergeRowFloats]: this CTA's state
+// Barrier set-up of the attention ring (thread 0; the caller's next CTA barrier publishes it).
+__device__ __forceinline__ void ad_init(AdSmem& S) {
+  for (int s = 0; s < kAdStages; ++s) {
+    mbar_init(&S.full[s], 1);
+    mbar_init(&S.empty[s], kAttnConsumers);
+  }
+  mbar_init(&S.qbar, 1);
+  S.abort = 0;
+  fence_mbar_init();
+}
 
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int crank = static_cast<int>(cluster.block_rank());
-  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
-  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int qrow = b * p.Hq + g * p.G;
+// This CTA's share of an item, all threads: the group's query tile and the n blocks
+// blocks[0 .. n) (shared memory) streamed through the ring, the four consumer warps'
+// online softmax, then their states combined in the drained ring into this CTA's state
+// (S.cm, S.cl and the unnormalised rows in ad_comb(ring)).  Ends after a CTA barrier.
+__device__ __forceinline__ float* ad_comb(unsigned char* ring) {
+  return reinterpret_cast<float*>(ring) + kAttnConsumers * kAdWarpRows;
+}
+__device__ __forceinline__ void ad_partial(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                           const AttnParams& p, long long bg, int qrow, int t, const int* blocks,
+                                           int n, unsigned char* ring, unsigned char* qtile, AdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // prologue that reads no input: it overlaps the end of the selection kernel
-  allow_dependent_launch();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kAdStages; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kAttnConsumers);
-    }
-    mbar_init(&S.qbar, 1);
-    S.abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == kAttnConsumers && lane == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-  }
-  grid_dependency_wait();  // block_idx (and q, the caches, lens) are complete from here on
-  const int t = min(p.lens[b], p.Lmax) - 1;  // < 0: empty sequence
-  const int cur = t >= 0 ? t / kBlock : -1;
-  if (warp == kAttnConsumers) {  // compact the item's valid block indices, in list order
-    const int32_t* row = p.idx + bg * static_cast<long long>(p.topk);
-    int count = 0;
-    for (int e0 = 0; e0 < p.topk; e0 += 32) {
-      const int e = e0 + lane;
-      const int j = e < p.topk ? row[e] : -1;
-      const bool ok = j >= 0 && j <= cur;
-      const unsigned msk = __ballot_sync(0xffffffffu, ok);
-      if (ok) S.list[count + __popc(msk & ((1u << lane) - 1u))] = j;
-      count += __popc(msk);
-    }
-    if (lane == 0) S.n_blocks = count;
-  }
-  __syncthreads();
-  const int n_all = S.n_blocks;
-  const int per = (n_all + C - 1) / C;
-  const int lo = min(crank * per, n_all);
-  const int n = min(lo + per, n_all) - lo;
-
+  float* part = reinterpret_cast<float*>(ring);  // [4 warps][16][kMergeRowFloats], once the ring drained
+  float* comb = ad_comb(ring);                   // [16][kMergeRowFloats]: this CTA's state
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float o[16][4];
 #pragma unroll
@@ -109,20 +75,20 @@ __global__ void __launch_bounds__(kAdThreads)
     // ------------------------------------------------------------ producer
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(&S.qbar, kQTileBytes);
-      tma_load_2d(qtile, &tm_q, &S.qbar, 0, qrow);
-      tma_load_2d(qtile + kQTileBytes / 2, &tm_q, &S.qbar, 64, qrow);
+      tma_load_2d(qtile, tm_q, &S.qbar, 0, qrow);
+      tma_load_2d(qtile + kQTileBytes / 2, tm_q, &S.qbar, 64, qrow);
       const long long kvrow0 = bg * p.Lmax;
       int i = 0;
       for (; i < n; ++i) {
         const int st = i % kAdStages, u = i / kAdStages;
         if (u > 0 && !mbar_wait(&S.empty[st], (u - 1) & 1, &S.abort)) break;
-        const int krow = static_cast<int>(kvrow0 + static_cast<long long>(S.list[lo + i]) * kBlock);
+        const int krow = static_cast<int>(kvrow0 + static_cast<long long>(blocks[i]) * kBlock);
         unsigned char* sk = ring + st * kAttnStageBytes;
         mbar_arrive_expect_tx(&S.full[st], kAttnStageBytes);
-        tma_load_2d(sk, &tm_k, &S.full[st], 0, krow);
-        tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.full[st], 64, krow);
-        tma_load_2d(sk + kKvTileBytes, &tm_v, &S.full[st], 0, krow);
-        tma_load_2d(sk + kKvTileBytes + kKvTileBytes / 2, &tm_v, &S.full[st], 64, krow);
+        tma_load_2d(sk, tm_k, &S.full[st], 0, krow);
+        tma_load_2d(sk + kKvTileBytes / 2, tm_k, &S.full[st], 64, krow);
+        tma_load_2d(sk + kKvTileBytes, tm_v, &S.full[st], 0, krow);
+        tma_load_2d(sk + kKvTileBytes + kKvTileBytes / 2, tm_v, &S.full[st], 64, krow);
       }
       mbar_wait_drain(&S.qbar, 0);
       if (S.abort) {  // let every issued copy land before the ring is reused
@@ -145,8 +111,8 @@ __global__ void __launch_bounds__(kAdThreads)
       for (int i = 0; i < n; ++i) {
         const int st = i % kAdStages;
         if (!mbar_wait(&S.full[st], (i / kAdStages) & 1, &S.abort)) break;
-        attn_block_update(ring + st * kAttnStageBytes, S.list[lo + i], t, 16 * warp, qa, p.scale_log2, m0, m1, l0,
-                          l1, o);
+        attn_block_update(ring + st * kAttnStageBytes, blocks[i], t, 16 * warp, qa, p.scale_log2, m0, m1, l0, l1,
+                          o);
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[st]);
       }
@@ -203,26 +169,51 @@ __global__ void __launch_bounds__(kAdThreads)
       }
     }
   }
-  cluster.sync();  // every CTA's state is final
+  __syncthreads();
+}
 
-  // CTA crank merges head rows [crank h_per, (crank + 1) h_per) across the cluster
+// Cluster merge, all threads of every CTA (it contains two cluster barriers): CTA crank
+// merges head rows [crank 16 / C, (crank + 1) 16 / C) of the C CTAs' states, read through
+// distributed shared memory (a warp per row: lane r reads CTA r's max and sum, the
+// C partial rows are all in flight before they are summed), and writes O and the lse.
+__device__ __forceinline__ void ad_merge(cooperative_groups::cluster_group& cluster, const AttnParams& p, int qrow,
+                                         unsigned char* ring, AdSmem& S) {
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* comb = ad_comb(ring);
+  cluster.sync();  // every CTA's state is final
   const int h_per = kGroupRows / C;
   for (int hh = warp; hh < h_per; hh += kAdThreads / 32) {
     const int h = crank * h_per + hh;
-    float M = -INFINITY;
-    for (int r = 0; r < C; ++r) M = fmaxf(M, cluster.map_shared_rank(&S.cm[0], r)[h]);
-    float L = 0.f;
+    const float cmr = lane < C ? cluster.map_shared_rank(&S.cm[0], lane)[h] : -INFINITY;
+    const float clr = lane < C ? cluster.map_shared_rank(&S.cl[0], lane)[h] : 0.f;
+    float M = cmr;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wt = (M != -INFINITY && lane < C) ? ex2(cmr - M) : 0.f;
+    float L = wt * clr;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-      for (int r = 0; r < C; ++r) {
-        const float wt = ex2(cluster.map_shared_rank(&S.cm[0], r)[h] - M);
-        L += wt * cluster.map_shared_rank(&S.cl[0], r)[h];
-        const float4 v =
-            *reinterpret_cast<const float4*>(cluster.map_shared_rank(comb, r) + h * kMergeRowFloats + 4 * lane);
-        acc.x += wt * v.x;
-        acc.y += wt * v.y;
-        acc.z += wt * v.z;
-        acc.w += wt * v.w;
+#pragma unroll
+    for (int r0 = 0; r0 < kAdMaxCluster; r0 += 8) {
+      float4 v[8];
+      float w8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u;
+        w8[u] = __shfl_sync(0xffffffffu, wt, r);
+        v[u] = r < C ? *reinterpret_cast<const float4*>(cluster.map_shared_rank(comb, r) + h * kMergeRowFloats +
+                                                        4 * lane)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x += w8[u] * v[u].x;
+        acc.y += w8[u] * v[u].y;
+        acc.z += w8[u] * v[u].z;
+        acc.w += w8[u] * v[u].w;
       }
     }
     if (h < p.G) {
@@ -236,6 +227,57 @@ __global__ void __launch_bounds__(kAdThreads)
     }
   }
   cluster.sync();  // peers' shared memory stays valid until every CTA has read it
+}
+
+// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.  C divides 16.
+__global__ void __launch_bounds__(kAdThreads)
+    attn_decode_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* ring = align_smem(smem_raw, 1024);
+  unsigned char* qtile = ring + kAdStages * kAttnStageBytes;
+  AdSmem& S = *reinterpret_cast<AdSmem*>(qtile + kQTileBytes);
+
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int crank = static_cast<int>(cluster.block_rank());
+  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
+  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+  const int qrow = b * p.Hq + g * p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // prologue that reads no input: it overlaps the end of the selection kernel
+  allow_dependent_launch();
+  if (threadIdx.x == 0) ad_init(S);
+  if (warp == kAttnConsumers && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  grid_dependency_wait();  // block_idx (and q, the caches, lens) are complete from here on
+  const int t = min(p.lens[b], p.Lmax) - 1;  // < 0: empty sequence
+  const int cur = t >= 0 ? t / kBlock : -1;
+  if (warp == kAttnConsumers) {  // compact the item's valid block indices, in list order
+    const int32_t* row = p.idx + bg * static_cast<long long>(p.topk);
+    int count = 0;
+    for (int e0 = 0; e0 < p.topk; e0 += 32) {
+      const int e = e0 + lane;
+      const int j = e < p.topk ? row[e] : -1;
+      const bool ok = j >= 0 && j <= cur;
+      const unsigned msk = __ballot_sync(0xffffffffu, ok);
+      if (ok) S.list[count + __popc(msk & ((1u << lane) - 1u))] = j;
+      count += __popc(msk);
+    }
+    if (lane == 0) S.n_blocks = count;
+  }
+  __syncthreads();
+  const int n_all = S.n_blocks;
+  const int per = (n_all + C - 1) / C;
+  const int lo = min(crank * per, n_all);
+  const int n = min(lo + per, n_all) - lo;
+  ad_partial(&tm_q, &tm_k, &tm_v, p, bg, qrow, t, S.list + lo, n, ring, qtile, S);
+  ad_merge(cluster, p, qrow, ring, S);
 }
 
 }  // namespace infllmv2

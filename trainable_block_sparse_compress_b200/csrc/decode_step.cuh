@@ -1,0 +1,106 @@
+// decode_step.cuh -- a whole decode step (block selection, then sparse attention over
+// the selected blocks) for one query per sequence, in one launch.
+//
+// MiniCPM4 summary page (端设备上的超高效大型语言模型) s2.1: InfLLM v2 selects context
+// blocks for decoding as well as prefill; s2.1.2 / s2.1.3: the group's heads share the
+// selected blocks and attend only to them.
+//
+// A thread-block cluster per (sequence, kv-head) runs the selection phases of
+// select_decode.cuh (Kc streamed and scored by every CTA, keys gathered in CTA 0, CTA 0's
+// top-k into its shared memory and block_idx), then, after one more cluster barrier, the
+// attention phases of attn_dec.cuh over that list (each CTA copies its contiguous share of
+// the list from CTA 0 through distributed shared memory, streams those K/V blocks and the
+// partial states are merged across the cluster).  Clusters do not wait for one another,
+// so a cluster whose sequence is short streams its K/V while longer sequences are still
+// being scored, and nothing round-trips through global memory between the two halves.
+// The selection's tile ring and block maxima and the attention's ring share one region of
+// shared memory: each half's data is dead before the other half writes it.
+#pragma once
+#include <cooperative_groups.h>
+
+#include "attn_dec.cuh"
+#include "select_decode.cuh"
+
+namespace infllmv2 {
+
+constexpr size_t kDsAttnRegion = static_cast<size_t>(kAdStages) * kAttnStageBytes + kQTileBytes;
+constexpr size_t kDsRegion = kSdRegionBytes > kDsAttnRegion ? kSdRegionBytes : kDsAttnRegion;
+
+struct DsSmem {
+  SdSmem sel;
+  AdSmem attn;          // attn.list: the item's list as CTA 0 emits it
+  int share[kMaxTopk];  // this CTA's blocks of that list
+};
+
+constexpr size_t decode_step_smem_bytes() { return 1024 + kDsRegion + sizeof(DsSmem); }
+
+struct DecodeStepParams {
+  SelDecodeParams sel;
+  AttnParams attn;
+};
+
+// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.  C divides 16.
+__global__ void __launch_bounds__(kSdThreads)
+    decode_step_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const DecodeStepParams P) {
+  static_assert(kSdThreads == kAdThreads, "one block shape for both halves");
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* region = align_smem(smem_raw, 1024);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(region + kSdStages * kKcTileBytes);  // selection: [16][kSdBStride]
+  unsigned char* qtile = region + kAdStages * kAttnStageBytes;                      // attention: the query tile
+  DsSmem& D = *reinterpret_cast<DsSmem*>(region + kDsRegion);
+
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int c = static_cast<int>(cluster.block_rank());
+  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int topk = P.sel.topk;
+
+  allow_dependent_launch();
+  if (threadIdx.x == 0) ad_init(D.attn);  // published by the first CTA barrier of the selection
+  if (warp == kSdConsumers && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  grid_dependency_wait();  // q, the caches, Kc and lens may come from the previous kernel
+  const SdItem it = sd_item(P.sel, C, c, bg);
+
+  // ---- selection
+  sd_score_chunk(&tm_kc, P.sel, it, region, bm, D.sel);
+  cluster.sync();  // every CTA's tiles are consumed and its partial state is final
+  sd_block_keys(cluster, P.sel, it, reinterpret_cast<uint32_t*>(region + kSdKeysOff), bm, D.sel);
+  cluster.sync();  // CTA 0 holds every key
+  if (c == 0) {
+    sd_select(P.sel, it, region, D.attn.list, D.sel);
+    int32_t* out = P.sel.idx + bg * topk;
+    for (int e = threadIdx.x; e < topk; e += kSdThreads) out[e] = D.attn.list[e];
+    if (warp == 0) {  // the list is ascending and -1 padded: count its blocks
+      int count = 0;
+      for (int e0 = 0; e0 < topk; e0 += 32) {
+        const int e = e0 + lane;
+        count += __popc(__ballot_sync(0xffffffffu, e < topk && D.attn.list[e] >= 0));
+      }
+      if (lane == 0) D.attn.n_blocks = count;
+    }
+  }
+  cluster.sync();  // CTA 0's list is complete; no CTA reads a selection array after this
+
+  // ---- attention over this CTA's contiguous share of the list
+  const int n_all = *cluster.map_shared_rank(&D.attn.n_blocks, 0);
+  const int per = (n_all + C - 1) / C;
+  const int lo = min(c * per, n_all);
+  const int n = min(lo + per, n_all) - lo;
+  const int* list0 = cluster.map_shared_rank(D.attn.list, 0);
+  for (int i = threadIdx.x; i < n; i += kSdThreads) D.share[i] = list0[lo + i];
+  fence_proxy_async_smem();  // the region's generic accesses before the ring's copies
+  __syncthreads();
+  const int qrow = it.b * P.attn.Hq + it.g * P.attn.G;
+  ad_partial(&tm_q, &tm_k, &tm_v, P.attn, bg, qrow, it.n - 1, D.share, n, region, qtile, D.attn);
+  ad_merge(cluster, P.attn, qrow, region, D.attn);
+}
+
+}  // namespace infllmv2

@@ -21,6 +21,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "decode_step.cuh"
 #include "select_decode.cuh"
 #include "select_prefill.cuh"
 #include "select_prefill_tc.cuh"
@@ -213,6 +214,52 @@ int select_cluster(const infllmv2_params* p, int64_t nk) {
   return c;
 }
 
+// Clusters of C CTAs of `kern` that the device holds at once (cached per kernel, size,
+// shared memory and device).
+template <typename... Params>
+int max_active_clusters(void (*kern)(Params...), int C, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
+  const void* fn = reinterpret_cast<const void*>(kern);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(fn, C, smem, dev);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  if (set_smem(fn, smem) != INFLLMV2_OK) return 0;
+  if (C > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(C));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess) active = 0;
+  cache.emplace(key, active);
+  return active;
+}
+
+// Decode-step cluster size: enough CTAs for the longest sequence's kernels (at most
+// kSdMaxChunk per CTA), then doubled while all CTAs stay at two per SM and every item's
+// cluster is resident at once (a cluster left for a second wave costs a whole step).
+int decode_step_cluster(const infllmv2_params* p, int64_t nk) {
+  const long long items = static_cast<long long>(p->batch) * p->num_kv_heads;
+  const long long target = 2LL * num_sms();
+  int c = 1;
+  while (c < kSdMaxCluster && static_cast<int64_t>(c) * kSdMaxChunk < nk) c *= 2;
+  while (c < kSdMaxCluster && items * c * 2 <= target &&
+         items <= max_active_clusters(decode_step_kernel, 2 * c, kSdThreads, decode_step_smem_bytes()))
+    c *= 2;
+  return c;
+}
+
 // Workspace of the backward pass, in order (each part 256-byte aligned): D [B, Hq, L]
 // fp32; cnt, cursor, off [n] and segoff [n + 1] int32 (n = B * Hkv * blocks); the row
 // lists [B * Hkv * L * topk] int32; dK and dV accumulators [B, Hkv, L, d] fp32.
@@ -368,8 +415,11 @@ int attn_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const void
   a.lse = lse;
   a.part_o = nullptr;
   a.part_lse = nullptr;
-  if (a.G == kGroupRows) {
-    // tensor-core path: per item, K/V block pairs against the group's 16 query rows
+  {
+    // tensor-core path: per item, K/V block pairs against 16 query rows from the group's
+    // first head (for G < 16 the rows past the group are other heads' queries: their
+    // columns of S, P and O are computed and never written; rows past the end of q are
+    // zero-filled by the copy)
     CUtensorMap tq, tk, tv;
     if (!make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k, kv_rows, kBlock) ||
         !make_map(&tv, v, kv_rows, kBlock))
@@ -378,10 +428,10 @@ int attn_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const void
     int st = set_smem(reinterpret_cast<const void*>(attn_tc_kernel), smem);
     if (st != INFLLMV2_OK) return st;
     const long long grid = std::min<long long>(a.num_items, num_sms());
+    if (grid <= 0) return INFLLMV2_OK;
     attn_tc_kernel<<<static_cast<unsigned>(grid), kAtThreads, smem, s>>>(tq, tk, tv, a);
     return launch_status();
   }
-  return launch_attn(p, q, q_rows, k, v, kv_rows, a, s);
 }
 
 int launch_attn(const infllmv2_params* p, const void* q, uint64_t q_rows, const void* k, const void* v,
@@ -692,6 +742,77 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
   attn_merge_kernel<<<static_cast<unsigned>(static_cast<long long>(p->batch) * p->num_kv_heads * a.G), 128, 0, s>>>(
       a.part_o, a.part_lse, d.n_splits, p->num_q_heads, p->num_kv_heads, a.G, static_cast<__nv_bfloat16*>(o), lse);
   return launch_status();
+}
+
+int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,
+                         const void* kc, const int32_t* lens, int32_t Lmax, int32_t* block_idx, void* o, float* lse,
+                         infllmv2_stream_t stream) {
+  int st = check_params(p);
+  if (st != INFLLMV2_OK) return st;
+  if ((st = check_len(Lmax)) != INFLLMV2_OK) return st;
+  if (!q || !k_cache || !v_cache || !lens || !block_idx || !o) return INFLLMV2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(block_idx) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lens) & 3u))
+    return INFLLMV2_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
+  const int64_t nk = num_kernels(Lmax);
+  if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
+  const uint64_t kv_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * Lmax;
+  if (kv_rows > 0x7fffffffULL ||
+      static_cast<uint64_t>(p->batch) * p->num_kv_heads * static_cast<uint64_t>(nk) > 0x7fffffffULL)
+    return INFLLMV2_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  const int G = p->num_q_heads / p->num_kv_heads;
+  DecodeStepParams P;
+  SelDecodeParams& a = P.sel;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.lens = lens;
+  a.idx = block_idx;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = G;
+  a.Lmax = Lmax;
+  a.NKmax = static_cast<int>(nk);
+  a.topk = p->topk;
+  a.n_init = p->n_init;
+  a.n_local = p->n_local;
+  a.score_mode = p->score_mode;
+  a.pool_mode = p->pool_mode;
+  a.scale_log2 = scale_log2(p);
+  AttnParams& t = P.attn;
+  t.idx = block_idx;
+  t.lens = lens;
+  t.q_lens = nullptr;
+  t.kv_lens = nullptr;
+  t.B = p->batch;
+  t.Hq = p->num_q_heads;
+  t.Hkv = p->num_kv_heads;
+  t.G = G;
+  t.Lq = 1;
+  t.Lmax = Lmax;
+  t.topk = p->topk;
+  t.n_splits = 1;
+  t.blocks_per_split = p->topk;
+  t.scale_log2 = a.scale_log2;
+  t.num_items = static_cast<long long>(p->batch) * p->num_kv_heads;
+  t.o = static_cast<__nv_bfloat16*>(o);
+  t.lse = lse;
+  t.part_o = nullptr;
+  t.part_lse = nullptr;
+  CUtensorMap tm_kc, tq, tk, tv;
+  std::memset(&tm_kc, 0, sizeof tm_kc);
+  const uint64_t q_rows = static_cast<uint64_t>(p->batch) * p->num_q_heads;
+  // with no complete kernel a map over a dummy extent is never dereferenced
+  if (!(nk > 0 ? make_map(&tm_kc, kc, static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk, kKcTile)
+               : make_map(&tm_kc, q, kKcTile, kKcTile)) ||
+      !make_map(&tq, q, q_rows, kGroupRows) || !make_map(&tk, k_cache, kv_rows, kBlock) ||
+      !make_map(&tv, v_cache, kv_rows, kBlock))
+    return INFLLMV2_ERR_CUDA;
+  const int C = decode_step_cluster(p, nk);
+  const long long grid = static_cast<long long>(C) * p->batch * p->num_kv_heads;
+  if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+  return launch_cluster(decode_step_kernel, static_cast<unsigned>(grid), C, kSdThreads, decode_step_smem_bytes(),
+                        reinterpret_cast<cudaStream_t>(stream), true, tm_kc, tq, tk, tv, P);
 }
 
 }  // extern "C"

@@ -15,10 +15,13 @@
 //      shared memory, all loads in parallel), computes S(j) = sum_h exp(m_h(j) - lse_h)
 //      (or, with logit-sum scoring, sum_h m_h(j)) for its blocks and stores the keys into
 //      CTA 0 (with inside pooling block j pools kernels 4j .. 4j+2 only, and no carry);
-//   3. CTA 0 finds the k-th largest key by a 32-way radix search (lane l of every warp
-//      counts the keys at or above candidate digit l; once the digit's bucket holds at
-//      most 32 keys they are ranked directly) and all its threads write the ascending
-//      list (prefix sums place ties and outputs).
+//   3. CTA 0 finds the k-th largest key: the candidates' common leading bits come from
+//      one AND / OR reduction, the bits below them from shared-memory histograms of
+//      11-bit digits (a suffix scan picks the digit that holds the k-th key; once its
+//      bucket holds at most 32 keys they are ranked directly), and all its threads
+//      write the ascending list (prefix sums place ties and outputs).
+// The phases are device functions: select_decode_kernel runs them alone, the fused decode
+// step (decode_step.cuh) runs them before the attention in the same cluster.
 // No workspace, one launch; reading Kc once bounds it (HBM).
 #pragma once
 #include <cooperative_groups.h>
@@ -38,9 +41,18 @@ constexpr int kSdMaxQuads = kSdMaxChunk / 4;
 constexpr int kSdBStride = kSdMaxQuads + 4;  // per-head block-max rows (quads + 1 carry), padded
 constexpr int kSdMaxCluster = 16;
 // CTA 0's top-k visits the keys slot-major: thread i takes keys i + kSdThreads s.
-constexpr int kSdMaxR = (INFLLMV2_MAX_SEQ_LEN / kBlock + kSdThreads - 1) / kSdThreads;
-static_assert(kSdStages * kKcTileBytes >= 4 * (INFLLMV2_MAX_SEQ_LEN / kBlock),
-              "the block keys of CTA 0 reuse its tile ring");
+constexpr int kSdMaxKeys = INFLLMV2_MAX_SEQ_LEN / kBlock;
+constexpr int kSdMaxR = (kSdMaxKeys + kSdThreads - 1) / kSdThreads;
+constexpr int kSdHistBits = 11;  // digit width of the threshold search
+constexpr int kSdHistBins = 1 << kSdHistBits;
+constexpr int kSdBinsPerThread = (kSdHistBins + kSdThreads - 1) / kSdThreads;
+// CTA 0's selection scratch, in its drained tile ring: block keys, the digit histogram
+// and the take flags of a tie-ranked emission
+constexpr int kSdKeysOff = 0;
+constexpr int kSdHistOff = kSdKeysOff + 4 * kSdMaxKeys;
+constexpr int kSdFlagOff = kSdHistOff + 4 * kSdHistBins;
+constexpr int kSdScratchBytes = kSdFlagOff + kSdMaxR * kSdThreads;
+static_assert(kSdStages * kKcTileBytes >= kSdScratchBytes, "the selection scratch of CTA 0 reuses its tile ring");
 static_assert(kSdMaxCluster * kSdMaxChunk >= (INFLLMV2_MAX_SEQ_LEN - kKernel) / kStride + 1,
               "a cluster covers the longest sequence");
 
@@ -60,72 +72,62 @@ struct SdSmem {
   float pm[kSdMaxCluster][kGroupRows], pl[kSdMaxCluster][kGroupRows];  // every CTA's, gathered
   float lse2[kGroupRows];  // log2-sum-exp2 per head over the whole sequence
   float carry[kGroupRows];  // previous CTA's last kernel, for this CTA's first block
-  int cnt[2][kSdWarps][32];
+  int wred[3][kSdWarps];               // per-warp candidates, AND, OR of the keys
+  int wsum[kSdWarps];                  // per-warp histogram totals of the digit search
+  int dig, dig_above, dig_in;          // the digit found, keys above its bin, keys in it
   int wc[kSdMaxR][kSdWarps];          // per (slot, warp) counts of the emission
   int sbase[kSdMaxR];                 // flagged keys in earlier slots
   int total;
-  unsigned char tflag[kSdMaxR][kSdThreads];  // take flags when tie ranks are needed
   int nlist;
   uint32_t list[32];
   volatile int abort;
 };
 
-constexpr size_t sel_decode_smem_bytes() {
-  return 1024 + static_cast<size_t>(kSdStages) * kKcTileBytes + static_cast<size_t>(kGroupRows) * kSdBStride * 4 +
-         sizeof(SdSmem);
+// Tile ring (reused by CTA 0 as the selection scratch) and per-head block maxima.
+constexpr size_t kSdRegionBytes =
+    static_cast<size_t>(kSdStages) * kKcTileBytes + static_cast<size_t>(kGroupRows) * kSdBStride * 4;
+
+constexpr size_t sel_decode_smem_bytes() { return 1024 + kSdRegionBytes + sizeof(SdSmem); }
+
+// One (sequence, kv-head) item of a decode-selection cluster and this CTA's share of it.
+struct SdItem {
+  int C, c;  // cluster size and rank
+  long long bg;
+  int b, g;
+  int n, nk, cur;  // sequence length (clamped), complete kernels, current block (-1: empty)
+  int chunk, nq;   // kernels and blocks per CTA
+  int k0, ntiles;  // this CTA's first kernel and Kc tiles
+};
+
+// Reads lens: call after grid_dependency_wait().
+__device__ __forceinline__ SdItem sd_item(const SelDecodeParams& p, int C, int c, long long bg) {
+  SdItem it;
+  it.C = C;
+  it.c = c;
+  it.bg = bg;
+  it.b = static_cast<int>(bg / p.Hkv);
+  it.g = static_cast<int>(bg % p.Hkv);
+  it.n = min(max(p.lens[it.b], 0), p.Lmax);
+  it.nk = it.n >= kKernel ? (it.n - kKernel) / kStride + 1 : 0;
+  it.cur = it.n > 0 ? (it.n - 1) / kBlock : -1;
+  it.chunk = ((it.nk + C - 1) / C + kKcTile - 1) / kKcTile * kKcTile;
+  it.nq = it.chunk / 4;
+  it.k0 = c * it.chunk;
+  it.ntiles = it.nk > it.k0 ? (min(it.chunk, it.nk - it.k0) + kKcTile - 1) / kKcTile : 0;
+  return it;
 }
 
-// For each lane l: how many of this warp's keys (thread i takes keys i + kSdThreads s,
-// s < R) are >= T | l << shift, where the bits of T below shift + w are zero and l < 2^w
-// (lanes l >= 2^w count the keys at or above T + 2^(shift + w), the bucket's upper end).
-// `first`: lane 0 counts the keys >= 1 instead (the candidates).  Bit-sliced: one
-// ballot per digit bit and slot, then a comparison of the lane's digit l against every
-// key's digit on the ballot masks.
-__device__ __forceinline__ int warp_count_digits(const uint32_t* keys, int n, int R, uint32_t T, int shift, int w,
-                                                 bool first) {
-  const int lane = threadIdx.x & 31;
-  const bool top = shift + w >= 32;  // the digit holds the key's top bits (a shift by 32 is undefined)
-  const uint32_t hT = top ? 0u : T >> (shift + w);
-  const uint32_t dmask = (1u << w) - 1u;
-  int cnt = 0;
-#pragma unroll 2
-  for (int s = 0; s < R; ++s) {
-    const int j = static_cast<int>(threadIdx.x) + kSdThreads * s;
-    const uint32_t k = j < n ? keys[j] : 0u;
-    const uint32_t hk = top ? 0u : k >> (shift + w);
-    const bool in = hk == hT;
-    const uint32_t d = (k >> shift) & dmask;
-    const unsigned A = __ballot_sync(0xffffffffu, hk > hT);
-    unsigned gt = 0u, eq = __ballot_sync(0xffffffffu, in);
-#pragma unroll
-    for (int i = 4; i >= 0; --i) {
-      if (i < w) {
-        const unsigned Bi = __ballot_sync(0xffffffffu, in && ((d >> i) & 1u));
-        const unsigned tt = eq & Bi;
-        const bool one = (lane >> i) & 1;
-        gt = one ? gt : (gt | tt);
-        eq = one ? tt : (eq & ~Bi);
-      }
-    }
-    int c = __popc(A) + (lane < (1 << w) ? __popc(gt | eq) : 0);
-    if (first) {
-      const int cand = __popc(__ballot_sync(0xffffffffu, k != 0u));
-      if (lane == 0) c = cand;
-    }
-    cnt += c;
-  }
-  return cnt;
-}
-
-// k-th largest of the n keys in shared memory by all kSdThreads threads; same result as
-// warp_radix_threshold.  Radix search on the 32 key bits in digits of 5 (the last one
-// 2): lane l of every warp counts the keys >= T | l << shift (warp_count_digits), the
-// counts meet in S.cnt (double-buffered: one barrier per digit) and the largest digit
-// with at least `want` keys at or above it is taken.  As soon as the chosen digit's
-// bucket holds at most 32 keys, they are gathered and ranked directly.
-__device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys, int n, int want, SdSmem& S) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int R = (n + kSdThreads - 1) / kSdThreads;
+// k-th largest of the n keys in shared memory (0: not a candidate) by all kSdThreads
+// threads; same result as warp_radix_threshold.  One pass counts the candidates and
+// takes the AND and OR of their keys: the bits above the highest bit where they differ
+// are common to all of them.  Below it the threshold is resolved in digits of up to
+// kSdHistBits bits: a shared-memory histogram of the digit over the keys of the current
+// bucket (keys that agree with the threshold on every bit above the digit), then a
+// suffix scan over the bins finds the digit whose bin holds the (want - above)-th
+// largest key.  As soon as that bin holds at most 32 keys they are ranked directly.
+__device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys, int n, int want, uint32_t* hist,
+                                                            SdSmem& S) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   TopkThreshold r;
   r.all_ties = false;
   if (want <= 0) {
@@ -133,36 +135,101 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     r.ties = 0;
     return r;
   }
-  int buf = 0;
-  auto count_ge = [&](uint32_t T, int shift, int w, bool first) -> int {
-    S.cnt[buf][warp][lane] = warp_count_digits(keys, n, R, T, shift, w, first);
-    __syncthreads();
-    int tot = 0;
+  int cnt = 0;
+  uint32_t kand = 0xffffffffu, kor = 0u;
+  for (int j = tid; j < n; j += kSdThreads) {
+    const uint32_t k = keys[j];
+    if (k != 0u) {
+      ++cnt;
+      kand &= k;
+      kor |= k;
+    }
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  kand = __reduce_and_sync(0xffffffffu, kand);
+  kor = __reduce_or_sync(0xffffffffu, kor);
+  if (lane == 0) {
+    S.wred[0][warp] = cnt;
+    S.wred[1][warp] = static_cast<int>(kand);
+    S.wred[2][warp] = static_cast<int>(kor);
+  }
+  __syncthreads();
+  cnt = 0;
+  kand = 0xffffffffu;
+  kor = 0u;
 #pragma unroll
-    for (int ww = 0; ww < kSdWarps; ++ww) tot += S.cnt[buf][ww][lane];
-    buf ^= 1;
-    return tot;
-  };
-  // first digit (bits 31..27); lane 0 counts the candidates (keys >= 1): bucket 0 is [1, 2^27)
-  int tot = count_ge(0u, 27, 5, true);
-  if (__shfl_sync(0xffffffffu, tot, 0) <= want) {  // at most `want` candidates: take them all
+  for (int w = 0; w < kSdWarps; ++w) {
+    cnt += S.wred[0][w];
+    kand &= static_cast<uint32_t>(S.wred[1][w]);
+    kor |= static_cast<uint32_t>(S.wred[2][w]);
+  }
+  if (cnt <= want) {  // at most `want` candidates: take them all
     r.key = 0;
     r.ties = 0;
     return r;
   }
-  uint32_t T = 0;
-  int shift = 27, above = 0, inb = 0;  // bucket [max(T, 1), T + 2^shift): `inb` keys, `above` keys above it
+  if (kand == kor) {  // every candidate has the same key
+    r.key = kand;
+    r.ties = want;
+    return r;
+  }
+  int top = 31 - __clz(kand ^ kor);  // highest bit in which candidates differ
+  uint32_t T = top == 31 ? 0u : (kand >> (top + 1)) << (top + 1);  // the common bits above it
+  int above = 0;                      // candidates above the current bucket
+  int shift = 0, inb = 0;
   for (;;) {
-    const unsigned ok = __ballot_sync(0xffffffffu, tot >= want);  // lane 0 always qualifies
-    const int l = 31 - __clz(ok);
-    const int nxt = __shfl_sync(0xffffffffu, tot, min(l + 1, 31));
-    if (l < 31) above = nxt;
-    inb = __shfl_sync(0xffffffffu, tot, l) - above;
-    T |= static_cast<uint32_t>(l) << shift;
-    if (inb <= 32 || shift == 0) break;
-    const int w = shift >= 7 ? 5 : shift;  // 27, 22, 17, 12, 7, 2 (5 bits each), then bits 1..0
-    shift -= w;
-    tot = count_ge(T, shift, w, false);
+    const int w = min(kSdHistBits, top + 1);
+    shift = top + 1 - w;
+    const int nb = 1 << w;
+    for (int i = tid; i < nb; i += kSdThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int j = tid; j < n; j += kSdThreads) {
+      const uint32_t k = keys[j];
+      const bool in = k != 0u && (top == 31 || (k >> (top + 1)) == (T >> (top + 1)));
+      if (in) atomicAdd(&hist[(k >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
+    }
+    __syncthreads();
+    // thread i owns bins [i B, i B + B); `higher` counts the keys in the bins of the
+    // threads above it, so the bin of the (need)-th largest key is in the thread with
+    // higher < need <= higher + own
+    const int need = want - above;
+    const int b0 = tid * kSdBinsPerThread;
+    int own = 0;
+#pragma unroll
+    for (int e = 0; e < kSdBinsPerThread; ++e) own += b0 + e < nb ? static_cast<int>(hist[b0 + e]) : 0;
+    int incl = own;  // this lane's and the higher lanes' bins
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    if (lane == 0) S.wsum[warp] = incl;
+    __syncthreads();
+    int higher = incl - own;
+#pragma unroll
+    for (int ww = 0; ww < kSdWarps; ++ww) higher += ww > warp ? S.wsum[ww] : 0;
+    if (higher < need && need <= higher + own) {
+      int acc = higher;
+#pragma unroll 1
+      for (int e = kSdBinsPerThread - 1; e >= 0; --e) {
+        const int bin = b0 + e;
+        if (bin >= nb) continue;
+        const int h = static_cast<int>(hist[bin]);
+        if (acc + h >= need) {
+          S.dig = bin;
+          S.dig_above = acc;
+          S.dig_in = h;
+          break;
+        }
+        acc += h;
+      }
+    }
+    __syncthreads();
+    T |= static_cast<uint32_t>(S.dig) << shift;
+    above += S.dig_above;
+    inb = S.dig_in;
+    if (shift == 0 || inb <= 32) break;
+    top = shift - 1;
   }
   if (shift == 0) {  // the bucket is the single value T
     r.key = T;
@@ -172,9 +239,9 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   }
   // rank the <= 32 keys of the bucket directly: the answer is the (want - above)-th largest
   const uint32_t lo = max(T, 1u), hi = T + (1u << shift);
-  if (threadIdx.x == 0) S.nlist = 0;
+  if (tid == 0) S.nlist = 0;
   __syncthreads();
-  for (int j = threadIdx.x; j < n; j += kSdThreads) {
+  for (int j = tid; j < n; j += kSdThreads) {
     const uint32_t k = keys[j];
     if (k >= lo && k < hi) S.list[atomicAdd(&S.nlist, 1)] = k;
   }
@@ -205,7 +272,8 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
 // the warp and in the slot.  Tie ranks (only when some keys equal to T stay out) come
 // from the same two passes run on the tie flags first.
 __device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, TopkThreshold th, int cur,
-                                                   int n_init, int n_local, int topk, int32_t* out, SdSmem& S) {
+                                                   int n_init, int n_local, int topk, int32_t* out,
+                                                   unsigned char* tflag, SdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   const int R = (n + kSdThreads - 1) / kSdThreads;
@@ -276,11 +344,11 @@ __device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, 
     const int rk = rank_of(s, __ballot_sync(0xffffffffu, f));
     int j;
     const uint32_t k = key_at(s, j);
-    S.tflag[s][threadIdx.x] = static_cast<unsigned char>(
+    tflag[s * kSdThreads + threadIdx.x] = static_cast<unsigned char>(
         j < n && (forced(j) || k > th.key || (k == th.key && rk < th.ties)) ? 1 : 0);
   }
   __syncthreads();
-  auto take = [&](int s) { return S.tflag[s][threadIdx.x] != 0; };
+  auto take = [&](int s) { return tflag[s * kSdThreads + threadIdx.x] != 0; };
   const int total = slot_counts(take);
   for (int s = 0; s < R; ++s) {
     const bool f = take(s);
@@ -291,32 +359,13 @@ __device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, 
   __syncthreads();
 }
 
-// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.
-__global__ void __launch_bounds__(kSdThreads)
-    select_decode_kernel(const __grid_constant__ CUtensorMap tm_kc, const SelDecodeParams p) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* ring = align_smem(smem_raw, 1024);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(ring + kSdStages * kKcTileBytes);  // [16][kSdBStride], ord_enc
-  SdSmem& S = *reinterpret_cast<SdSmem*>(bm + kGroupRows * kSdBStride);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ring);  // CTA 0 only, once every tile is consumed
-
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int c = static_cast<int>(cluster.block_rank());
-  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
-  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  allow_dependent_launch();  // the decode attention may set up while this selection runs
-  grid_dependency_wait();    // q, Kc and lens may come from the previous kernel
-  const int n = min(max(p.lens[b], 0), p.Lmax);
-  const int nk = n >= kKernel ? (n - kKernel) / kStride + 1 : 0;
-  const int cur = n > 0 ? (n - 1) / kBlock : -1;
-  const int chunk = ((nk + C - 1) / C + kKcTile - 1) / kKcTile * kKcTile;  // kernels per CTA
-  const int nq = chunk / 4;                                                 // blocks per CTA
-  const int k0 = c * chunk;
-  const int ntiles = nk > k0 ? (min(chunk, nk - k0) + kKcTile - 1) / kKcTile : 0;
+// Phase 1, all threads of the CTA: barrier set-up, then this CTA's Kc tiles streamed and
+// scored (online (max, sum of exp2) per head, block maxima in bm), then the CTA's state
+// per head in S.cm / S.cl.  Ends after a CTA barrier.
+__device__ __forceinline__ void sd_score_chunk(const CUtensorMap* tm_kc, const SelDecodeParams& p, const SdItem& it,
+                                               unsigned char* ring, uint32_t* bm, SdSmem& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
+  const int nk = it.nk, nq = it.nq, k0 = it.k0, ntiles = it.ntiles;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSdStages; ++s) {
       mbar_init(&S.full[s], 1);
@@ -334,16 +383,16 @@ __global__ void __launch_bounds__(kSdThreads)
   if (warp == kSdConsumers) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && ntiles > 0) {
-      prefetch_tmap(&tm_kc);
-      const int row0 = static_cast<int>(bg * p.NKmax) + k0;
+      prefetch_tmap(tm_kc);
+      const int row0 = static_cast<int>(it.bg * p.NKmax) + k0;
       int i = 0;
       for (; i < ntiles; ++i) {
         const int st = i % kSdStages, u = i / kSdStages;
         if (u > 0 && !mbar_wait(&S.empty[st], (u - 1) & 1, &S.abort)) break;
         unsigned char* dst = ring + st * kKcTileBytes;
         mbar_arrive_expect_tx(&S.full[st], kKcTileBytes);
-        tma_load_2d(dst, &tm_kc, &S.full[st], 0, row0 + i * kKcTile);
-        tma_load_2d(dst + kKcTileBytes / 2, &tm_kc, &S.full[st], 64, row0 + i * kKcTile);
+        tma_load_2d(dst, tm_kc, &S.full[st], 0, row0 + i * kKcTile);
+        tma_load_2d(dst + kKcTileBytes / 2, tm_kc, &S.full[st], 64, row0 + i * kKcTile);
       }
       if (S.abort) {  // let every issued copy land before the ring is reused or released
         for (int j = max(0, i - kSdStages); j < i; ++j) mbar_wait_drain(&S.full[j % kSdStages], (j / kSdStages) & 1);
@@ -356,7 +405,7 @@ __global__ void __launch_bounds__(kSdThreads)
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     if (ntiles > 0) {
       uint32_t qa[8][4];
-      load_q_frags(p.q + (static_cast<long long>(b) * p.Hq + g * p.G) * kHeadDim, p.G, qa);
+      load_q_frags(p.q + (static_cast<long long>(it.b) * p.Hq + it.g * p.G) * kHeadDim, p.G, qa);
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % kSdStages;
         if (!mbar_wait(&S.full[st], (i / kSdStages) & 1, &S.abort)) break;
@@ -455,8 +504,15 @@ __global__ void __launch_bounds__(kSdThreads)
     S.cm[h] = M;
     S.cl[h] = L;
   }
-  cluster.sync();  // every CTA's tiles are consumed and its partial state is final
+  __syncthreads();
+}
 
+// Phase 2, after a cluster barrier that follows phase 1 in every CTA: the log-sum-exp per
+// head from every CTA's state, the previous CTA's carry, and the keys of this CTA's blocks
+// stored into CTA 0's key array (`keys` is this CTA's own scratch address of that array).
+__device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group& cluster, const SelDecodeParams& p,
+                                              const SdItem& it, uint32_t* keys, const uint32_t* bm, SdSmem& S) {
+  const int C = it.C, c = it.c, nq = it.nq, cur = it.cur;
   // gather every CTA's (max, sum) and the previous CTA's carry, all loads in flight at once
   for (int e = threadIdx.x; e < kGroupRows * C; e += kSdThreads) {
     const int r = e / kGroupRows, h = e % kGroupRows;
@@ -465,9 +521,10 @@ __global__ void __launch_bounds__(kSdThreads)
   }
   if (threadIdx.x >= kSdThreads - kGroupRows) {
     const int h = threadIdx.x - (kSdThreads - kGroupRows);
-    S.carry[h] = c > 0 ? ord_dec(cluster.map_shared_rank(bm, c - 1)[h * kSdBStride + nq]) : -INFINITY;
+    S.carry[h] = c > 0 ? ord_dec(cluster.map_shared_rank(const_cast<uint32_t*>(bm), c - 1)[h * kSdBStride + nq])
+                       : -INFINITY;
   }
-  if (c == 0) {  // zero padding up to a multiple of 4 keys for the vector scan
+  if (c == 0) {  // zero padding up to a multiple of 4 keys
     for (int j = cur + 1 + threadIdx.x; j < ((cur + 4) & ~3); j += kSdThreads) keys[j] = 0u;
   }
   __syncthreads();
@@ -483,38 +540,65 @@ __global__ void __launch_bounds__(kSdThreads)
   }
   __syncthreads();
   // this CTA's blocks: [c nq, (c + 1) nq); the last CTA also takes the rest up to cur
-  {
-    uint32_t* keys0 = cluster.map_shared_rank(keys, 0);
-    const int jb0 = c * nq;
-    const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
-    for (int j = jb0 + threadIdx.x; j < jb1; j += kSdThreads) {
-      const int ql = j - jb0;  // <= nq, since cur + 1 <= ceil(nk / 4) + 1 <= C nq + 1
-      const bool eligible = block_eligible(j, nk - 1, p.pool_mode);
-      const bool forced = j < p.n_init || j > cur - p.n_local;
-      uint32_t key = 0u;
-      if (eligible && !forced && ql <= nq) {
-        float sc = 0.f;
-        for (int h = 0; h < p.G; ++h) {
-          float mb = ord_dec(bm[h * kSdBStride + ql]);
-          if (ql == 0 && p.pool_mode == kPoolOverlap) mb = fmaxf(mb, S.carry[h]);
-          sc += p.score_mode == kScoreLogitSum ? mb : ex2(mb - S.lse2[h]);
-        }
-        key = score_key(sc, p.score_mode);
+  uint32_t* keys0 = cluster.map_shared_rank(keys, 0);
+  const int jb0 = c * nq;
+  const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
+  for (int j = jb0 + threadIdx.x; j < jb1; j += kSdThreads) {
+    const int ql = j - jb0;  // <= nq, since cur + 1 <= ceil(nk / 4) + 1 <= C nq + 1
+    const bool eligible = block_eligible(j, it.nk - 1, p.pool_mode);
+    const bool forced = j < p.n_init || j > cur - p.n_local;
+    uint32_t key = 0u;
+    if (eligible && !forced && ql <= nq) {
+      float sc = 0.f;
+      for (int h = 0; h < p.G; ++h) {
+        float mb = ord_dec(bm[h * kSdBStride + ql]);
+        if (ql == 0 && p.pool_mode == kPoolOverlap) mb = fmaxf(mb, S.carry[h]);
+        sc += p.score_mode == kScoreLogitSum ? mb : ex2(mb - S.lse2[h]);
       }
-      keys0[j] = key;
+      key = score_key(sc, p.score_mode);
     }
+    keys0[j] = key;
   }
-  cluster.sync();  // CTA 0 holds every key; no CTA reads a peer's shared memory after this
-  if (c != 0) return;
+}
 
-  int32_t* out = p.idx + bg * p.topk;
-  if (cur < 0) {
+// Phase 3, CTA 0 after a cluster barrier that follows phase 2 in every CTA: the top-k of
+// the keys in `scratch` (kSdScratchBytes, the drained tile ring) and the ascending list,
+// -1 padded, written to out[0 .. topk) (global or shared memory).  Ends after a CTA barrier.
+__device__ __forceinline__ void sd_select(const SelDecodeParams& p, const SdItem& it, unsigned char* scratch,
+                                          int32_t* out, SdSmem& S) {
+  const uint32_t* keys = reinterpret_cast<const uint32_t*>(scratch + kSdKeysOff);
+  if (it.cur < 0) {
     for (int e = threadIdx.x; e < p.topk; e += kSdThreads) out[e] = -1;
+    __syncthreads();
     return;
   }
-  const int want = p.topk - forced_count(cur, p.n_init, p.n_local);
-  const TopkThreshold th = cta_topk_threshold(keys, cur + 1, want, S);
-  cta_emit_selection(keys, cur + 1, th, cur, p.n_init, p.n_local, p.topk, out, S);
+  const int want = p.topk - forced_count(it.cur, p.n_init, p.n_local);
+  const TopkThreshold th =
+      cta_topk_threshold(keys, it.cur + 1, want, reinterpret_cast<uint32_t*>(scratch + kSdHistOff), S);
+  cta_emit_selection(keys, it.cur + 1, th, it.cur, p.n_init, p.n_local, p.topk, out, scratch + kSdFlagOff, S);
+}
+
+// grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.
+__global__ void __launch_bounds__(kSdThreads)
+    select_decode_kernel(const __grid_constant__ CUtensorMap tm_kc, const SelDecodeParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* ring = align_smem(smem_raw, 1024);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(ring + kSdStages * kKcTileBytes);  // [16][kSdBStride], ord_enc
+  SdSmem& S = *reinterpret_cast<SdSmem*>(ring + kSdRegionBytes);
+
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int c = static_cast<int>(cluster.block_rank());
+  allow_dependent_launch();  // the decode attention may set up while this selection runs
+  grid_dependency_wait();    // q, Kc and lens may come from the previous kernel
+  const SdItem it = sd_item(p, C, c, blockIdx.x / C);  // clusters are consecutive blocks
+  sd_score_chunk(&tm_kc, p, it, ring, bm, S);
+  cluster.sync();  // every CTA's tiles are consumed and its partial state is final
+  sd_block_keys(cluster, p, it, reinterpret_cast<uint32_t*>(ring + kSdKeysOff), bm, S);
+  cluster.sync();  // CTA 0 holds every key; no CTA reads a peer's shared memory after this
+  if (c != 0) return;
+  sd_select(p, it, ring, p.idx + it.bg * p.topk, S);
 }
 
 }  // namespace infllmv2

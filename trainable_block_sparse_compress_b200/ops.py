@@ -328,8 +328,35 @@ def prefill_chunk(p: Params, q, k_cache, v_cache, kc, q_lens=None, kv_lens=None)
     return o, lse, idx
 
 
+def decode_step(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, kc: torch.Tensor,
+                lens: torch.Tensor, block_idx: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+    """One decode step in one launch: block selection for the query at lens[b]-1, then
+    sparse attention over the selected blocks.  Returns (o, lse, block_idx)."""
+    Lmax = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (p.batch, p.num_q_heads, p.head_dim))
+    _need(k_cache, "k_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(v_cache, "v_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
+    _need(kc, "kc", torch.bfloat16, (p.batch, p.num_kv_heads, num_kernels(p, Lmax), p.head_dim))
+    _need(lens, "lens", torch.int32, (p.batch,))
+    if block_idx is None:
+        block_idx = torch.empty((p.batch, p.num_kv_heads, 1, p.topk), dtype=torch.int32, device=q.device)
+    _need(block_idx, "block_idx", torch.int32, (p.batch, p.num_kv_heads, 1, p.topk))
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "o", torch.bfloat16, tuple(q.shape))
+    if want_lse and lse is None:
+        lse = torch.empty((p.batch, p.num_q_heads), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (p.batch, p.num_q_heads))
+    st = _lib.load().infllmv2_decode_step(ctypes.byref(p.c()), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kc),
+                                          _ptr(lens), Lmax, _ptr(block_idx), _ptr(out), _ptr(lse), _stream())
+    _lib.check("infllmv2_decode_step", st)
+    return out, lse, block_idx
+
+
 def decode(p: Params, q, k_cache, v_cache, kc, lens, Lmax):
-    """One decode step over a filled cache: select -> sparse attention.  Returns (o, lse, idx)."""
-    idx = select_blocks_decode(p, q, kc, lens, Lmax)
-    o, lse = sparse_attn_decode(p, q, k_cache, v_cache, lens, idx)
-    return o, lse, idx
+    """One decode step over a filled cache (Lmax = the caches' length): select -> sparse
+    attention, fused in one launch.  Returns (o, lse, idx)."""
+    assert k_cache.shape[2] == Lmax, "Lmax is the caches' length"
+    return decode_step(p, q, k_cache, v_cache, kc, lens)
