@@ -361,9 +361,12 @@ def run_e2e(args, p, x, device):
 
 
 def run_decode(args, workload, rank, world, device, pk, peak_src):
-    """One decode step (selection -> attention, fused in one launch) over filled caches, L2
-    flushed before every step (outside the timed events).  Inputs: the same seed as the
-    parity tests.  The two separate calls are timed too, for the per-kernel split."""
+    """One decode step over filled caches, in one launch: the new token appended (its K/V
+    rows and the semantic kernel it completes), block selection, attention.  L2 flushed
+    before every step (outside the timed events).  Inputs: the same seed as the parity
+    tests; the appended token is each sequence's last one (rewritten in place, so every
+    step sees the same cache).  The step without the append and the two separate calls are
+    timed too, for the split."""
     wl = WORKLOADS[workload]
     p = ops.Params.from_workload(wl)
     x = make_inputs(wl, seed=dist.rank_seed(args.seed, rank))
@@ -378,11 +381,23 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
+    last = (lens.long() - 1).clamp(min=0)
+    bidx = torch.arange(p.batch, device=device)
+    k_new = k[bidx, :, last].contiguous()
+    v_new = v[bidx, :, last].contiguous()
+    lens_prev = lens - 1  # cached tokens before the step
+    lens_out = torch.empty_like(lens)
+
     def step():
+        ops.decode_step(p, q, k, v, kc, lens_prev, k_new=k_new, v_new=v_new, lens_out=lens_out, block_idx=idx,
+                        out=o, lse=lse)
+
+    def step_no_append():
         ops.decode_step(p, q, k, v, kc, lens, block_idx=idx, out=o, lse=lse)
 
     for _ in range(max(3, args.warmup)):
         step()
+        step_no_append()
     n = max(args.steps, 20)
 
     def flush_l2():
@@ -397,6 +412,14 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         ev[s][1].record(stream)
     torch.cuda.synchronize()
     step_us = [ev[s][0].elapsed_time(ev[s][1]) * 1e3 for s in range(n)]
+    evn = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for s in range(n):
+        flush_l2()
+        evn[s][0].record(stream)
+        step_no_append()
+        evn[s][1].record(stream)
+    torch.cuda.synchronize()
+    noapp_us = statistics.median(evn[s][0].elapsed_time(evn[s][1]) * 1e3 for s in range(n))
     # the two separate calls: the pair (the attention launch overlaps the end of the
     # selection), then each kernel alone (an event between them keeps the attention from
     # starting early)
@@ -420,12 +443,8 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     att_us = [evk[s][1].elapsed_time(evk[s][2]) * 1e3 for s in range(n)]
     us = statistics.median(step_us)
     us = dist.max_over_ranks(us, world, device)
-    # cache maintenance of the step (measured apart from the step above): re-append each
+    # the standalone append kernel (infllmv2_append_kv), for comparison: re-append each
     # sequence's last token, which rewrites the same rows and kernel and leaves lens as it was
-    last = (lens.long() - 1).clamp(min=0)
-    bidx = torch.arange(p.batch, device=device)
-    k_new = k[bidx, :, last].contiguous()
-    v_new = v[bidx, :, last].contiguous()
     lens_w = torch.empty_like(lens)
     eva = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
     for s in range(n):
@@ -438,6 +457,8 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
     app_us = statistics.median(eva[s][0].elapsed_time(eva[s][1]) * 1e3 for s in range(n))
     app_bytes = p.batch * p.num_kv_heads * 2 * 2 * p.head_dim  # the new K and V rows read and written
     sel_b, att_b = decode_bytes(p, x.lens.numpy())
+    assert torch.equal(lens_out, lens)
+    step_b = sel_b + att_b + app_bytes  # Kc, the selected K/V blocks, the appended rows
     att_kernel = "attn_decode_cluster_kernel" if ws_a.numel() == 0 else "attn_kernel + attn_merge_kernel"
     hbm = pk["hbm_gbs"]
     sel_med, att_med = statistics.median(sel_us), statistics.median(att_us)
@@ -448,14 +469,16 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
         "workload": workload, "value": us, "unit": "us/step", "higher_is_better": False,
         "batch": p.batch, "mean_len": float(x.lens.float().mean()), "steps": n,
         "l2": "flushed before every step (write then read a 2x L2 buffer, outside the timed events)",
-        "roofline": {"bound": "hbm", "achieved": (sel_b + att_b) / us / 1e3, "peak": hbm, "unit": "GB/s",
-                     "frac": (sel_b + att_b) / us / 1e3 / hbm, "algorithmic_bytes": sel_b + att_b,
+        "roofline": {"bound": "hbm", "achieved": step_b / us / 1e3, "peak": hbm, "unit": "GB/s",
+                     "frac": step_b / us / 1e3 / hbm, "algorithmic_bytes": step_b,
                      "traffic": tr_f, "peak_source": f"{peak_src} (hbm_gbs)"},
         "kernels": {
-            "step": {"kernel": "decode_step_kernel", "us": us, "algorithmic_bytes": sel_b + att_b,
-                     "achieved_GBps": (sel_b + att_b) / us / 1e3, "traffic": tr_f},
+            "step": {"kernel": "decode_step_kernel", "us": us, "algorithmic_bytes": step_b,
+                     "achieved_GBps": step_b / us / 1e3, "traffic": tr_f},
         },
         "gpu_launches_per_step": 1,
+        "step": "append of the new token + block selection + sparse attention (infllmv2_decode_step with k_new)",
+        "step_without_append_us": noapp_us,
         "separate_calls": {
             "note": "infllmv2_select_blocks(DECODE) then infllmv2_sparse_attn_decode on the same inputs",
             "pair_us": statistics.median(pair_us),
@@ -465,7 +488,7 @@ def run_decode(args, workload, rank, world, device, pk, peak_src):
                      "achieved_GBps": att_b / att_med / 1e3, "traffic": tr_a},
         },
         "append": {"kernel": "append_kv_kernel", "us": app_us, "bytes_per_step": app_bytes,
-                   "note": "cache maintenance of a decode step (new K/V rows, completed kernels), timed apart"},
+                   "note": "the standalone cache-maintenance call, timed apart; the step above appends itself"},
     }
 
 

@@ -222,27 +222,39 @@ INFLLMV2_API int infllmv2_sparse_attn_decode(const infllmv2_params* p, const voi
                                 const int32_t* block_idx, void* o, float* lse, void* ws,
                                 size_t ws_bytes, infllmv2_stream_t stream);
 
-/* One whole decode step: infllmv2_select_blocks(DECODE) followed by
- * infllmv2_sparse_attn_decode on the list it selects, in one launch ([S] s2.1: the block
- * selection serves decoding as well as prefill; s2.1.2: the group's heads share the
- * blocks; s2.1.3: attention over the selected blocks only).  A thread-block cluster per
- * (b, kv-head) scores Kc, selects the blocks and attends to them without a round trip
- * through global memory, so clusters overlap each other's selection and attention.
- * Same results as the two calls: block_idx bit-identical, o and lse from the same
- * per-block arithmetic (the split of the list over the cluster's CTAs may differ, so o
- * and lse may differ from the separate call in the last bits).
+/* One whole decode step in one launch: optionally the cache maintenance of
+ * infllmv2_append_kv for the new token, then infllmv2_select_blocks(DECODE) and
+ * infllmv2_sparse_attn_decode on the list it selects ([S] s2.1: the block selection
+ * serves decoding as well as prefill; s2.1.2: the group's heads share the blocks and the
+ * semantic kernels summarise the cached keys; s2.1.3: attention over the selected blocks
+ * only).  A thread-block cluster per (b, kv-head) scores Kc, selects the blocks and
+ * attends to them without a round trip through global memory, so clusters overlap each
+ * other's selection and attention.  Same results as the separate calls: block_idx
+ * bit-identical, o and lse from the same per-block arithmetic (the split of the list over
+ * the cluster's CTAs may differ, so o and lse may differ from the separate call in the
+ * last bits).
  *   q          bf16 [B, Hq, d]
- *   k_cache, v_cache  bf16 [B, Hkv, Lmax, d]
- *   kc         bf16 [B, Hkv, NK(Lmax), d] (may be NULL when NK(Lmax) = 0)
- *   lens       int32 [B] device; the query sits at min(lens[b], Lmax) - 1 (none when
- *              lens[b] <= 0: the list is all -1, o is 0 and lse is -inf)
+ *   k_new, v_new  bf16 [B, Hkv, d], or both NULL.  Given: lens[b] counts the cached
+ *              tokens before the step; the token's rows are written at position lens[b]
+ *              of the caches and the semantic kernel it completes to kc (exactly as
+ *              infllmv2_append_kv), the query sits at lens[b] and lens_out[b] = lens[b] + 1.
+ *              A sequence with lens[b] outside [0, Lmax) is not appended (lens_out[b] =
+ *              lens[b], INFLLMV2_DEVERR_CACHE_FULL in the device error word).  NULL: the
+ *              caches already hold the query's token, which sits at min(lens[b], Lmax) - 1.
+ *   k_cache, v_cache  bf16 [B, Hkv, Lmax, d] (written only when appending)
+ *   kc         bf16 [B, Hkv, NK(Lmax), d] (may be NULL when NK(Lmax) = 0 and nothing is appended)
+ *   lens       int32 [B] device (read only); a sequence with no query (length <= 0) gets
+ *              an all -1 list, o = 0 and lse = -inf
+ *   lens_out   int32 [B] device, distinct from lens; required when appending, else ignored
  *   block_idx  int32 [B, Hkv, 1, topk] (output)
  *   o          bf16 [B, Hq, d];  lse fp32 [B, Hq] or NULL
- * No workspace.  INVALID_ARG for null / misaligned pointers, UNSUPPORTED when the
- * device cannot hold one cluster of the chosen size. */
-INFLLMV2_API int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_cache,
-                                      const void* v_cache, const void* kc, const int32_t* lens, int32_t Lmax,
-                                      int32_t* block_idx, void* o, float* lse, infllmv2_stream_t stream);
+ * No workspace.  INVALID_ARG for null / misaligned pointers (or k_new without v_new,
+ * lens_out missing or equal to lens), UNSUPPORTED when the device cannot hold one cluster
+ * of the chosen size. */
+INFLLMV2_API int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new, const void* v_new,
+                                      void* k_cache, void* v_cache, void* kc, const int32_t* lens, int32_t* lens_out,
+                                      int32_t Lmax, int32_t* block_idx, void* o, float* lse,
+                                      infllmv2_stream_t stream);
 
 /* Backward of the prefill sparse attention over fixed block lists ([S] s2.1, s2.1.3:
  * the sparse attention is trained; the top-k block choice is constant almost

@@ -198,27 +198,46 @@ def test_backward_rejects_bad_arguments_before_launch(lib):
 
 def test_decode_step_rejects_bad_arguments_before_launch(lib):
     good = 4096  # a fake, 16-byte aligned "device address": never dereferenced
+    other = 8192
     f = lib.infllmv2_decode_step
-    # q, k_cache, v_cache, kc, lens, Lmax, block_idx, o, lse
-    args = [good, good, good, good, good, 1024, good, good, None]
-    for i in (0, 1, 2, 4, 6, 7):  # required pointers
+    # q, k_new, v_new, k_cache, v_cache, kc, lens, lens_out, Lmax, block_idx, o, lse
+    args = [good, None, None, good, good, good, good, None, 1024, good, good, None]
+    for i in (0, 3, 4, 6, 9, 10):  # required pointers
         bad = list(args)
         bad[i] = None
         assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG, i
-    for i in (0, 1, 2, 3, 6, 7):  # 16-byte aligned
+    for i in (0, 3, 4, 5, 9, 10):  # 16-byte aligned
         bad = list(args)
         bad[i] = good + 8
         assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG, i
     bad = list(args)
-    bad[4] = good + 2  # lens 4-byte aligned
+    bad[6] = good + 2  # lens 4-byte aligned
     assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
     bad = list(args)
-    bad[8] = good + 1  # lse 4-byte aligned
+    bad[11] = good + 1  # lse 4-byte aligned
     assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
     bad = list(args)
-    bad[3] = None  # kc is needed once a semantic kernel exists
+    bad[5] = None  # kc is needed once a semantic kernel exists
     assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
     bad = list(args)
-    bad[5] = 0
+    bad[8] = 0
     assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
     assert f(cp(head_dim=64), *args, None) == _lib.ERR_UNSUPPORTED
+    # appending: both new rows, 16-byte aligned, and a lens_out distinct from lens
+    app = list(args)
+    app[1], app[2], app[7] = good, good, other
+    bad = list(app)
+    bad[2] = None
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(app)
+    bad[1] = good + 8
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(app)
+    bad[7] = None
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(app)
+    bad[7] = good  # == lens
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG
+    bad = list(app)
+    bad[7] = other + 2
+    assert f(cp(), *bad, None) == _lib.ERR_INVALID_ARG

@@ -112,6 +112,8 @@ SELECT_CASES = [
     (1, 2000, 16, 1, 256, 1, 2),  # topk larger than the number of blocks
     (1, 20, 16, 1, 4, 1, 2),      # no complete kernel: forced blocks only
     (1, 1100, 4, 1, 3, 0, 0),     # nothing forced
+    (1, 1500, 4, 2, 8, 1, 2),     # G = 2
+    (1, 14000, 2, 2, 24, 1, 2),   # G = 1 past the tensor-core kernel's key storage: m16n8k16 kernel
 ]
 
 
@@ -130,6 +132,21 @@ def test_select_prefill_matches_oracle(B, L, Hq, Hkv, topk, ni, nl):
     kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
     idx_g = ops.select_blocks_prefill(p, x.q.cuda(), kc_t).cpu().numpy()
     rows = prefill_rows(L)
+    idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
+    compare_selection(idx_g[:, :, rows], idx_o, sc, np.tile(rows, (B, 1)), p)
+
+
+def test_select_prefill_long_sequence():
+    # 200,000 tokens at G = 16: 3125 blocks of keys per query row, which the tensor-core
+    # kernel holds by running its Kc ring with two slots instead of three
+    B, L, Hq, Hkv, topk = 1, 200000, 16, 1, 96
+    x = inputs(B, L, Hq, Hkv, seed=210)
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    op = oparams(p)
+    kc_o = oracle.compress(op, as_u16(x.k))
+    kc_t = torch.from_numpy(kc_o.view(np.int16)).view(torch.bfloat16).cuda()
+    idx_g = ops.select_blocks_prefill(p, x.q.cuda(), kc_t).cpu().numpy()
+    rows = np.unique(np.concatenate([np.arange(0, L, 997), np.arange(L - 64, L)]))
     idx_o, sc = oracle.select(op, as_u16(x.q), kc_o, rows=rows, want_scores=True)
     compare_selection(idx_g[:, :, rows], idx_o, sc, np.tile(rows, (B, 1)), p)
 
@@ -221,7 +238,8 @@ def test_select_decode_matches_oracle(lens, Lmax, Hq, Hkv, topk):
 
 # -------------------------------------------------------------------- attention
 
-ATTN_CASES = [(1, 4500, 32, 2, 16), (2, 1000, 8, 1, 6), (1, 777, 2, 2, 5), (1, 700, 16, 1, 16), (1, 64, 16, 1, 4)]
+ATTN_CASES = [(1, 4500, 32, 2, 16), (2, 1000, 8, 1, 6), (1, 777, 2, 2, 5), (1, 700, 16, 1, 16), (1, 64, 16, 1, 4),
+              (1, 900, 8, 2, 6), (1, 500, 4, 2, 4)]
 
 
 @pytest.mark.parametrize("B,L,Hq,Hkv,topk", ATTN_CASES)
@@ -436,6 +454,40 @@ def test_decode_step_empty_sequence_and_determinism():
     compare_selection(idx_gn, idx_o, sc, (lens_np - 1)[:, None], ops.Params(B - 1, Hq, Hkv, topk=topk))
     o_o, lse_o = oracle.attn(op, as_u16(x.q[1:])[:, None], as_u16(x.k[1:]), as_u16(x.v[1:]), idx_gn, lens=lens_np)
     compare_attention(o_ref[1:].float().cpu().numpy(), o_o[:, 0], lse_ref[1:].cpu().numpy(), lse_o[:, :, 0])
+
+
+def test_decode_step_with_append_equals_append_then_step():
+    # the step that appends the new token itself must leave the caches, kc and the lengths
+    # as infllmv2_append_kv does, and give the outputs of a step on the appended cache;
+    # lengths cover a completed kernel (n = 32 + 16 i), a block boundary, an empty cache
+    # and a full one (left untouched, flagged)
+    Lmax, Hq, Hkv, topk = 3000, 32, 2, 16
+    lens0 = [2015, 2047, 63, 0, 31, 2999, 1000, 3000]  # cached tokens before the step
+    B = len(lens0)
+    x = inputs(B, Lmax, Hq, Hkv, seed=990, mode="decode", lens=[max(n, 1) for n in lens0])
+    p = ops.Params(B, Hq, Hkv, topk=topk)
+    g = torch.Generator().manual_seed(991)
+    k_new = torch.randn((B, Hkv, 128), generator=g).to(torch.bfloat16).cuda()
+    v_new = torch.randn((B, Hkv, 128), generator=g).to(torch.bfloat16).cuda()
+    q, k0, v0 = x.q.cuda(), x.k.cuda(), x.v.cuda()
+    l0 = torch.tensor(lens0, dtype=torch.int32).cuda()
+    kc0 = ops.compress_keys(p, k0, lens=l0)
+    # reference: the append kernel, then the step without append
+    k_a, v_a, kc_a, l_a = k0.clone(), v0.clone(), kc0.clone(), l0.clone()
+    ops.append_kv(p, k_new, v_new, k_a, v_a, l_a, kc_a)
+    o_a, lse_a, idx_a = ops.decode_step(p, q, k_a, v_a, kc_a, l_a)
+    assert ops.device_error(clear=True) != 0  # the full cache (lens 3000) was flagged
+    # the fused step with append
+    k_f, v_f, kc_f = k0.clone(), v0.clone(), kc0.clone()
+    l_out = torch.full_like(l0, -5)
+    o_f, lse_f, idx_f, l_f = ops.decode_step(p, q, k_f, v_f, kc_f, l0, k_new=k_new, v_new=v_new, lens_out=l_out)
+    torch.cuda.synchronize()
+    assert ops.device_error(clear=True) != 0
+    assert torch.equal(l_f, l_a) and torch.equal(l0.cpu(), torch.tensor(lens0, dtype=torch.int32))
+    bits = lambda t: t.view(torch.int16)  # bitwise: kc rows past a sequence's kernels are never written
+    assert torch.equal(bits(k_f), bits(k_a)) and torch.equal(bits(v_f), bits(v_a))
+    assert torch.equal(bits(kc_f), bits(kc_a))
+    assert torch.equal(idx_f, idx_a) and torch.equal(o_f, o_a) and torch.equal(lse_f, lse_a)
 
 
 # ---------------------------------------------------------- whole path, workloads

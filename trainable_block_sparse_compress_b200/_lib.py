@@ -75,7 +75,7 @@ SIGNATURES = {
                                               _vp]),
     "infllmv2_sparse_attn_decode_noalloc": (_int, [_P, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "infllmv2_append_kv": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp]),
-    "infllmv2_decode_step": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "infllmv2_decode_step": (_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp]),
     "infllmv2_workspace_size": (_sz, [_P, _int, _i32]),
     "infllmv2_check_params": (_int, [_P]),
     "infllmv2_status_string": (ctypes.c_char_p, [_int]),

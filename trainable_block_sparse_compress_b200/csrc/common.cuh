@@ -127,6 +127,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same for global memory: this thread's generic writes before later bulk-tensor
+// (async proxy) reads of them, by this or (after a barrier) another thread.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 // Programmatic dependent launch.  grid_dependency_wait() returns once every grid this
 // one depends on has completed and its memory writes are visible (at once when there is
 // none); nothing may read what an earlier kernel on the stream wrote before it.

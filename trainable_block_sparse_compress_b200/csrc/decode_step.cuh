@@ -15,9 +15,14 @@
 // being scored, and nothing round-trips through global memory between the two halves.
 // The selection's tile ring and block maxima and the attention's ring share one region of
 // shared memory: each half's data is dead before the other half writes it.
+// Optionally the step first appends the new token (the cache maintenance of
+// append_kv_kernel, same arithmetic): the CTA that scores the sequence's last kernel
+// writes the token's key and value rows and the kernel the token completes, before its
+// own Kc stream starts; the new length goes to lens_out.
 #pragma once
 #include <cooperative_groups.h>
 
+#include "append.cuh"
 #include "attn_dec.cuh"
 #include "select_decode.cuh"
 
@@ -37,7 +42,41 @@ constexpr size_t decode_step_smem_bytes() { return 1024 + kDsRegion + sizeof(DsS
 struct DecodeStepParams {
   SelDecodeParams sel;
   AttnParams attn;
+  // the token to append (nullptr: none; lens then counts the query's own token)
+  const __nv_bfloat16* k_new;  // [B, Hkv, d]
+  const __nv_bfloat16* v_new;  // [B, Hkv, d]
+  __nv_bfloat16* k_cache;      // [B, Hkv, Lmax, d]
+  __nv_bfloat16* v_cache;
+  __nv_bfloat16* kc;           // [B, Hkv, NKmax, d]
+  int32_t* lens_out;           // [B]: the new lengths
 };
+
+// Appends the token of (b, g) at position pos (< Lmax): key and value rows, and the
+// semantic kernel it completes when n = pos + 1 = 32 + 16 i -- kernel i, the mean of key
+// rows [16 i, 16 i + 32), fp64 sum rounded once (append_kv_kernel's arithmetic).  Threads
+// 0..127, thread = column d; each fences its writes for later bulk-tensor reads.
+__device__ __forceinline__ void ds_append(const DecodeStepParams& P, long long bg, int pos) {
+  const int d = threadIdx.x;
+  if (d >= kHeadDim) return;
+  const long long Lmax = P.sel.Lmax;
+  const __nv_bfloat16 kv = P.k_new[bg * kHeadDim + d];
+  P.k_cache[(bg * Lmax + pos) * kHeadDim + d] = kv;
+  P.v_cache[(bg * Lmax + pos) * kHeadDim + d] = P.v_new[bg * kHeadDim + d];
+  const int n = pos + 1;
+  if (n >= kKernel && (n - kKernel) % kStride == 0) {
+    const int ki = (n - kKernel) / kStride;
+    const __nv_bfloat16* rows = P.k_cache + (bg * Lmax + static_cast<long long>(kStride) * ki) * kHeadDim + d;
+    __nv_bfloat16 r_[kKernel - 1];
+#pragma unroll
+    for (int r = 0; r < kKernel - 1; ++r) r_[r] = rows[r * kHeadDim];
+    double sum = 0.0;
+#pragma unroll
+    for (int r = 0; r < kKernel - 1; ++r) sum += static_cast<double>(__bfloat162float(r_[r]));
+    sum += static_cast<double>(__bfloat162float(kv));  // the new row, from the input
+    P.kc[(bg * P.sel.NKmax + ki) * kHeadDim + d] = __double2bfloat16(sum * (1.0 / kKernel));
+  }
+  fence_proxy_async_global();
+}
 
 // grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.  C divides 16.
 __global__ void __launch_bounds__(kSdThreads)
@@ -67,7 +106,19 @@ __global__ void __launch_bounds__(kSdThreads)
     prefetch_tmap(&tm_v);
   }
   grid_dependency_wait();  // q, the caches, Kc and lens may come from the previous kernel
-  const SdItem it = sd_item(P.sel, C, c, bg);
+  const int b = static_cast<int>(bg / P.sel.Hkv);
+  const int Lmax = P.sel.Lmax;
+  const int raw = P.sel.lens[b];
+  const bool append = P.k_new != nullptr && raw >= 0 && raw < Lmax;
+  const int n = append ? raw + 1 : min(max(raw, 0), Lmax);
+  const SdItem it = sd_item(P.sel, C, c, bg, n);
+  if (P.k_new != nullptr) {
+    if (append && c == (it.nk > 0 ? (it.nk - 1) / it.chunk : 0)) ds_append(P, bg, raw);
+    if (c == 0 && it.g == 0 && threadIdx.x == 0) {
+      P.lens_out[b] = append ? n : raw;
+      if (!append) atomicOr(&g_device_error, kDevErrCacheFull);  // left untouched, as append_kv does
+    }
+  }
 
   // ---- selection
   sd_score_chunk(&tm_kc, P.sel, it, region, bm, D.sel);
@@ -93,13 +144,13 @@ __global__ void __launch_bounds__(kSdThreads)
   const int n_all = *cluster.map_shared_rank(&D.attn.n_blocks, 0);
   const int per = (n_all + C - 1) / C;
   const int lo = min(c * per, n_all);
-  const int n = min(lo + per, n_all) - lo;
+  const int nsh = min(lo + per, n_all) - lo;
   const int* list0 = cluster.map_shared_rank(D.attn.list, 0);
-  for (int i = threadIdx.x; i < n; i += kSdThreads) D.share[i] = list0[lo + i];
+  for (int i = threadIdx.x; i < nsh; i += kSdThreads) D.share[i] = list0[lo + i];
   fence_proxy_async_smem();  // the region's generic accesses before the ring's copies
   __syncthreads();
   const int qrow = it.b * P.attn.Hq + it.g * P.attn.G;
-  ad_partial(&tm_q, &tm_k, &tm_v, P.attn, bg, qrow, it.n - 1, D.share, n, region, qtile, D.attn);
+  ad_partial(&tm_q, &tm_k, &tm_v, P.attn, bg, qrow, it.n - 1, D.share, nsh, region, qtile, D.attn);
   ad_merge(cluster, P.attn, qrow, region, D.attn);
 }
 

@@ -98,14 +98,14 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
   return r == CUDA_SUCCESS;
 }
 
-// 3-D view [tokens, heads, 128] of the prefill queries, box {64 columns, 16 heads, 8
+// 3-D view [tokens, heads, 128] of the prefill queries, box {64 columns, G heads, 128 / G
 // tokens}: the 128 (token, head) rows of one selection tile.
-bool make_q_map_3d(CUtensorMap* m, const void* q, uint64_t tokens, uint64_t heads) {
+bool make_q_map_3d(CUtensorMap* m, const void* q, uint64_t tokens, uint64_t heads, int G) {
   if (!get_encoder()) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
                         static_cast<cuuint64_t>(tokens)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, static_cast<cuuint64_t>(heads * kHeadDim * 2)};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kGroupRows), static_cast<cuuint32_t>(kTcTokens)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -357,23 +357,39 @@ int select_prefill(const infllmv2_params* p, const void* q, int32_t Lq, const vo
   a.pool_mode = p->pool_mode;
   a.nblk_cap = nblk_cap;
   a.scale_log2 = scale_log2(p);
+  int st;
+  // tensor-core path: 128 / G tokens x G heads per 128-row UMMA tile, with a 3-slot Kc
+  // ring, or 2 slots when the block keys of long sequences need the room
+  a.stages = sel_tc_smem_bytes(nblk_cap, G, 3) <= kMaxSmem ? 3 : 2;
+  if (nk > 0 && sel_tc_smem_bytes(nblk_cap, G, a.stages) <= kMaxSmem) {
+    const int tt = sel_tc_tokens(G);
+    a.tiles_per_bg = (Lq + tt - 1) / tt;
+    const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
+    if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+    CUtensorMap tm_q3, tm_kca, tm_kcb;
+    const uint64_t kc_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk;
+    if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * Lq, p->num_q_heads, G) ||
+        !make_map(&tm_kca, kc, kc_rows, kTcN) || !make_map(&tm_kcb, kc, kc_rows, kTcNB))
+      return INFLLMV2_ERR_CUDA;
+    const size_t smem = sel_tc_smem_bytes(nblk_cap, G, a.stages);
+    auto run = [&](auto kern) -> int {
+      int r = set_smem(reinterpret_cast<const void*>(kern), smem);
+      if (r != INFLLMV2_OK) return r;
+      kern<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kca, tm_kcb, a);
+      return launch_status();
+    };
+    switch (G) {
+      case 16: return run(select_prefill_tc_kernel<16>);
+      case 8: return run(select_prefill_tc_kernel<8>);
+      case 4: return run(select_prefill_tc_kernel<4>);
+      case 2: return run(select_prefill_tc_kernel<2>);
+      default: return run(select_prefill_tc_kernel<1>);
+    }
+  }
+  // m16n8k16 path: 8 tokens per CTA, one warp per token
   a.tiles_per_bg = (Lq + kSelWarps - 1) / kSelWarps;
   const long long grid = static_cast<long long>(a.tiles_per_bg) * p->batch * p->num_kv_heads;
   if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
-  int st;
-  if (G == kGroupRows && nk > 0 && sel_tc_smem_bytes(nblk_cap) <= kMaxSmem) {
-    // tensor-core path: 8 tokens x 16 heads per 128-row UMMA tile
-    static_assert(kTcTokens == kSelWarps, "both prefill selection kernels tile 8 tokens");
-    CUtensorMap tm_q3, tm_kca, tm_kcb;
-    const uint64_t kc_rows = static_cast<uint64_t>(p->batch) * p->num_kv_heads * nk;
-    if (!make_q_map_3d(&tm_q3, q, static_cast<uint64_t>(p->batch) * Lq, p->num_q_heads) ||
-        !make_map(&tm_kca, kc, kc_rows, kTcN) || !make_map(&tm_kcb, kc, kc_rows, kTcNB))
-      return INFLLMV2_ERR_CUDA;
-    const size_t smem = sel_tc_smem_bytes(nblk_cap);
-    if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_tc_kernel), smem)) != INFLLMV2_OK) return st;
-    select_prefill_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(tm_q3, tm_kca, tm_kcb, a);
-    return launch_status();
-  }
   const size_t smem = sel_prefill_smem_bytes(nblk_cap);
   if ((st = set_smem(reinterpret_cast<const void*>(select_prefill_kernel), smem)) != INFLLMV2_OK) return st;
   select_prefill_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(tm_kc, a);
@@ -504,9 +520,10 @@ int infllmv2_compress_keys(const infllmv2_params* p, const void* k, const int32_
   const int nk = static_cast<int>(num_kernels(Lmax));
   if (nk == 0) return INFLLMV2_OK;  // kc has no rows (and may be NULL)
   if (kc == nullptr || !aligned16(kc)) return INFLLMV2_ERR_INVALID_ARG;
-  const int halfwarps = (nk + kCompressKPH - 1) / kCompressKPH;
-  dim3 grid((halfwarps + 7) / 8, p->num_kv_heads, p->batch);
-  compress_kernel<<<grid, kCompressThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  const long long grid =
+      static_cast<long long>(p->batch) * p->num_kv_heads * ((nk + kCompressKPC - 1) / kCompressKPC);
+  if (grid > 0x7fffffffLL) return INFLLMV2_ERR_UNSUPPORTED;
+  compress_kernel<<<static_cast<unsigned>(grid), kCompressThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(k), lens, Lmax, nk, p->num_kv_heads, static_cast<__nv_bfloat16*>(kc));
   return launch_status();
 }
@@ -744,9 +761,9 @@ int infllmv2_sparse_attn_decode(const infllmv2_params* p, const void* q, const v
   return launch_status();
 }
 
-int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_cache, const void* v_cache,
-                         const void* kc, const int32_t* lens, int32_t Lmax, int32_t* block_idx, void* o, float* lse,
-                         infllmv2_stream_t stream) {
+int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                         void* v_cache, void* kc, const int32_t* lens, int32_t* lens_out, int32_t Lmax,
+                         int32_t* block_idx, void* o, float* lse, infllmv2_stream_t stream) {
   int st = check_params(p);
   if (st != INFLLMV2_OK) return st;
   if ((st = check_len(Lmax)) != INFLLMV2_OK) return st;
@@ -754,6 +771,12 @@ int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(block_idx) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lens) & 3u))
     return INFLLMV2_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return INFLLMV2_ERR_INVALID_ARG;
+  if (k_new != nullptr) {  // append: the new rows, and a separate array for the new lengths
+    if (!aligned16(k_new) || !aligned16(v_new) || lens_out == nullptr || lens_out == lens ||
+        (reinterpret_cast<uintptr_t>(lens_out) & 3u) || kc == nullptr)
+      return INFLLMV2_ERR_INVALID_ARG;
+  }
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return INFLLMV2_ERR_INVALID_ARG;
   const int64_t nk = num_kernels(Lmax);
   if (nk > 0 && (kc == nullptr || !aligned16(kc))) return INFLLMV2_ERR_INVALID_ARG;
@@ -799,6 +822,12 @@ int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_
   t.lse = lse;
   t.part_o = nullptr;
   t.part_lse = nullptr;
+  P.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  P.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  P.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  P.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  P.kc = static_cast<__nv_bfloat16*>(kc);
+  P.lens_out = lens_out;
   CUtensorMap tm_kc, tq, tk, tv;
   std::memset(&tm_kc, 0, sizeof tm_kc);
   const uint64_t q_rows = static_cast<uint64_t>(p->batch) * p->num_q_heads;

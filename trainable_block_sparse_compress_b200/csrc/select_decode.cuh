@@ -99,15 +99,15 @@ struct SdItem {
   int k0, ntiles;  // this CTA's first kernel and Kc tiles
 };
 
-// Reads lens: call after grid_dependency_wait().
-__device__ __forceinline__ SdItem sd_item(const SelDecodeParams& p, int C, int c, long long bg) {
+// n: the sequence's length, clamped to [0, Lmax] by the caller.
+__device__ __forceinline__ SdItem sd_item(const SelDecodeParams& p, int C, int c, long long bg, int n) {
   SdItem it;
   it.C = C;
   it.c = c;
   it.bg = bg;
   it.b = static_cast<int>(bg / p.Hkv);
   it.g = static_cast<int>(bg % p.Hkv);
-  it.n = min(max(p.lens[it.b], 0), p.Lmax);
+  it.n = n;
   it.nk = it.n >= kKernel ? (it.n - kKernel) / kStride + 1 : 0;
   it.cur = it.n > 0 ? (it.n - 1) / kBlock : -1;
   it.chunk = ((it.nk + C - 1) / C + kKcTile - 1) / kKcTile * kKcTile;
@@ -194,9 +194,13 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     // higher < need <= higher + own
     const int need = want - above;
     const int b0 = tid * kSdBinsPerThread;
+    int hv[kSdBinsPerThread];
     int own = 0;
 #pragma unroll
-    for (int e = 0; e < kSdBinsPerThread; ++e) own += b0 + e < nb ? static_cast<int>(hist[b0 + e]) : 0;
+    for (int e = 0; e < kSdBinsPerThread; ++e) {
+      hv[e] = b0 + e < nb ? static_cast<int>(hist[b0 + e]) : 0;
+      own += hv[e];
+    }
     int incl = own;  // this lane's and the higher lanes' bins
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -209,20 +213,19 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
 #pragma unroll
     for (int ww = 0; ww < kSdWarps; ++ww) higher += ww > warp ? S.wsum[ww] : 0;
     if (higher < need && need <= higher + own) {
-      int acc = higher;
-#pragma unroll 1
+      int acc = higher, found = -1, fa = 0, fi = 0;
+#pragma unroll
       for (int e = kSdBinsPerThread - 1; e >= 0; --e) {
-        const int bin = b0 + e;
-        if (bin >= nb) continue;
-        const int h = static_cast<int>(hist[bin]);
-        if (acc + h >= need) {
-          S.dig = bin;
-          S.dig_above = acc;
-          S.dig_in = h;
-          break;
+        if (found < 0 && acc + hv[e] >= need) {
+          found = b0 + e;
+          fa = acc;
+          fi = hv[e];
         }
-        acc += h;
+        acc += hv[e];
       }
+      S.dig = found;
+      S.dig_above = fa;
+      S.dig_in = fi;
     }
     __syncthreads();
     T |= static_cast<uint32_t>(S.dig) << shift;
@@ -249,10 +252,11 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   const int nl = S.nlist;  // == inb
   const uint32_t x = lane < nl ? S.list[lane] : 0u;
   int gt = 0, ge = 0;
-  for (int i = 0; i < nl; ++i) {
-    const uint32_t v = S.list[i];
-    gt += v > x ? 1 : 0;
-    ge += v >= x ? 1 : 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t v = __shfl_sync(0xffffffffu, x, i);
+    gt += (i < nl && v > x) ? 1 : 0;
+    ge += (i < nl && v >= x) ? 1 : 0;
   }
   const int rank = want - above;
   const unsigned hit = __ballot_sync(0xffffffffu, lane < nl && gt < rank && rank <= ge);
@@ -592,7 +596,8 @@ __global__ void __launch_bounds__(kSdThreads)
   const int c = static_cast<int>(cluster.block_rank());
   allow_dependent_launch();  // the decode attention may set up while this selection runs
   grid_dependency_wait();    // q, Kc and lens may come from the previous kernel
-  const SdItem it = sd_item(p, C, c, blockIdx.x / C);  // clusters are consecutive blocks
+  const long long bg = blockIdx.x / C;  // clusters are consecutive blocks
+  const SdItem it = sd_item(p, C, c, bg, min(max(p.lens[bg / p.Hkv], 0), p.Lmax));
   sd_score_chunk(&tm_kc, p, it, ring, bm, S);
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
   sd_block_keys(cluster, p, it, reinterpret_cast<uint32_t*>(ring + kSdKeysOff), bm, S);

@@ -37,7 +37,8 @@ struct SelPrefillParams {
   int score_mode, pool_mode;  // kScore*, kPool*
   int nblk_cap;  // score slots per token (>= number of blocks in Lmax tokens, multiple of 32)
   float scale_log2;
-  int tiles_per_bg;  // ceil(Lq / 8)
+  int tiles_per_bg;  // ceil(Lq / query rows per CTA)
+  int stages;        // tensor-core kernel: Kc ring slots (2 or 3)
 };
 
 struct SelSmem {

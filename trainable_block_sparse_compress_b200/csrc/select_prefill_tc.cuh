@@ -6,21 +6,23 @@
 // block, sum over the group's heads, top-k with forced initial/local blocks (and the
 // same variants: logit-sum scoring without pass A, inside pooling).
 //
-// One CTA = 8 consecutive query rows of one (sequence, kv-head): 8 x 16 heads = the 128
-// rows (M) of a UMMA tile.  A chunk's rows are the last q_len tokens of a cache of kv_len
-// tokens (a fresh prefill: q_len = kv_len = L).  Warp roles (448 threads):
+// One CTA = 128 / G consecutive query rows of one (sequence, kv-head) with the G heads
+// of its group each: the 128 rows (M) of a UMMA tile, row = token * G + head.  A chunk's
+// rows are the last q_len tokens of a cache of kv_len tokens (a fresh prefill: q_len =
+// kv_len = L).  Warp roles (448 threads):
 //   warp 12 TMA: the 128 x 128 query tile once (3-D map: token, head, dim), then Kc tiles
-//           through a 3-stage ring: pass A tiles of 128 kernels, pass B tiles of 144
-//           kernels that start 16 kernels early, so each pass-B tile also holds the
-//           kernel straddling its first block (4j - 1) and is self-contained;
+//           through a ring of 3 slots (2 when the block keys of long sequences need the
+//           room): pass A tiles of 128 kernels, pass B tiles of 144 kernels that start
+//           16 kernels early, so each pass-B tile also holds the kernel straddling its
+//           first block (4j - 1) and is self-contained;
 //   warp 13 allocates TMEM and, from one thread, issues per tile 8 UMMAs (M128 x N128 or
 //           N144, K16, bf16 -> fp32) into one of three TMEM accumulators;
 //   warps 0-11 three epilogue warpgroups taking every third tile; thread (w, lane) owns TMEM
 //           lane 32 (w % 4) + lane = row (token, head).  Pass A keeps an online
 //           log-sum-exp per row (the warpgroups' partials are merged once); pass B
-//           pools block maxima along the row, forms p = exp(m - lse) and sums the 16
-//           heads of a token with a 16-lane transpose-reduce; block keys go to shared
-//           memory; finally warp w < 8 selects the top blocks of token w.
+//           pools block maxima along the row, forms p = exp(m - lse) and sums the G
+//           heads of a token with a G-lane transpose-reduce; block keys go to shared
+//           memory; finally warp w selects the top blocks of tokens w, w + 12, ...
 #pragma once
 #include "common.cuh"
 #include "select_prefill.cuh"
@@ -29,7 +31,7 @@
 
 namespace infllmv2 {
 
-constexpr int kTcTokens = 8;
+constexpr int kTcTokens = 8;           // query rows per CTA at G = 16 (128 / G in general)
 constexpr int kTcN = 128;              // kernels per pass-A tile
 constexpr int kTcOverlap = 16;         // extra leading kernels of a pass-B tile
 constexpr int kTcNB = kTcN + kTcOverlap;  // 144 kernels per pass-B tile
@@ -51,75 +53,63 @@ struct SelTcSmem {
   volatile int abort;
 };
 
-inline size_t sel_tc_smem_bytes(int nblk_cap) {
-  return 1024 + kTcQBytes + static_cast<size_t>(kTcStages) * kTcStageBytes +
-         static_cast<size_t>(kTcTokens) * nblk_cap * 4 + kTcTokens * 256 * 4 + sizeof(SelTcSmem);
+// Query rows per CTA and warps that run a top-k, for a group of G heads.
+inline int sel_tc_tokens(int G) { return 128 / G; }
+inline int sel_tc_topk_warps(int G) { return sel_tc_tokens(G) < kTcEpiWarps ? sel_tc_tokens(G) : kTcEpiWarps; }
+
+inline size_t sel_tc_smem_bytes(int nblk_cap, int G, int stages) {
+  return 1024 + kTcQBytes + static_cast<size_t>(stages) * kTcStageBytes +
+         static_cast<size_t>(sel_tc_tokens(G)) * nblk_cap * 4 + static_cast<size_t>(sel_tc_topk_warps(G)) * 256 * 4 +
+         sizeof(SelTcSmem);
 }
 
-// Sum of v over the 16 lanes that share lane bit 4 (one token's heads), scattered: lane
-// L (mod 16) returns the total of entry L.  15 shuffles.
-__device__ __forceinline__ float reduce_scatter16(const float (&v)[16]) {
+// Sum of v over the kG lanes that hold one token's heads (lanes sharing lane / kG),
+// scattered: lane L returns in v[r], r < 16 / kG, the total of entry (L % kG) * (16 / kG) + r.
+// log2(kG) halving steps of one shuffle per kept value (15 shuffles at kG = 16).
+template <int kG>
+__device__ __forceinline__ void reduce_scatter_group(float (&v)[16]) {
   const int lane = threadIdx.x & 31;
-  float a[8];
-  {
-    const bool up = lane & 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float send = up ? v[i] : v[i + 8];
-      const float keep = up ? v[i + 8] : v[i];
-      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  for (int m = kG / 2; m >= 1; m >>= 1) {
+    const int h = 16 * m / kG;  // values kept after this step
+    const bool up = lane & m;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = up ? v[i] : v[i + h];
+      const float keep = up ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
     }
   }
-  float b4[4];
-  {
-    const bool up = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float send = up ? a[i] : a[i + 4];
-      const float keep = up ? a[i + 4] : a[i];
-      b4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-  }
-  float c2[2];
-  {
-    const bool up = lane & 2;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float send = up ? b4[i] : b4[i + 2];
-      const float keep = up ? b4[i + 2] : b4[i];
-      c2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-  }
-  const bool up = lane & 1;
-  const float send = up ? c2[0] : c2[1];
-  const float keep = up ? c2[1] : c2[0];
-  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
 __device__ __forceinline__ float max4(float a, float b, float c, float d) { return fmaxf(fmaxf(a, b), fmaxf(c, d)); }
 
-// grid = B * Hkv * ceil(Lq / 8) (latest tiles first), block = 448.  Requires G == 16.
+// grid = B * Hkv * ceil(Lq / (128 / kG)) (latest tiles first), block = 448.  p.G == kG.
+template <int kG>
 __global__ void __launch_bounds__(kTcThreads, 1)
     select_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q3, const __grid_constant__ CUtensorMap tm_kca,
                              const __grid_constant__ CUtensorMap tm_kcb, const SelPrefillParams p) {
+  constexpr int kTT = 128 / kG;                                     // query rows per CTA
+  constexpr int kTopkWarps = kTT < kTcEpiWarps ? kTT : kTcEpiWarps;  // warps that run a top-k
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = align_smem(smem_raw, 1024);
   unsigned char* qs = base;
   unsigned char* ring = qs + kTcQBytes;
-  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + kTcStages * kTcStageBytes);
-  uint32_t* hist_all = keys_all + kTcTokens * p.nblk_cap;
-  SelTcSmem& S = *reinterpret_cast<SelTcSmem*>(hist_all + kTcTokens * 256);
+  const int NS = p.stages;  // Kc ring slots
+  uint32_t* keys_all = reinterpret_cast<uint32_t*>(ring + NS * kTcStageBytes);
+  uint32_t* hist_all = keys_all + kTT * p.nblk_cap;
+  SelTcSmem& S = *reinterpret_cast<SelTcSmem*>(hist_all + kTopkWarps * 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long nbg = static_cast<long long>(p.B) * p.Hkv;
   const int tile = p.tiles_per_bg - 1 - static_cast<int>(blockIdx.x / nbg);
   const long long bg = blockIdx.x % nbg;
   const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int t0 = tile * kTcTokens;  // first query row of the tile
+  const int t0 = tile * kTT;  // first query row of the tile
   const ChunkLens cl = chunk_lens(p.q_lens, p.kv_lens, b, p.Lq, p.Lmax);
   if (t0 >= cl.q_len) return;  // padding rows only (uniform over the CTA, before any set-up)
   const int off = cl.kv_len - cl.q_len;  // position of query row 0
-  const int imax_last = last_visible_kernel(off + min(t0 + kTcTokens - 1, cl.q_len - 1));
+  const int imax_last = last_visible_kernel(off + min(t0 + kTT - 1, cl.q_len - 1));
   // pass A (the per-head lse) only for softmax-sum scoring
   const int TA = (imax_last >= 0 && p.score_mode == kScoreSoftmaxSum) ? imax_last / kTcN + 1 : 0;
   const int TB = imax_last >= 0 ? (imax_last + 1) / kTcN + 1 : 0;
@@ -127,7 +117,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&S.qbar, 1);
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
     }
@@ -155,12 +145,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       prefetch_tmap(&tm_kca);
       prefetch_tmap(&tm_kcb);
       mbar_arrive_expect_tx(&S.qbar, kTcQBytes);
-      tma_load_3d(qs, &tm_q3, &S.qbar, 0, g * kGroupRows, b * p.Lq + t0);
-      tma_load_3d(qs + kTcQBytes / 2, &tm_q3, &S.qbar, 64, g * kGroupRows, b * p.Lq + t0);
+      tma_load_3d(qs, &tm_q3, &S.qbar, 0, g * kG, b * p.Lq + t0);
+      tma_load_3d(qs + kTcQBytes / 2, &tm_q3, &S.qbar, 64, g * kG, b * p.Lq + t0);
       const int row0 = static_cast<int>(bg * p.NKmax);
+      int st = 0;        // ring slot of tile n (n % NS, kept incrementally: NS is a runtime value)
+      uint32_t ph = 0u;  // parity of (n / NS)
       for (int n = 0; n < T; ++n) {
-        const int st = n % kTcStages, u = n / kTcStages;
-        if (u > 0) mbar_wait(&S.empty[st], (u - 1) & 1, &S.abort);
+        if (n >= NS) mbar_wait(&S.empty[st], ph ^ 1u, &S.abort);
         if (S.abort) break;
         unsigned char* dst = ring + st * kTcStageBytes;
         if (n < TA) {
@@ -174,6 +165,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_load_2d(dst, &tm_kcb, &S.full[st], 0, r);
           tma_load_2d(dst + kTcHalfBytes, &tm_kcb, &S.full[st], 64, r);
         }
+        if (++st == NS) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
     }
     return;
@@ -186,9 +181,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t idesc_b = idesc_bf16_f32(128, kTcNB, false, false);
       mbar_wait(&S.qbar, 0, &S.abort);
       const uint32_t qa = smem_u32(qs);
+      int st = 0;        // ring slot of tile n, as in the TMA warp
+      uint32_t ph = 0u;
       for (int n = 0; n < T; ++n) {
-        const int st = n % kTcStages, acc = n % kTcEpiWGs, u = n / kTcEpiWGs;
-        mbar_wait(&S.full[st], (n / kTcStages) & 1, &S.abort);
+        const int acc = n % kTcEpiWGs, u = n / kTcEpiWGs;
+        mbar_wait(&S.full[st], ph, &S.abort);
         if (u > 0) mbar_wait(&S.tempty[acc], (u - 1) & 1, &S.abort);
         tc_fence_after();
         const uint32_t kb = smem_u32(ring + st * kTcStageBytes);
@@ -202,6 +199,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         umma_commit(&S.empty[st]);
         umma_commit(&S.tfull[acc]);
+        if (++st == NS) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
       umma_commit(&S.mma_done);
     }
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int wg = warp >> 2;   // warpgroup: takes tiles n with n % kTcEpiWGs == wg
   const int wq = warp & 3;    // TMEM lane quarter
   const int row = 32 * wq + lane;
-  const int tok = row >> 4;
+  const int tok = row / kG;
   const int t = off + min(t0 + tok, cl.q_len - 1);  // position; rows past q_len compute, write nothing
   const int imax = last_visible_kernel(t);
   const int cur = t / kBlock;
@@ -264,10 +265,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.tempty[acc]);
   }
-  // zero the key row of token `warp` (blocks 0..cur) while the warpgroups meet
-  if (warp < kTcTokens) {
-    const int tz = off + min(t0 + warp, cl.q_len - 1);
-    uint32_t* kz = keys_all + warp * p.nblk_cap;
+  // zero the key rows of tokens warp, warp + 12, ... (blocks 0..cur) while the warpgroups meet
+  for (int tw = warp; tw < kTT; tw += kTcEpiWarps) {
+    const int tz = off + min(t0 + tw, cl.q_len - 1);
+    uint32_t* kz = keys_all + tw * p.nblk_cap;
     for (int j = lane; j <= tz / kBlock; j += 32) kz[j] = 0u;
   }
   S.part[wg][row] = make_float2(m, l);
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // pass B: block maxima along the row, p = exp(m - lse) (or m itself for logit-sum
-  // scoring), group sum over the 16 heads
+  // scoring), group sum over the G heads
   const bool inside = p.pool_mode == kPoolInside, logit = p.score_mode == kScoreLogitSum;
   uint32_t* keys = keys_all + tok * p.nblk_cap;
   int nb = TA;
@@ -327,12 +328,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           carry = x[4 * gq + 3];
         }
       }
-      const float sum = reduce_scatter16(pb);
-      const int j = 32 * c + 16 * half + (lane & 15);
-      if (j <= cur) {
-        const bool eligible = block_eligible(j, imax, p.pool_mode);
-        const bool forced = j < p.n_init || j > cur - p.n_local;
-        keys[j] = (eligible && !forced) ? score_key(sum, p.score_mode) : 0u;
+      reduce_scatter_group<kG>(pb);
+#pragma unroll
+      for (int r = 0; r < 16 / kG; ++r) {
+        const int j = 32 * c + 16 * half + (lane % kG) * (16 / kG) + r;
+        if (j <= cur) {
+          const bool eligible = block_eligible(j, imax, p.pool_mode);
+          const bool forced = j < p.n_init || j > cur - p.n_local;
+          keys[j] = (eligible && !forced) ? score_key(pb[r], p.score_mode) : 0u;
+        }
       }
     }
     tc_fence_before();
@@ -343,18 +347,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   named_bar_sync(1, 32 * (kTcEpiWarps + 1));  // TMEM no longer read: the MMA warp may free it
   named_bar_sync(2, 32 * kTcEpiWarps);        // all keys written
 
-  // top-k of token `warp`
-  const int tr = t0 + warp;  // query row
-  if (warp < kTcTokens && tr < cl.q_len) {
-    const int cu = (off + tr) / kBlock;
-    const uint32_t* kt = keys_all + warp * p.nblk_cap;
-    const int want = p.topk - forced_count(cu, p.n_init, p.n_local);
-    int32_t* out = p.idx + ((bg * p.Lq + tr) * static_cast<long long>(p.topk));
-    if (cu + 1 <= 32 * kTopkRegKeys) {
-      warp_topk_select(kt, cu + 1, want, cu, p.n_init, p.n_local, p.topk, hist_all + warp * 256, out);
-    } else {
-      const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + warp * 256);
-      warp_emit_selection(kt, cu + 1, th, cu, p.n_init, p.n_local, p.topk, out);
+  // top-k of tokens warp, warp + 12, ...
+  if (warp < kTopkWarps) {
+    for (int tw = warp; tw < kTT; tw += kTopkWarps) {
+      const int tr = t0 + tw;  // query row
+      if (tr >= cl.q_len) break;
+      const int cu = (off + tr) / kBlock;
+      const uint32_t* kt = keys_all + tw * p.nblk_cap;
+      const int want = p.topk - forced_count(cu, p.n_init, p.n_local);
+      int32_t* out = p.idx + ((bg * p.Lq + tr) * static_cast<long long>(p.topk));
+      if (cu + 1 <= 32 * kTopkRegKeys) {
+        warp_topk_select(kt, cu + 1, want, cu, p.n_init, p.n_local, p.topk, hist_all + warp * 256, out);
+      } else {
+        const TopkThreshold th = warp_radix_threshold(kt, cu + 1, want, hist_all + warp * 256);
+        warp_emit_selection(kt, cu + 1, th, cu, p.n_init, p.n_local, p.topk, out);
+      }
+      __syncwarp();
     }
   }
 }

@@ -329,16 +329,29 @@ def prefill_chunk(p: Params, q, k_cache, v_cache, kc, q_lens=None, kv_lens=None)
 
 
 def decode_step(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, kc: torch.Tensor,
-                lens: torch.Tensor, block_idx: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                lse: Optional[torch.Tensor] = None, want_lse: bool = True):
-    """One decode step in one launch: block selection for the query at lens[b]-1, then
-    sparse attention over the selected blocks.  Returns (o, lse, block_idx)."""
+                lens: torch.Tensor, k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                lens_out: Optional[torch.Tensor] = None, block_idx: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True):
+    """One decode step in one launch.  With k_new / v_new [B, Hkv, d]: the new token is
+    appended at lens[b] (caches and kc updated in place) and lens_out[b] = lens[b] + 1
+    (lens_out allocated when None); without: the query sits at lens[b]-1.  Then block
+    selection and sparse attention over the selected blocks.  Returns (o, lse, block_idx)
+    and, when appending, lens_out as a fourth element."""
     Lmax = k_cache.shape[2]
     _need(q, "q", torch.bfloat16, (p.batch, p.num_q_heads, p.head_dim))
     _need(k_cache, "k_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
     _need(v_cache, "v_cache", torch.bfloat16, (p.batch, p.num_kv_heads, Lmax, p.head_dim))
     _need(kc, "kc", torch.bfloat16, (p.batch, p.num_kv_heads, num_kernels(p, Lmax), p.head_dim))
     _need(lens, "lens", torch.int32, (p.batch,))
+    appending = k_new is not None or v_new is not None
+    if appending:
+        _need(k_new, "k_new", torch.bfloat16, (p.batch, p.num_kv_heads, p.head_dim))
+        _need(v_new, "v_new", torch.bfloat16, (p.batch, p.num_kv_heads, p.head_dim))
+        if lens_out is None:
+            lens_out = torch.empty_like(lens)
+        _need(lens_out, "lens_out", torch.int32, (p.batch,))
+        if lens_out.data_ptr() == lens.data_ptr():
+            raise ValueError("lens_out must not be lens")
     if block_idx is None:
         block_idx = torch.empty((p.batch, p.num_kv_heads, 1, p.topk), dtype=torch.int32, device=q.device)
     _need(block_idx, "block_idx", torch.int32, (p.batch, p.num_kv_heads, 1, p.topk))
@@ -349,9 +362,12 @@ def decode_step(p: Params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         lse = torch.empty((p.batch, p.num_q_heads), dtype=torch.float32, device=q.device)
     if lse is not None:
         _need(lse, "lse", torch.float32, (p.batch, p.num_q_heads))
-    st = _lib.load().infllmv2_decode_step(ctypes.byref(p.c()), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kc),
-                                          _ptr(lens), Lmax, _ptr(block_idx), _ptr(out), _ptr(lse), _stream())
+    st = _lib.load().infllmv2_decode_step(ctypes.byref(p.c()), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                          _ptr(v_cache), _ptr(kc), _ptr(lens), _ptr(lens_out), Lmax, _ptr(block_idx),
+                                          _ptr(out), _ptr(lse), _stream())
     _lib.check("infllmv2_decode_step", st)
+    if appending:
+        return out, lse, block_idx, lens_out
     return out, lse, block_idx
 
 
