@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kSdThreads)
   // ---- selection
   sd_score_chunk(&tm_kc, P.sel, it, region, bm, D.sel);
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
-  sd_block_keys(cluster, P.sel, it, reinterpret_cast<uint32_t*>(region + kSdKeysOff), bm, D.sel);
+  sd_block_keys(cluster, P.sel, it, region, bm, D.sel);
   cluster.sync();  // CTA 0 holds every key
   if (c == 0) {
     sd_select(P.sel, it, region, D.attn.list, D.sel);

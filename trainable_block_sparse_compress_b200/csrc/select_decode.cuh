@@ -72,7 +72,8 @@ struct SdSmem {
   float pm[kSdMaxCluster][kGroupRows], pl[kSdMaxCluster][kGroupRows];  // every CTA's, gathered
   float lse2[kGroupRows];  // log2-sum-exp2 per head over the whole sequence
   float carry[kGroupRows];  // previous CTA's last kernel, for this CTA's first block
-  int wred[3][kSdWarps];               // per-warp candidates, AND, OR of the keys
+  int kcnt;                            // CTA 0: candidates among the keys, and the AND / OR of
+  unsigned int kand, kor;              // their keys (every CTA adds its blocks' through DSMEM)
   int wsum[kSdWarps];                  // per-warp histogram totals of the digit search
   int dig, dig_above, dig_in;          // the digit found, keys above its bin, keys in it
   int wc[kSdMaxR][kSdWarps];          // per (slot, warp) counts of the emission
@@ -118,9 +119,9 @@ __device__ __forceinline__ SdItem sd_item(const SelDecodeParams& p, int C, int c
 }
 
 // k-th largest of the n keys in shared memory (0: not a candidate) by all kSdThreads
-// threads; same result as warp_radix_threshold.  One pass counts the candidates and
-// takes the AND and OR of their keys: the bits above the highest bit where they differ
-// are common to all of them.  Below it the threshold is resolved in digits of up to
+// threads; same result as warp_radix_threshold.  The candidates' count and the AND and OR
+// of their keys (S.kcnt, S.kand, S.kor) arrive with the keys: the bits above the highest
+// bit where the candidates differ are common to all of them.  Below it the threshold is resolved in digits of up to
 // kSdHistBits bits: a shared-memory histogram of the digit over the keys of the current
 // bucket (keys that agree with the threshold on every bit above the digit), then a
 // suffix scan over the bins finds the digit whose bin holds the (want - above)-th
@@ -135,34 +136,8 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
     r.ties = 0;
     return r;
   }
-  int cnt = 0;
-  uint32_t kand = 0xffffffffu, kor = 0u;
-  for (int j = tid; j < n; j += kSdThreads) {
-    const uint32_t k = keys[j];
-    if (k != 0u) {
-      ++cnt;
-      kand &= k;
-      kor |= k;
-    }
-  }
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
-  kand = __reduce_and_sync(0xffffffffu, kand);
-  kor = __reduce_or_sync(0xffffffffu, kor);
-  if (lane == 0) {
-    S.wred[0][warp] = cnt;
-    S.wred[1][warp] = static_cast<int>(kand);
-    S.wred[2][warp] = static_cast<int>(kor);
-  }
-  __syncthreads();
-  cnt = 0;
-  kand = 0xffffffffu;
-  kor = 0u;
-#pragma unroll
-  for (int w = 0; w < kSdWarps; ++w) {
-    cnt += S.wred[0][w];
-    kand &= static_cast<uint32_t>(S.wred[1][w]);
-    kor |= static_cast<uint32_t>(S.wred[2][w]);
-  }
+  const int cnt = S.kcnt;  // gathered while the keys were stored (sd_block_keys)
+  const uint32_t kand = S.kand, kor = S.kor;
   if (cnt <= want) {  // at most `want` candidates: take them all
     r.key = 0;
     r.ties = 0;
@@ -177,12 +152,14 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
   uint32_t T = top == 31 ? 0u : (kand >> (top + 1)) << (top + 1);  // the common bits above it
   int above = 0;                      // candidates above the current bucket
   int shift = 0, inb = 0;
-  for (;;) {
+  for (int round = 0;; ++round) {
     const int w = min(kSdHistBits, top + 1);
     shift = top + 1 - w;
     const int nb = 1 << w;
-    for (int i = tid; i < nb; i += kSdThreads) hist[i] = 0u;
-    __syncthreads();
+    if (round > 0) {  // the first round's bins were zeroed while the keys were stored
+      for (int i = tid; i < nb; i += kSdThreads) hist[i] = 0u;
+      __syncthreads();
+    }
     for (int j = tid; j < n; j += kSdThreads) {
       const uint32_t k = keys[j];
       const bool in = k != 0u && (top == 31 || (k >> (top + 1)) == (T >> (top + 1)));
@@ -376,6 +353,9 @@ __device__ __forceinline__ void sd_score_chunk(const CUtensorMap* tm_kc, const S
       mbar_init(&S.empty[s], kSdConsumers);
     }
     S.abort = 0;
+    S.kcnt = 0;  // CTA 0's are filled by every CTA of the cluster after the next cluster barrier
+    S.kand = 0xffffffffu;
+    S.kor = 0u;
     fence_mbar_init();
   }
   // bm[h][q]: max over this CTA's kernels 4q-1 .. 4q+3 (local numbering); q = nq holds
@@ -513,9 +493,17 @@ __device__ __forceinline__ void sd_score_chunk(const CUtensorMap* tm_kc, const S
 
 // Phase 2, after a cluster barrier that follows phase 1 in every CTA: the log-sum-exp per
 // head from every CTA's state, the previous CTA's carry, and the keys of this CTA's blocks
-// stored into CTA 0's key array (`keys` is this CTA's own scratch address of that array).
+// stored into CTA 0's key array (`scratch` is this CTA's own address of the selection
+// scratch), with their candidate count, AND and OR added into CTA 0's; CTA 0 also zeroes
+// the first digit histogram of its threshold search.
 __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group& cluster, const SelDecodeParams& p,
-                                              const SdItem& it, uint32_t* keys, const uint32_t* bm, SdSmem& S) {
+                                              const SdItem& it, unsigned char* scratch, const uint32_t* bm,
+                                              SdSmem& S) {
+  uint32_t* keys = reinterpret_cast<uint32_t*>(scratch + kSdKeysOff);
+  if (it.c == 0) {
+    uint32_t* hist = reinterpret_cast<uint32_t*>(scratch + kSdHistOff);
+    for (int i = threadIdx.x; i < kSdHistBins; i += kSdThreads) hist[i] = 0u;
+  }
   const int C = it.C, c = it.c, nq = it.nq, cur = it.cur;
   // gather every CTA's (max, sum) and the previous CTA's carry, all loads in flight at once
   for (int e = threadIdx.x; e < kGroupRows * C; e += kSdThreads) {
@@ -547,6 +535,8 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
   uint32_t* keys0 = cluster.map_shared_rank(keys, 0);
   const int jb0 = c * nq;
   const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
+  int cnt = 0;
+  uint32_t kand = 0xffffffffu, kor = 0u;
   for (int j = jb0 + threadIdx.x; j < jb1; j += kSdThreads) {
     const int ql = j - jb0;  // <= nq, since cur + 1 <= ceil(nk / 4) + 1 <= C nq + 1
     const bool eligible = block_eligible(j, it.nk - 1, p.pool_mode);
@@ -562,6 +552,19 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
       key = score_key(sc, p.score_mode);
     }
     keys0[j] = key;
+    if (key != 0u) {
+      ++cnt;
+      kand &= key;
+      kor |= key;
+    }
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  kand = __reduce_and_sync(0xffffffffu, kand);
+  kor = __reduce_or_sync(0xffffffffu, kor);
+  if ((threadIdx.x & 31) == 0 && cnt > 0) {
+    atomicAdd(cluster.map_shared_rank(&S.kcnt, 0), cnt);
+    atomicAnd(cluster.map_shared_rank(&S.kand, 0), kand);
+    atomicOr(cluster.map_shared_rank(&S.kor, 0), kor);
   }
 }
 
@@ -600,7 +603,7 @@ __global__ void __launch_bounds__(kSdThreads)
   const SdItem it = sd_item(p, C, c, bg, min(max(p.lens[bg / p.Hkv], 0), p.Lmax));
   sd_score_chunk(&tm_kc, p, it, ring, bm, S);
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
-  sd_block_keys(cluster, p, it, reinterpret_cast<uint32_t*>(ring + kSdKeysOff), bm, S);
+  sd_block_keys(cluster, p, it, ring, bm, S);
   cluster.sync();  // CTA 0 holds every key; no CTA reads a peer's shared memory after this
   if (c != 0) return;
   sd_select(p, it, ring, p.idx + it.bg * p.topk, S);
