@@ -210,19 +210,45 @@ __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, in
     th.key = 0xffffffffu;
     th.ties = 0;
   } else {
-    // per-lane top 4 and candidate count in one pass
+    // per-lane top 4 and candidate count in one pass: four independent insertion chains
+    // (keys i % 4), merged at the end
     const int r = (want + 31) / 32;
-    uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
-    int c1 = 0;
+    uint32_t tt[4][4];
+    int cc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tt[c][0] = tt[c][1] = tt[c][2] = tt[c][3] = 0u;
 #pragma unroll
     for (int i = 0; i < kTopkRegKeys; ++i) {
+      const int c = i & 3;
       uint32_t x = kr[i], y;
-      c1 += x != 0u ? 1 : 0;
-      y = max(x, t0); x = min(x, t0); t0 = y;
-      y = max(x, t1); x = min(x, t1); t1 = y;
-      y = max(x, t2); x = min(x, t2); t2 = y;
-      t3 = max(x, t3);
+      cc[c] += x != 0u ? 1 : 0;
+      y = max(x, tt[c][0]); x = min(x, tt[c][0]); tt[c][0] = y;
+      y = max(x, tt[c][1]); x = min(x, tt[c][1]); tt[c][1] = y;
+      y = max(x, tt[c][2]); x = min(x, tt[c][2]); tt[c][2] = y;
+      tt[c][3] = max(x, tt[c][3]);
     }
+    // top 4 of two descending 4-lists: the elementwise max of one list and the other
+    // reversed is a bitonic sequence holding the 4 largest; two exchange steps sort it
+    auto merge4 = [](const uint32_t (&a)[4], const uint32_t (&b)[4], uint32_t (&o)[4]) {
+      uint32_t m0 = max(a[0], b[3]), m1 = max(a[1], b[2]), m2 = max(a[2], b[1]), m3 = max(a[3], b[0]);
+      uint32_t x = max(m0, m2), y = min(m0, m2);
+      m0 = x;
+      m2 = y;
+      x = max(m1, m3);
+      y = min(m1, m3);
+      m1 = x;
+      m3 = y;
+      o[0] = max(m0, m1);
+      o[1] = min(m0, m1);
+      o[2] = max(m2, m3);
+      o[3] = min(m2, m3);
+    };
+    uint32_t ua[4], ub[4], tf[4];
+    merge4(tt[0], tt[1], ua);
+    merge4(tt[2], tt[3], ub);
+    merge4(ua, ub, tf);
+    const uint32_t t0 = tf[0], t1 = tf[1], t2 = tf[2], t3 = tf[3];
+    const int c1 = (cc[0] + cc[1]) + (cc[2] + cc[3]);
     const int ncand = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c1)));
     if (ncand <= want) {  // at most `want` candidates: take them all
       th.key = 0;
@@ -274,9 +300,13 @@ __device__ __forceinline__ void warp_topk_select(const uint32_t* keys, int n, in
         th.ties = want - above;
         th.all_ties = above + eq == want;
       } else {
-        uint32_t T = 0;
+        // bisection between the bound c0 <= T and the largest key: the bits above their
+        // highest differing bit are T's too
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, t0);
+        const int top = (kmax ^ c0) == 0u ? -1 : 31 - __clz(kmax ^ c0);
+        uint32_t T = top >= 31 ? 0u : (kmax >> (top + 1)) << (top + 1);
 #pragma unroll 1
-        for (int bit = 31; bit >= 0; --bit) {
+        for (int bit = top; bit >= 0; --bit) {
           const uint32_t c = T | (1u << bit);
           if (warp_count_ge_regs(kr, c) >= want) T = c;
         }
