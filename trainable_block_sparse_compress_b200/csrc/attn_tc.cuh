@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     uint32_t gpair = 0;
     int it = 0;
+    const uint64_t qpol = l2_policy_evict_first();  // queries are read once: K/V keep L2
     long long k_last[kAtKStages];  // last pair loaded into each K stage (lane 0), for the drain
     int q_last[2] = {-1, -1};      // last use of each query-tile slot
     for (int st = 0; st < kAtKStages; ++st) k_last[st] = -1;
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       int count = 0, tail = -1;
       for (int e0 = 0; e0 < p.topk; e0 += 32) {
         const int e = e0 + lane;
-        const int j = (e < p.topk && a.valid) ? row[e] : -1;
+        const int j = (e < p.topk && a.valid) ? __ldcs(row + e) : -1;
         const bool ok = j >= 0 && j <= cur;
         const unsigned msk = __ballot_sync(0xffffffffu, ok);
         const int pos = count + __popc(msk & ((1u << lane) - 1u));
@@ -223,8 +224,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         unsigned char* qs = qtiles + slot * kQTileBytes;
         if (!S.abort) {
           mbar_arrive_expect_tx(&S.q_full[slot], kQTileBytes);
-          tma_load_2d(qs, &tm_q, &S.q_full[slot], 0, a.qrow);
-          tma_load_2d(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow);
+          tma_load_2d_hint(qs, &tm_q, &S.q_full[slot], 0, a.qrow, qpol);
+          tma_load_2d_hint(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow, qpol);
           q_last[slot] = use;
         }
         const long long kvrow0 = a.bg * p.Lmax;
@@ -513,13 +514,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
 #pragma unroll
       for (int h = 0; h < kGroupRows; ++h)
-        if (h < p.G && a.valid) p.o[(static_cast<long long>(a.qrow) + h) * kHeadDim + tid] = __float2bfloat16_rn(of[h]);
+        if (h < p.G && a.valid)
+          st_stream_bf16(p.o + (static_cast<long long>(a.qrow) + h) * kHeadDim + tid, __float2bfloat16_rn(of[h]));
       if (p.lse != nullptr && tid < p.G && a.valid) {
         float lv = -INFINITY;
 #pragma unroll
         for (int h = 0; h < kGroupRows; ++h)
           if (h == tid) lv = Lt[h] > 0.f ? (M[h] + lg2(Lt[h])) * 0.6931471805599453f : -INFINITY;
-        p.lse[(static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.row] = lv;
+        __stcs(p.lse + (static_cast<long long>(a.b) * p.Hq + a.g * p.G + tid) * p.Lq + a.row, lv);
       }
     }
     tc_fence_before();
