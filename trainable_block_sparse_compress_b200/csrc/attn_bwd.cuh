@@ -538,23 +538,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       dv[c][0] = dv[c][1] = dv[c][2] = dv[c][3] = 0.f;
     }
     const int32_t* rows = p.list + p.off[e] + rs;
-    for (int i = 0; i < nrows; ++i, ++gtok) {
-      const int st = static_cast<int>(gtok % kBwdTokStages);
-      mbar_wait(&S.tfull[st], (gtok / kBwdTokStages) & 1, &S.abort);
-      const int t = rows[i];
-      const uint32_t ts = smem_u32(toks + st * kBwdTokBytes);
-      // this lane's heads (columns): 8 nt + 2 q4 + {0, 1}
-      float lse2[2][2], dl[2][2];
+    // this lane's heads (columns): 8 nt + 2 q4 + {0, 1}; lse and D of row t, loaded one row
+    // ahead of their use (and the row index two ahead), off the MMA chain
+    auto load_row = [&](int t, float (&l2)[2][2], float (&d)[2][2]) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int h = 8 * nt + 2 * q4 + c;
           const long long li = (static_cast<long long>(b) * p.Hq + g * p.G + h) * p.L + t;
-          lse2[nt][c] = h < p.G ? p.lse[li] * 1.4426950408889634f : INFINITY;
-          dl[nt][c] = h < p.G ? p.delta[li] : 0.f;
+          l2[nt][c] = h < p.G ? p.lse[li] * 1.4426950408889634f : INFINITY;
+          d[nt][c] = h < p.G ? p.delta[li] : 0.f;
         }
       }
+    };
+    int t_next = nrows > 0 ? rows[0] : 0;
+    float lse_next[2][2], dl_next[2][2];
+    load_row(t_next, lse_next, dl_next);
+    int t_after = nrows > 1 ? rows[1] : 0;
+    for (int i = 0; i < nrows; ++i, ++gtok) {
+      const int st = static_cast<int>(gtok % kBwdTokStages);
+      const int t = t_next;
+      float lse2[2][2], dl[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          lse2[nt][c] = lse_next[nt][c];
+          dl[nt][c] = dl_next[nt][c];
+        }
+      }
+      if (i + 1 < nrows) {
+        t_next = t_after;
+        load_row(t_next, lse_next, dl_next);
+        t_after = i + 2 < nrows ? rows[i + 2] : 0;
+      }
+      mbar_wait(&S.tfull[st], (gtok / kBwdTokStages) & 1, &S.abort);
+      const uint32_t ts = smem_u32(toks + st * kBwdTokBytes);
       float s[2][4], dp[2][4];
       {
         uint32_t fa[8][4];  // this warp's 16 keys of K, then of V, as A fragments
