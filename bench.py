@@ -643,8 +643,9 @@ def run_reference(args):
 
 def profile_run(name, device):
     """The hot path of one workload, twice (a warm-up and one more run), for single-kernel
-    profiler captures on small cases: prefill (compress, select, attend) or a decode step
-    (compress the caches, select, attend).  Prints nothing."""
+    profiler captures: prefill (compress, select, attend) or a decode step (compress the
+    caches, then the fused step, then the separate selection and attention calls on the
+    same inputs).  Prints nothing."""
     wl = WORKLOADS[name]
     p = ops.Params.from_workload(wl)
     x = make_inputs(wl, seed=0)
@@ -656,6 +657,8 @@ def profile_run(name, device):
             lens = x.lens.to(device)
             kc = ops.compress_keys(p, k, lens=lens)
             ops.decode(p, q, k, v, kc, lens, wl.seq_len)
+            idx = ops.select_blocks_decode(p, q, kc, lens, wl.seq_len)
+            ops.sparse_attn_decode(p, q, k, v, lens, idx)
     torch.cuda.synchronize()
     assert ops.device_error(clear=True) == 0
 
