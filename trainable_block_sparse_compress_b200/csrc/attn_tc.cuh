@@ -11,7 +11,7 @@
 // pairs (warp 11), so a K slot is free again right after its QK and a V slot right
 // after its PV; per pair:
 //   warp 9 (one thread) issues  S^T = K_pair . Q^T   (UMMA M128 N16 K128: keys x heads)
-//          into one of six TMEM score buffers as soon as the pair has landed;
+//          into one of four TMEM score buffers as soon as the pair has landed;
 //   warp 10 (one thread) issues, as soon as P is in shared memory,
 //          O^T += V^T . P^T   (UMMA M128 N16 K128: V read through an MN-major
 //          descriptor, P K-major) into the TMEM output buffer of the pair's warpgroup.
@@ -37,7 +37,7 @@
 
 namespace infllmv2 {
 
-constexpr int kAtKStages = 3;                      // slots of the K ring
+constexpr int kAtKStages = 4;                      // slots of the K ring
 constexpr int kAtVStages = 2;                      // slots of the V ring
 constexpr int kAtKHalf = 2 * kKvTileBytes / 2;     // 16 KB: one 64-column half of 128 keys
 constexpr int kAtSlotBytes = 2 * kKvTileBytes;     // 32 KB: a pair of K (or V) blocks
@@ -46,7 +46,7 @@ constexpr int kAtSoftWGs = 2;
 constexpr int kAtThreads = 32 * (4 * kAtSoftWGs + 4);
 constexpr int kAtTmaWarp = 4 * kAtSoftWGs, kAtMmaWarp = kAtTmaWarp + 1, kAtPvWarp = kAtTmaWarp + 2,
               kAtVTmaWarp = kAtTmaWarp + 3;
-constexpr int kAtBufs = 6;  // score (TMEM) and probability (shared) buffers in flight
+constexpr int kAtBufs = 4;  // score (TMEM) and probability (shared) buffers in flight
 // TMEM columns: scores S[b] at 16 b, outputs O[item parity][wg] at 16 kAtBufs + 16 (2 it + wg);
 // the allocation is the next power of two
 constexpr uint32_t kAtOCol = 16 * kAtBufs;
@@ -191,9 +191,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     uint32_t gpair = 0;
     int it = 0;
     const uint64_t qpol = l2_policy_evict_first();  // queries are read once: K/V keep L2
-    long long k_last[kAtKStages];  // last pair loaded into each K stage (lane 0), for the drain
-    int q_last[2] = {-1, -1};      // last use of each query-tile slot
-    for (int st = 0; st < kAtKStages; ++st) k_last[st] = -1;
+    // copies issued so far (lane 0), in order: pairs 0 .. k_issued - 1 and query tiles of
+    // items 0 .. q_issued - 1 (after an abort nothing more is issued), for the drain
+    uint32_t k_issued = 0, q_issued = 0;
     for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
       const int slot = it & 1, use = it >> 1;
       if (use > 0) mbar_wait(&S.q_empty[slot], (use - 1) & 1, &S.abort);
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           mbar_arrive_expect_tx(&S.q_full[slot], kQTileBytes);
           tma_load_2d_hint(qs, &tm_q, &S.q_full[slot], 0, a.qrow, qpol);
           tma_load_2d_hint(qs + kQTileBytes / 2, &tm_q, &S.q_full[slot], 64, a.qrow, qpol);
-          q_last[slot] = use;
+          q_issued = static_cast<uint32_t>(it) + 1u;
         }
         const long long kvrow0 = a.bg * p.Lmax;
         for (int i = 0; i < np; ++i, ++gpair) {
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
           const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
           unsigned char* sk = kring + st * kAtSlotBytes;
-          k_last[st] = gpair;
+          k_issued = gpair + 1u;
           mbar_arrive_expect_tx(&S.k_full[st], kAtSlotBytes);
           // rows 0-63 of each 128-key half: block a; rows 64-127: block b (zeros when absent)
           tma_load_2d(sk, &tm_k, &S.k_full[st], 0, ra);
@@ -253,10 +253,16 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       gpair = __shfl_sync(0xffffffffu, gpair, 0);
     }
     if (lane == 0 && S.abort) {  // let every copy this warp issued land before the CTA ends
-      for (int st = 0; st < kAtKStages; ++st)
-        if (k_last[st] >= 0) mbar_wait_drain(&S.k_full[st], static_cast<uint32_t>((k_last[st] / kAtKStages) & 1));
-      for (int sl = 0; sl < 2; ++sl)
-        if (q_last[sl] >= 0) mbar_wait_drain(&S.q_full[sl], static_cast<uint32_t>(q_last[sl] & 1));
+      for (uint32_t st = 0; st < kAtKStages; ++st)
+        if (k_issued > st) {  // the last pair issued into stage st
+          const uint32_t last = st + kAtKStages * ((k_issued - 1u - st) / kAtKStages);
+          mbar_wait_drain(&S.k_full[st], (last / kAtKStages) & 1u);
+        }
+      for (uint32_t sl = 0; sl < 2; ++sl)
+        if (q_issued > sl) {  // the last item whose query tile went to slot sl
+          const uint32_t last = sl + 2u * ((q_issued - 1u - sl) / 2u);
+          mbar_wait_drain(&S.q_full[sl], (last >> 1) & 1u);
+        }
     }
     return;
   }
@@ -268,8 +274,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (lane == 0) {
       uint32_t gpair = 0, n_tail = 0;
       int it = 0;
-      long long v_last[kAtVStages];  // last pair loaded into each V stage, for the drain
-      for (int st = 0; st < kAtVStages; ++st) v_last[st] = -1;
+      uint32_t v_issued = 0;  // V pairs issued so far, in order (for the drain)
       for (long long item = blockIdx.x; item < p.num_items; item += gridDim.x, ++it) {
         const int slot = it & 1, use = it >> 1;
         mbar_wait(&S.q_full[slot], use & 1, &S.abort);  // the item's block list is ready
@@ -288,7 +293,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int ra = static_cast<int>(kvrow0 + static_cast<long long>(ja) * kBlock);
           const int rb = jb >= 0 ? static_cast<int>(kvrow0 + static_cast<long long>(jb) * kBlock) : -kBlock;
           unsigned char* sv = vring + st * kAtSlotBytes;
-          v_last[st] = gpair;
+          v_issued = gpair + 1u;
           if ((tail >> 1) != i) {  // (tail == -1: no straddling block in the item)
             mbar_arrive_expect_tx(&S.v_full[st], kAtSlotBytes);
             tma_load_2d(sv, &tm_v, &S.v_full[st], 0, ra);
@@ -314,7 +319,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       if (S.abort)  // let every copy this thread issued land before the CTA ends
         for (int st = 0; st < kAtVStages; ++st)
-          if (v_last[st] >= 0) mbar_wait_drain(&S.v_full[st], static_cast<uint32_t>((v_last[st] / kAtVStages) & 1));
+          if (v_issued > static_cast<uint32_t>(st)) {
+            const uint32_t last = st + kAtVStages * ((v_issued - 1u - st) / kAtVStages);
+            mbar_wait_drain(&S.v_full[st], (last / kAtVStages) & 1u);
+          }
     }
     return;
   }
