@@ -20,12 +20,12 @@
 //                      selected K/V blocks stream through a TMA ring; four warps take 16
 //                      keys of each block and accumulate dq (16 heads x 128) with
 //                      m16n8k16 MMAs, merged at the end of the item;
-//   bwd_dkdv_kernel    block-major: per segment the block's K and V stay in shared memory
-//                      while the segment's query rows stream their Q and dO tiles through
-//                      a TMA ring; warp w accumulates dK and dV of keys 16w .. 16w+15 in
-//                      registers and adds them to the fp32 workspace (atomics: a block's
-//                      segments run on different CTAs, so the summation order of dK / dV
-//                      may vary between runs, within fp32 rounding);
+//   bwd_dkdv_tc_kernel block-major, on the tcgen05 tensor cores (csrc/attn_bwd_tc.cuh): per
+//                      segment the block's K and V stay in shared memory while the segment's
+//                      tokens stream their Q and dO rows 8 at a time; dK and dV accumulate in
+//                      TMEM and are added to the fp32 workspace (atomics: a block's segments
+//                      run on different CTAs, so the summation order of dK / dV may vary
+//                      between runs, within fp32 rounding);
 //   bwd_cast_kernel    the fp32 dK / dV to bf16.
 #pragma once
 #include "attn.cuh"
@@ -37,8 +37,7 @@ constexpr int kBwdSeg = 128;       // query rows per dK/dV work item at most
 constexpr int kBwdConsumers = 4;
 constexpr int kBwdThreads = 32 * (kBwdConsumers + 1);
 constexpr int kBwdKvStages = 4;    // dq kernel: K+V block stages (32 KB each)
-constexpr int kBwdTokStages = 8;   // dkdv kernel: Q+dO row-tile stages (8 KB each)
-constexpr int kBwdTokBytes = 2 * kQTileBytes;
+constexpr int kBwdTokBytes = 2 * kQTileBytes;  // dq kernel: a token's Q then dO rows
 constexpr int kBwdDqRowFloats = kHeadDim + 4;
 
 struct BwdParams {
@@ -422,16 +421,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-struct BwdKvSmem {
-  uint64_t kv_full[2], kv_empty[2], tfull[kBwdTokStages], tempty[kBwdTokStages];
-  volatile int abort;
-};
-
-constexpr size_t bwd_dkdv_smem_bytes() {
-  return 1024 + 2 * static_cast<size_t>(kAttnStageBytes) + static_cast<size_t>(kBwdTokStages) * kBwdTokBytes +
-         sizeof(BwdKvSmem);
-}
-
 // Segment `item` -> (entry e = bg * nblk + j, segment within the entry's list).
 __device__ __forceinline__ int bwd_find_entry(const int32_t* segoff, int n, int item) {
   int lo = 0, hi = n - 1;  // largest e with segoff[e] <= item
@@ -441,185 +430,6 @@ __device__ __forceinline__ int bwd_find_entry(const int32_t* segoff, int n, int 
     else hi = mid - 1;
   }
   return lo;
-}
-
-// grid = persistent CTAs over the segments (their total is segoff[n]), block = 160.
-__global__ void __launch_bounds__(kBwdThreads, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const BwdParams p) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = align_smem(smem_raw, 1024);
-  unsigned char* kv = base;                              // 2 slots: K then V of a block
-  unsigned char* toks = kv + 2 * kAttnStageBytes;        // token ring: Q then dO rows
-  BwdKvSmem& S = *reinterpret_cast<BwdKvSmem*>(toks + kBwdTokStages * kBwdTokBytes);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_entries = p.B * p.Hkv * p.nblk;
-  const int total = p.segoff[n_entries];
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&S.kv_full[s], 1);
-      mbar_init(&S.kv_empty[s], kBwdConsumers);
-    }
-    for (int s = 0; s < kBwdTokStages; ++s) {
-      mbar_init(&S.tfull[s], 1);
-      mbar_init(&S.tempty[s], kBwdConsumers);
-    }
-    S.abort = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == kBwdConsumers) {
-    // ------------------------------------------------------------ producer (lane 0)
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      uint32_t gtok = 0;
-      int it = 0;
-      for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
-        const int e = bwd_find_entry(p.segoff, n_entries, item);
-        const int seg = item - p.segoff[e];
-        const int bg = e / p.nblk, j = e % p.nblk;
-        const int b = bg / p.Hkv, g = bg % p.Hkv;
-        const int r0 = seg * kBwdSeg, nrows = min(kBwdSeg, p.cnt[e] - r0);
-        const int slot = it & 1, use = it >> 1;
-        if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, &S.abort);
-        if (S.abort) break;
-        unsigned char* sk = kv + slot * kAttnStageBytes;
-        const int krow = bg * p.L + j * kBlock;
-        mbar_arrive_expect_tx(&S.kv_full[slot], kAttnStageBytes);
-        tma_load_2d(sk, &tm_k, &S.kv_full[slot], 0, krow);
-        tma_load_2d(sk + kKvTileBytes / 2, &tm_k, &S.kv_full[slot], 64, krow);
-        tma_load_2d(sk + kKvTileBytes, &tm_v, &S.kv_full[slot], 0, krow);
-        tma_load_2d(sk + kKvTileBytes + kKvTileBytes / 2, &tm_v, &S.kv_full[slot], 64, krow);
-        const int32_t* rows = p.list + p.off[e] + r0;
-        for (int i = 0; i < nrows; ++i, ++gtok) {
-          const int st = static_cast<int>(gtok % kBwdTokStages);
-          const uint32_t u = gtok / kBwdTokStages;
-          if (u > 0) mbar_wait(&S.tempty[st], (u - 1) & 1, &S.abort);
-          if (S.abort) break;
-          const int qrow = (b * p.L + rows[i]) * p.Hq + g * p.G;
-          unsigned char* ts = toks + st * kBwdTokBytes;
-          mbar_arrive_expect_tx(&S.tfull[st], kBwdTokBytes);
-          tma_load_2d(ts, &tm_q, &S.tfull[st], 0, qrow);
-          tma_load_2d(ts + kQTileBytes / 2, &tm_q, &S.tfull[st], 64, qrow);
-          tma_load_2d(ts + kQTileBytes, &tm_do, &S.tfull[st], 0, qrow);
-          tma_load_2d(ts + kQTileBytes + kQTileBytes / 2, &tm_do, &S.tfull[st], 64, qrow);
-        }
-        if (S.abort) break;
-      }
-    }
-    return;
-  }
-
-  // --------------------------------------------------------------- consumer warps
-  const int q4 = lane & 3, r0l = lane >> 2;
-  const int kofs = 16 * warp;
-  const float sl2 = p.scale_log2;
-  uint32_t gtok = 0;
-  int it = 0;
-  for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
-    const int e = bwd_find_entry(p.segoff, n_entries, item);
-    const int seg = item - p.segoff[e];
-    const int bg = e / p.nblk, j = e % p.nblk;
-    const int b = bg / p.Hkv, g = bg % p.Hkv;
-    const int rs = seg * kBwdSeg, nrows = min(kBwdSeg, p.cnt[e] - rs);
-    const int slot = it & 1, use = it >> 1;
-    mbar_wait(&S.kv_full[slot], use & 1, &S.abort);
-    const uint32_t sk = smem_u32(kv + slot * kAttnStageBytes);
-    const uint32_t sv = sk + kKvTileBytes;
-    float dk[16][4], dv[16][4];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      dk[c][0] = dk[c][1] = dk[c][2] = dk[c][3] = 0.f;
-      dv[c][0] = dv[c][1] = dv[c][2] = dv[c][3] = 0.f;
-    }
-    const int32_t* rows = p.list + p.off[e] + rs;
-    // this lane's heads (columns): 8 nt + 2 q4 + {0, 1}; lse and D of row t, loaded one row
-    // ahead of their use (and the row index two ahead), off the MMA chain
-    auto load_row = [&](int t, float (&l2)[2][2], float (&d)[2][2]) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int h = 8 * nt + 2 * q4 + c;
-          const long long li = (static_cast<long long>(b) * p.Hq + g * p.G + h) * p.L + t;
-          l2[nt][c] = h < p.G ? p.lse[li] * 1.4426950408889634f : INFINITY;
-          d[nt][c] = h < p.G ? p.delta[li] : 0.f;
-        }
-      }
-    };
-    int t_next = nrows > 0 ? rows[0] : 0;
-    float lse_next[2][2], dl_next[2][2];
-    load_row(t_next, lse_next, dl_next);
-    int t_after = nrows > 1 ? rows[1] : 0;
-    for (int i = 0; i < nrows; ++i, ++gtok) {
-      const int st = static_cast<int>(gtok % kBwdTokStages);
-      const int t = t_next;
-      float lse2[2][2], dl[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          lse2[nt][c] = lse_next[nt][c];
-          dl[nt][c] = dl_next[nt][c];
-        }
-      }
-      if (i + 1 < nrows) {
-        t_next = t_after;
-        load_row(t_next, lse_next, dl_next);
-        t_after = i + 2 < nrows ? rows[i + 2] : 0;
-      }
-      mbar_wait(&S.tfull[st], (gtok / kBwdTokStages) & 1, &S.abort);
-      const uint32_t ts = smem_u32(toks + st * kBwdTokBytes);
-      float s[2][4], dp[2][4];
-      {
-        uint32_t fa[8][4];  // this warp's 16 keys of K, then of V, as A fragments
-        load_a_frags(sk, kofs, kKvTileBytes / 2, fa);
-        mma_rows_t(fa, ts, 0, kQTileBytes / 2, s);  // S^T  = K Q^T   (16 keys x 16 heads)
-        load_a_frags(sv, kofs, kKvTileBytes / 2, fa);
-        mma_rows_t(fa, ts + kQTileBytes, 0, kQTileBytes / 2, dp);  // dP^T = V dO^T
-      }
-      float pr[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int key = j * kBlock + kofs + r0l + 8 * (e2 >> 1);
-          const float x = key <= t ? ex2(fmaf(s[nt][e2], sl2, -lse2[nt][e2 & 1])) : 0.f;
-          pr[nt][e2] = x;
-          s[nt][e2] = x * (dp[nt][e2] - dl[nt][e2 & 1]);  // dS^T
-        }
-      }
-      uint32_t pa[4], dsa[4];
-      acc_to_a(pr, pa);
-      acc_to_a(s, dsa);
-      mma_acc_rows(pa, ts + kQTileBytes, 0, kQTileBytes / 2, dv);  // dV += P^T dO
-      mma_acc_rows(dsa, ts, 0, kQTileBytes / 2, dk);               // dK += dS^T Q
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.tempty[st]);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.kv_empty[slot]);  // the block's K and V are no longer read
-    // add this segment's dK, dV of keys kofs + r0l (+ 8) to the fp32 workspace
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int key = j * kBlock + kofs + r0l + 8 * hr;
-      if (key < p.L) {
-        const long long rowi = (static_cast<long long>(bg) * p.L + key) * kHeadDim;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int col = 8 * c + 2 * q4;
-          atomicAdd(reinterpret_cast<float2*>(p.dk32 + rowi + col),
-                    make_float2(dk[c][2 * hr] * p.scale, dk[c][2 * hr + 1] * p.scale));
-          atomicAdd(reinterpret_cast<float2*>(p.dv32 + rowi + col), make_float2(dv[c][2 * hr], dv[c][2 * hr + 1]));
-        }
-      }
-    }
-  }
 }
 
 // dk / dv (bf16) from the fp32 workspace; n4 = elements / 4.

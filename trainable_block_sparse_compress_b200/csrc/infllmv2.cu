@@ -17,6 +17,7 @@
 #include "append.cuh"
 #include "attn.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_dec.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -690,12 +691,12 @@ int infllmv2_sparse_attn_backward(const infllmv2_params* p, const void* q, const
   bwd_fill_kernel<<<rgrid, 256, 0, s>>>(block_idx, static_cast<int>(rows), L, p->topk, a.nblk, a.off,
                                         reinterpret_cast<int32_t*>(wb + w.cursor), const_cast<int32_t*>(a.list));
   if ((st = launch_status()) != INFLLMV2_OK) return st;
-  const size_t smem_q = bwd_dq_smem_bytes(), smem_kv = bwd_dkdv_smem_bytes();
+  const size_t smem_q = bwd_dq_smem_bytes(), smem_kv = bwd_dkdv_tc_smem_bytes();
   if ((st = set_smem(reinterpret_cast<const void*>(bwd_dq_kernel), smem_q)) != INFLLMV2_OK) return st;
-  if ((st = set_smem(reinterpret_cast<const void*>(bwd_dkdv_kernel), smem_kv)) != INFLLMV2_OK) return st;
+  if ((st = set_smem(reinterpret_cast<const void*>(bwd_dkdv_tc_kernel), smem_kv)) != INFLLMV2_OK) return st;
   bwd_dq_kernel<<<static_cast<unsigned>(std::min<long long>(rows, num_sms())), kBwdThreads, smem_q, s>>>(tq, tdo, tk,
                                                                                                         tv, a);
-  bwd_dkdv_kernel<<<static_cast<unsigned>(num_sms()), kBwdThreads, smem_kv, s>>>(tq, tdo, tk, tv, a);
+  bwd_dkdv_tc_kernel<<<static_cast<unsigned>(num_sms()), kBtThreads, smem_kv, s>>>(tq, tdo, tk, tv, a);
   const long long n4 = rows * kHeadDim / 4;
   bwd_cast_kernel<<<static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 8LL * num_sms())), 256, 0, s>>>(
       reinterpret_cast<const float4*>(a.dk32), reinterpret_cast<const float4*>(a.dv32), n4, static_cast<uint2*>(dk),
