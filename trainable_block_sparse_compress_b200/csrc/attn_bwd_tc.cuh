@@ -128,16 +128,22 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         kv_issued = static_cast<uint32_t>(it) + 1u;
         const int32_t* rows = p.list + p.off[e] + r0;
         for (int ti = 0; ti < ntiles; ++ti, ++gt) {
+          // the tile's 8 list entries, loaded together (padding tokens repeat the first row,
+          // masked in the epilogue)
+          int tok[kBtTok];
+#pragma unroll
+          for (int u = 0; u < kBtTok; ++u) {
+            const int r = ti * kBtTok + u;
+            tok[u] = rows[r < nrows ? r : 0];
+          }
           const int st = static_cast<int>(gt & 1u);
           if (gt >= kBtStages) mbar_wait(&S.t_empty[st], ((gt >> 1) - 1u) & 1u, &S.abort);
           if (S.abort) break;
           unsigned char* tq = tiles + st * kBtStageBytes;
           mbar_arrive_expect_tx(&S.t_full[st], kBtStageBytes);
-#pragma unroll 1
+#pragma unroll
           for (int u = 0; u < kBtTok; ++u) {
-            const int r = ti * kBtTok + u;
-            const int t = rows[r < nrows ? r : 0];  // padding tokens repeat the first row (masked)
-            const int qrow = (b * p.L + t) * p.Hq + g * p.G;
+            const int qrow = (b * p.L + tok[u]) * p.Hq + g * p.G;
             tma_load_2d(tq + u * 2048, &tm_q, &S.t_full[st], 0, qrow);
             tma_load_2d(tq + kBtHalfBytes + u * 2048, &tm_q, &S.t_full[st], 64, qrow);
             tma_load_2d(tq + kBtTileBytes + u * 2048, &tm_do, &S.t_full[st], 0, qrow);
@@ -249,14 +255,24 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     const int r0 = seg * kBwdSeg, nrows = min(kBwdSeg, p.cnt[e] - r0);
     const int ntiles = (nrows + kBtTok - 1) / kBtTok;
     const int32_t* rows = p.list + p.off[e] + r0;
-    for (int ti = 0; ti < ntiles; ++ti, ++gt) {
-      const uint32_t sb = gt & 1u;
+    // this row's token, lse and D, loaded one tile ahead of their use
+    auto load_row = [&](int ti, int& t, float& lse2, float& dl) {
       const int r = ti * kBtTok + u;
       const bool rv = r < nrows && h < p.G;
-      const int t = rows[r < nrows ? r : 0];
+      t = rows[r < nrows ? r : 0];
       const long long li = (static_cast<long long>(b) * p.Hq + g * p.G + (h < p.G ? h : 0)) * p.L + t;
-      const float lse2 = rv ? p.lse[li] * 1.4426950408889634f : 0.f;
-      const float dl = rv ? p.delta[li] : 0.f;
+      lse2 = rv ? p.lse[li] * 1.4426950408889634f : 0.f;
+      dl = rv ? p.delta[li] : 0.f;
+    };
+    int t_n;
+    float lse2_n, dl_n;
+    load_row(0, t_n, lse2_n, dl_n);
+    for (int ti = 0; ti < ntiles; ++ti, ++gt) {
+      const uint32_t sb = gt & 1u;
+      const bool rv = ti * kBtTok + u < nrows && h < p.G;
+      const int t = t_n;
+      const float lse2 = lse2_n, dl = dl_n;
+      if (ti + 1 < ntiles) load_row(ti + 1, t_n, lse2_n, dl_n);
       mbar_wait(&S.sdp_full[sb], (gt >> 1) & 1u, &S.abort);
       if (gt > 0) mbar_wait(&S.pds_empty, (gt - 1u) & 1u, &S.abort);  // dV / dK of the previous tile done
       tc_fence_after();
