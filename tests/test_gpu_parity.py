@@ -78,7 +78,7 @@ GOLDEN_CASES = [c for f in ("select_closed_form.json", "select_variants.json")
 
 
 @pytest.mark.parametrize("case", GOLDEN_CASES, ids=lambda c: c["name"])
-@pytest.mark.parametrize("mode", ["prefill", "decode"])
+@pytest.mark.parametrize("mode", ["prefill", "decode", "step"])
 def test_select_closed_form_cases(case, mode):
     L, Hq = case["seq_len"], case["num_q_heads"]
     k = torch.zeros((1, 1, L, 128))
@@ -97,10 +97,15 @@ def test_select_closed_form_cases(case, mode):
         kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda())
         idx = ops.select_blocks_prefill(p, q.to(torch.bfloat16).cuda(), kc).cpu().numpy()
         assert idx[0, 0, t].tolist() == case["expected"]
-    else:  # the same row as a decode query over a cache of t + 1 tokens
+    else:  # the same row as a decode query over a cache of t + 1 tokens (alone, or in the fused step)
         lens = torch.tensor([t + 1], dtype=torch.int32).cuda()
-        kc = ops.compress_keys(p, k.to(torch.bfloat16).cuda(), lens=lens)
-        idx = ops.select_blocks_decode(p, q[:, t].to(torch.bfloat16).contiguous().cuda(), kc, lens, L)
+        kg = k.to(torch.bfloat16).cuda()
+        kc = ops.compress_keys(p, kg, lens=lens)
+        qd = q[:, t].to(torch.bfloat16).contiguous().cuda()
+        if mode == "decode":
+            idx = ops.select_blocks_decode(p, qd, kc, lens, L)
+        else:
+            _, _, idx = ops.decode_step(p, qd, kg, torch.zeros_like(kg), kc, lens)
         assert idx.cpu().numpy()[0, 0, 0].tolist() == case["expected"]
 
 

@@ -6,11 +6,12 @@
 // selected blocks and attend only to them.
 //
 // A thread-block cluster per (sequence, kv-head) runs the selection phases of
-// select_decode.cuh (Kc streamed and scored by every CTA, keys gathered in CTA 0, CTA 0's
-// top-k into its shared memory and block_idx), then, after one more cluster barrier, the
-// attention phases of attn_dec.cuh over that list (each CTA copies its contiguous share of
-// the list from CTA 0 through distributed shared memory, streams those K/V blocks and the
-// partial states are merged across the cluster).  Clusters do not wait for one another,
+// select_decode.cuh (Kc streamed and scored by every CTA, every CTA's block keys stored
+// into every CTA of the cluster), then each CTA runs the same deterministic top-k over all
+// keys in its own shared memory -- so no CTA waits for another's list -- and goes straight
+// on to the attention phases of attn_dec.cuh over its contiguous share of that list (it
+// streams those K/V blocks, and the partial states are merged across the cluster); CTA 0
+// also writes the list to block_idx.  Clusters do not wait for one another,
 // so a cluster whose sequence is short streams its K/V while longer sequences are still
 // being scored, and nothing round-trips through global memory between the two halves.
 // The selection's tile ring and block maxima and the attention's ring share one region of
@@ -33,8 +34,7 @@ constexpr size_t kDsRegion = kSdRegionBytes > kDsAttnRegion ? kSdRegionBytes : k
 
 struct DsSmem {
   SdSmem sel;
-  AdSmem attn;          // attn.list: the item's list as CTA 0 emits it
-  int share[kMaxTopk];  // this CTA's blocks of that list
+  AdSmem attn;  // attn.list: the item's list, as every CTA emits it
 };
 
 constexpr size_t decode_step_smem_bytes() { return 1024 + kDsRegion + sizeof(DsSmem); }
@@ -120,37 +120,25 @@ __global__ void __launch_bounds__(kSdThreads)
     }
   }
 
-  // ---- selection
+  // ---- selection: every CTA receives every key and derives the same list
   sd_score_chunk(&tm_kc, P.sel, it, region, bm, D.sel);
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
-  sd_block_keys(cluster, P.sel, it, region, bm, D.sel);
-  cluster.sync();  // CTA 0 holds every key
+  sd_block_keys<true>(cluster, P.sel, it, region, bm, D.sel);
+  cluster.sync();  // every CTA holds every key; no CTA touches a peer's memory until the merge
+  const int n_all = sd_select(P.sel, it, region, D.attn.list, D.sel);
   if (c == 0) {
-    sd_select(P.sel, it, region, D.attn.list, D.sel);
     int32_t* out = P.sel.idx + bg * topk;
     for (int e = threadIdx.x; e < topk; e += kSdThreads) out[e] = D.attn.list[e];
-    if (warp == 0) {  // the list is ascending and -1 padded: count its blocks
-      int count = 0;
-      for (int e0 = 0; e0 < topk; e0 += 32) {
-        const int e = e0 + lane;
-        count += __popc(__ballot_sync(0xffffffffu, e < topk && D.attn.list[e] >= 0));
-      }
-      if (lane == 0) D.attn.n_blocks = count;
-    }
   }
-  cluster.sync();  // CTA 0's list is complete; no CTA reads a selection array after this
 
   // ---- attention over this CTA's contiguous share of the list
-  const int n_all = *cluster.map_shared_rank(&D.attn.n_blocks, 0);
   const int per = (n_all + C - 1) / C;
   const int lo = min(c * per, n_all);
   const int nsh = min(lo + per, n_all) - lo;
-  const int* list0 = cluster.map_shared_rank(D.attn.list, 0);
-  for (int i = threadIdx.x; i < nsh; i += kSdThreads) D.share[i] = list0[lo + i];
   fence_proxy_async_smem();  // the region's generic accesses before the ring's copies
   __syncthreads();
   const int qrow = it.b * P.attn.Hq + it.g * P.attn.G;
-  ad_partial(&tm_q, &tm_k, &tm_v, P.attn, bg, qrow, it.n - 1, D.share, nsh, region, qtile, D.attn);
+  ad_partial(&tm_q, &tm_k, &tm_v, P.attn, bg, qrow, it.n - 1, D.attn.list + lo, nsh, region, qtile, D.attn);
   ad_merge(cluster, P.attn, qrow, region, D.attn);
 }
 

@@ -50,9 +50,8 @@ constexpr int kSdBinsPerThread = (kSdHistBins + kSdThreads - 1) / kSdThreads;
 // and the take flags of a tie-ranked emission
 constexpr int kSdKeysOff = 0;
 constexpr int kSdHistOff = kSdKeysOff + 4 * kSdMaxKeys;
-constexpr int kSdFlagOff = kSdHistOff + 4 * kSdHistBins;
-constexpr int kSdScratchBytes = kSdFlagOff + kSdMaxR * kSdThreads;
-static_assert(kSdStages * kKcTileBytes >= kSdScratchBytes, "the selection scratch of CTA 0 reuses its tile ring");
+constexpr int kSdScratchBytes = kSdHistOff + 4 * kSdHistBins;
+static_assert(kSdStages * kKcTileBytes >= kSdScratchBytes, "the selection scratch reuses the tile ring");
 static_assert(kSdMaxCluster * kSdMaxChunk >= (INFLLMV2_MAX_SEQ_LEN - kKernel) / kStride + 1,
               "a cluster covers the longest sequence");
 
@@ -245,99 +244,69 @@ __device__ __forceinline__ TopkThreshold cta_topk_threshold(const uint32_t* keys
 }
 
 // All kSdThreads threads write the selected blocks of one row, ascending, padded with
-// -1: block j in [0, n) is taken when forced, or key > T, or key == T among the first
-// `ties` such keys in ascending j (the rule of warp_emit_selection).  Keys are visited
-// slot-major (thread i, slot s: key i + kSdThreads s), which is ascending j: one pass
-// counts the taken keys per (slot, warp) with ballots, a warp scan turns the slot totals
-// into slot bases, and a second pass writes each taken key at its base plus its rank in
-// the warp and in the slot.  Tie ranks (only when some keys equal to T stay out) come
-// from the same two passes run on the tie flags first.
-__device__ __forceinline__ void cta_emit_selection(const uint32_t* keys, int n, TopkThreshold th, int cur,
-                                                   int n_init, int n_local, int topk, int32_t* out,
-                                                   unsigned char* tflag, SdSmem& S) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  const int R = (n + kSdThreads - 1) / kSdThreads;
-  const bool simple = topk_simple(th);  // no tie ranks needed: take forced or key >= lo
-  const uint32_t lo = take_from(th);
-  // per (slot, warp) counts of a flag, then S.sbase[s] = flagged keys in slots < s
-  auto slot_counts = [&](auto flag) -> int {
-    for (int s = 0; s < R; ++s) {
-      const unsigned m = __ballot_sync(0xffffffffu, flag(s));
-      if (lane == 0) S.wc[s][warp] = __popc(m);
-    }
-    __syncthreads();
-    int total = 0;
-    if (warp == 0) {
-      int v = 0;
-      if (lane < R)
-#pragma unroll
-        for (int ww = 0; ww < kSdWarps; ++ww) v += S.wc[lane][ww];
-      int incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane < R) S.sbase[lane] = incl - v;
-      if (lane == 31) S.total = incl;
-    }
-    __syncthreads();
-    total = S.total;
-    return total;
-  };
-  auto rank_of = [&](int s, unsigned m) -> int {  // flagged keys before this thread's key of slot s
-    int before = S.sbase[s];
-#pragma unroll
-    for (int ww = 0; ww < kSdWarps; ++ww) before += ww < warp ? S.wc[s][ww] : 0;
-    return before + __popc(m & lt);
-  };
-  auto key_at = [&](int s, int& j) -> uint32_t {
-    j = static_cast<int>(threadIdx.x) + kSdThreads * s;
-    return j < n ? keys[j] : 0u;
-  };
-  auto forced = [&](int j) { return j < n && (j < n_init || j > cur - n_local); };
-  if (simple) {
-    auto take = [&](int s) {
-      int j;
-      const uint32_t k = key_at(s, j);
-      return j < n && (forced(j) || k >= lo);
-    };
-    const int total = slot_counts(take);
-    for (int s = 0; s < R; ++s) {
-      const bool f = take(s);
-      const int pos = rank_of(s, __ballot_sync(0xffffffffu, f));
-      if (f && pos < topk) out[pos] = static_cast<int>(threadIdx.x) + kSdThreads * s;
-    }
-    for (int e = total + static_cast<int>(threadIdx.x); e < topk; e += kSdThreads) out[e] = -1;
-    __syncthreads();  // S.wc, S.sbase are free again
-    return;
+// -1, and return how many there are: block j in [0, n) is taken when forced, or key > T,
+// or key == T among the first `ties` such keys in ascending j (the rule of
+// warp_emit_selection).  Thread i owns the contiguous keys [i R, i R + R), R odd so that a
+// warp's strided reads hit 32 different banks: it counts its strict takes (forced or
+// above T) and its keys equal to T, one CTA-wide exclusive scan gives every thread the
+// counts before its range, and a second pass over the range writes each taken key at
+// (strict takes before it) + min(ties before it, ties).
+__device__ __forceinline__ int cta_emit_selection(const uint32_t* keys, int n, TopkThreshold th, int cur, int n_init,
+                                                  int n_local, int topk, int32_t* out, SdSmem& S) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int R = ((n + kSdThreads - 1) / kSdThreads) | 1;
+  const int j0 = min(tid * R, n), j1 = min(j0 + R, n);
+  const bool simple = topk_simple(th);  // no tie ranks: take forced or key >= take_from(th)
+  const uint32_t lo = simple ? take_from(th) : th.key + 1u;  // strict takes: key >= lo (T < 0xffffffff here)
+  const uint32_t tkey = th.key;
+  const int ties = simple ? 0 : th.ties;
+  auto forced = [&](int j) { return j < n_init || j > cur - n_local; };
+  int a = 0, b = 0;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t k = keys[j];
+    const bool f = forced(j);
+    a += (f || k >= lo) ? 1 : 0;
+    b += (!simple && !f && k == tkey) ? 1 : 0;
   }
-  // tie ranks first: S.tie_base[s] + warp part, recomputed per slot below
-  auto tie = [&](int s) {
-    int j;
-    const uint32_t k = key_at(s, j);
-    return j < n && k == th.key;
-  };
-  slot_counts(tie);
-  for (int s = 0; s < R; ++s) {  // keep each slot's tie base for this thread's warp
-    const bool f = tie(s);
-    const int rk = rank_of(s, __ballot_sync(0xffffffffu, f));
-    int j;
-    const uint32_t k = key_at(s, j);
-    tflag[s * kSdThreads + threadIdx.x] = static_cast<unsigned char>(
-        j < n && (forced(j) || k > th.key || (k == th.key && rk < th.ties)) ? 1 : 0);
+  int ia = a, ib = b;  // inclusive scans over the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ya;
+      ib += yb;
+    }
+  }
+  if (lane == 31) {
+    S.wc[0][warp] = ia;
+    S.wc[1][warp] = ib;
   }
   __syncthreads();
-  auto take = [&](int s) { return tflag[s * kSdThreads + threadIdx.x] != 0; };
-  const int total = slot_counts(take);
-  for (int s = 0; s < R; ++s) {
-    const bool f = take(s);
-    const int pos = rank_of(s, __ballot_sync(0xffffffffu, f));
-    if (f && pos < topk) out[pos] = static_cast<int>(threadIdx.x) + kSdThreads * s;
+  int sa = ia - a, sb = ib - b, ta = 0, tb = 0;
+#pragma unroll
+  for (int w = 0; w < kSdWarps; ++w) {
+    const int x = S.wc[0][w], y = S.wc[1][w];
+    if (w < warp) {
+      sa += x;
+      sb += y;
+    }
+    ta += x;
+    tb += y;
   }
-  for (int e = total + static_cast<int>(threadIdx.x); e < topk; e += kSdThreads) out[e] = -1;
-  __syncthreads();
+  const int total = min(ta + min(tb, ties), topk);
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t k = keys[j];
+    const bool f = forced(j);
+    const bool st = f || k >= lo;
+    const bool ti = !simple && !f && k == tkey;
+    const int pos = sa + min(sb, ties);
+    if ((st || (ti && sb < ties)) && pos < topk) out[pos] = j;
+    sa += st ? 1 : 0;
+    sb += ti ? 1 : 0;
+  }
+  for (int e = total + tid; e < topk; e += kSdThreads) out[e] = -1;
+  __syncthreads();  // S.wc is free again; out is complete
+  return total;
 }
 
 // Phase 1, all threads of the CTA: barrier set-up, then this CTA's Kc tiles streamed and
@@ -493,14 +462,16 @@ __device__ __forceinline__ void sd_score_chunk(const CUtensorMap* tm_kc, const S
 
 // Phase 2, after a cluster barrier that follows phase 1 in every CTA: the log-sum-exp per
 // head from every CTA's state, the previous CTA's carry, and the keys of this CTA's blocks
-// stored into CTA 0's key array (`scratch` is this CTA's own address of the selection
-// scratch), with their candidate count, AND and OR added into CTA 0's; CTA 0 also zeroes
-// the first digit histogram of its threshold search.
+// stored into CTA 0's key array (kAll: into every CTA's), with their candidate count, AND
+// and OR added into the same CTAs' (`scratch` is this CTA's own address of the selection
+// scratch); each CTA that will select zeroes the first digit histogram of its threshold
+// search.
+template <bool kAll>
 __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group& cluster, const SelDecodeParams& p,
                                               const SdItem& it, unsigned char* scratch, const uint32_t* bm,
                                               SdSmem& S) {
   uint32_t* keys = reinterpret_cast<uint32_t*>(scratch + kSdKeysOff);
-  if (it.c == 0) {
+  if (kAll || it.c == 0) {
     uint32_t* hist = reinterpret_cast<uint32_t*>(scratch + kSdHistOff);
     for (int i = threadIdx.x; i < kSdHistBins; i += kSdThreads) hist[i] = 0u;
   }
@@ -516,7 +487,7 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
     S.carry[h] = c > 0 ? ord_dec(cluster.map_shared_rank(const_cast<uint32_t*>(bm), c - 1)[h * kSdBStride + nq])
                        : -INFINITY;
   }
-  if (c == 0) {  // zero padding up to a multiple of 4 keys
+  if (kAll || c == 0) {  // zero padding up to a multiple of 4 keys
     for (int j = cur + 1 + threadIdx.x; j < ((cur + 4) & ~3); j += kSdThreads) keys[j] = 0u;
   }
   __syncthreads();
@@ -532,7 +503,6 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
   }
   __syncthreads();
   // this CTA's blocks: [c nq, (c + 1) nq); the last CTA also takes the rest up to cur
-  uint32_t* keys0 = cluster.map_shared_rank(keys, 0);
   const int jb0 = c * nq;
   const int jb1 = c == C - 1 ? cur + 1 : min(jb0 + nq, cur + 1);
   int cnt = 0;
@@ -551,7 +521,11 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
       }
       key = score_key(sc, p.score_mode);
     }
-    keys0[j] = key;
+    if (kAll) {
+      for (int r = 0; r < C; ++r) cluster.map_shared_rank(keys, r)[j] = key;
+    } else {
+      cluster.map_shared_rank(keys, 0)[j] = key;
+    }
     if (key != 0u) {
       ++cnt;
       kand &= key;
@@ -562,27 +536,30 @@ __device__ __forceinline__ void sd_block_keys(cooperative_groups::cluster_group&
   kand = __reduce_and_sync(0xffffffffu, kand);
   kor = __reduce_or_sync(0xffffffffu, kor);
   if ((threadIdx.x & 31) == 0 && cnt > 0) {
-    atomicAdd(cluster.map_shared_rank(&S.kcnt, 0), cnt);
-    atomicAnd(cluster.map_shared_rank(&S.kand, 0), kand);
-    atomicOr(cluster.map_shared_rank(&S.kor, 0), kor);
+    for (int r = 0; r < (kAll ? C : 1); ++r) {
+      atomicAdd(cluster.map_shared_rank(&S.kcnt, r), cnt);
+      atomicAnd(cluster.map_shared_rank(&S.kand, r), kand);
+      atomicOr(cluster.map_shared_rank(&S.kor, r), kor);
+    }
   }
 }
 
-// Phase 3, CTA 0 after a cluster barrier that follows phase 2 in every CTA: the top-k of
-// the keys in `scratch` (kSdScratchBytes, the drained tile ring) and the ascending list,
-// -1 padded, written to out[0 .. topk) (global or shared memory).  Ends after a CTA barrier.
-__device__ __forceinline__ void sd_select(const SelDecodeParams& p, const SdItem& it, unsigned char* scratch,
-                                          int32_t* out, SdSmem& S) {
+// Phase 3, a CTA that holds every key, after a cluster barrier that follows phase 2 in
+// every CTA: the top-k of the keys in `scratch` (kSdScratchBytes, the drained tile ring)
+// and the ascending list, -1 padded, written to out[0 .. topk) (global or shared memory);
+// returns the number of blocks in it.  Ends after a CTA barrier.
+__device__ __forceinline__ int sd_select(const SelDecodeParams& p, const SdItem& it, unsigned char* scratch,
+                                         int32_t* out, SdSmem& S) {
   const uint32_t* keys = reinterpret_cast<const uint32_t*>(scratch + kSdKeysOff);
   if (it.cur < 0) {
     for (int e = threadIdx.x; e < p.topk; e += kSdThreads) out[e] = -1;
     __syncthreads();
-    return;
+    return 0;
   }
   const int want = p.topk - forced_count(it.cur, p.n_init, p.n_local);
   const TopkThreshold th =
       cta_topk_threshold(keys, it.cur + 1, want, reinterpret_cast<uint32_t*>(scratch + kSdHistOff), S);
-  cta_emit_selection(keys, it.cur + 1, th, it.cur, p.n_init, p.n_local, p.topk, out, scratch + kSdFlagOff, S);
+  return cta_emit_selection(keys, it.cur + 1, th, it.cur, p.n_init, p.n_local, p.topk, out, S);
 }
 
 // grid = C * B * Hkv (cluster r serves item r), cluster = (C, 1, 1), block = 160.
@@ -603,7 +580,7 @@ __global__ void __launch_bounds__(kSdThreads)
   const SdItem it = sd_item(p, C, c, bg, min(max(p.lens[bg / p.Hkv], 0), p.Lmax));
   sd_score_chunk(&tm_kc, p, it, ring, bm, S);
   cluster.sync();  // every CTA's tiles are consumed and its partial state is final
-  sd_block_keys(cluster, p, it, ring, bm, S);
+  sd_block_keys<false>(cluster, p, it, ring, bm, S);
   cluster.sync();  // CTA 0 holds every key; no CTA reads a peer's shared memory after this
   if (c != 0) return;
   sd_select(p, it, ring, p.idx + it.bg * p.topk, S);
