@@ -20,7 +20,9 @@
 //          tile's dV / dK, so the tensor pipe overlaps the epilogue;
 //   warps 0-3, thread = TMEM lane = tile row: P and dS of its row (64 keys; keys past
 //          the row's position, padding heads and padding tokens give 0), written as bf16
-//          rows of 128 bytes (the MN-major B operands of the dV / dK products).
+//          rows of 128 bytes (the MN-major B operands of the dV / dK products) into one of
+//          two buffer pairs, so a tile's epilogue runs while the previous tile's dV / dK
+//          products read the other pair.
 // At the end of a segment the epilogue reads dV^T and dK^T (thread = dimension d, 64
 // keys) and adds them to the fp32 workspace (float atomics, coalesced over d: a block's
 // segments run on different CTAs).
@@ -36,6 +38,8 @@ constexpr int kBtTileBytes = 2 * kBtHalfBytes;     // 128 rows x 128 bf16: 32 KB
 constexpr int kBtStages = 2;                       // Q + dO tile pairs in flight
 constexpr int kBtStageBytes = 2 * kBtTileBytes;    // Q tile, then dO tile: 64 KB
 constexpr int kBtPBytes = 128 * 128;               // P or dS: 128 rows x 64 keys bf16 = 16 KB
+constexpr int kBtPBufs = 2;                        // P / dS buffer pairs: a tile's epilogue overlaps the
+                                                   // previous tile's dV / dK products
 constexpr int kBtEpiWarps = 4;
 constexpr int kBtTmaWarp = kBtEpiWarps, kBtMmaWarp = kBtEpiWarps + 1;
 constexpr int kBtThreads = 32 * (kBtEpiWarps + 2);
@@ -45,14 +49,14 @@ constexpr uint32_t kBtColS = 0, kBtColDP = 128, kBtColDV = 256, kBtColDK = 320;
 
 struct BtSmem {
   uint64_t kv_full, kv_empty, t_full[kBtStages], t_empty[kBtStages], sdp_full[2], sdp_empty[2];
-  uint64_t pds_full, pds_empty, acc_full, acc_empty, mma_done;
+  uint64_t pds_full[kBtPBufs], pds_empty[kBtPBufs], acc_full, acc_empty, mma_done;
   uint32_t tmem_base;
   volatile int abort;
 };
 
 constexpr size_t bwd_dkdv_tc_smem_bytes() {
   return 1024 + static_cast<size_t>(kAttnStageBytes) + static_cast<size_t>(kBtStages) * kBtStageBytes +
-         2 * static_cast<size_t>(kBtPBytes) + sizeof(BtSmem);
+         2 * kBtPBufs * static_cast<size_t>(kBtPBytes) + sizeof(BtSmem);
 }
 static_assert(bwd_dkdv_tc_smem_bytes() <= 227 * 1024, "shared memory of one CTA");
 
@@ -65,9 +69,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   unsigned char* base = align_smem(smem_raw, 1024);
   unsigned char* kv = base;                              // K block (16 KB) then V block (16 KB)
   unsigned char* tiles = kv + kAttnStageBytes;           // ring: Q tile then dO tile per stage
-  unsigned char* pbuf = tiles + kBtStages * kBtStageBytes;
-  unsigned char* dsbuf = pbuf + kBtPBytes;
-  BtSmem& S = *reinterpret_cast<BtSmem*>(dsbuf + kBtPBytes);
+  unsigned char* pbuf = tiles + kBtStages * kBtStageBytes;  // P of buffer x at pbuf + 2 x kBtPBytes,
+                                                            // dS right after it
+  BtSmem& S = *reinterpret_cast<BtSmem*>(pbuf + 2 * kBtPBufs * kBtPBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_entries = p.B * p.Hkv * p.nblk;
   const int total = p.segoff[n_entries];
@@ -83,8 +87,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       mbar_init(&S.sdp_full[s], 1);
       mbar_init(&S.sdp_empty[s], kBtEpiWarps);
     }
-    mbar_init(&S.pds_full, kBtEpiWarps);
-    mbar_init(&S.pds_empty, 1);
+    for (int s = 0; s < kBtPBufs; ++s) {
+      mbar_init(&S.pds_full[s], kBtEpiWarps);
+      mbar_init(&S.pds_empty[s], 1);
+    }
     mbar_init(&S.acc_full, 1);
     mbar_init(&S.acc_empty, kBtEpiWarps);
     mbar_init(&S.mma_done, 1);
@@ -170,16 +176,14 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       constexpr uint32_t id_rk = idesc_bf16_f32(128, 64, false, false);  // rows x keys, both K-major
       constexpr uint32_t id_dk = idesc_bf16_f32(128, 64, true, true);    // dims x keys, both MN-major
       const uint32_t kb = smem_u32(kv), vb = kb + kKvTileBytes;
-      const uint32_t pb = smem_u32(pbuf), db = smem_u32(dsbuf);
+      const uint32_t pb0 = smem_u32(pbuf);
       uint32_t gt = 0;  // tiles whose S / dP were issued
       int it = 0;
-      // S = Q K^T and dP = dO V^T of global tile n into buffer pair n & 1
+      // S = Q K^T and dP = dO V^T of global tile n into buffer pair n & 1 (its Q / dO tile
+      // has landed and the epilogue has read the pair's previous contents)
       auto issue_sdp = [&](uint32_t n) {
         const int st = static_cast<int>(n & 1u);
         const uint32_t sb = n & 1u;
-        mbar_wait(&S.t_full[st], (n >> 1) & 1u, &S.abort);
-        if (n >= 2) mbar_wait(&S.sdp_empty[sb], ((n >> 1) - 1u) & 1u, &S.abort);  // the epilogue read it
-        tc_fence_after();
         const uint32_t qa = smem_u32(tiles + st * kBtStageBytes), da = qa + kBtTileBytes;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -196,37 +200,82 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         }
         umma_commit(&S.sdp_full[sb]);
       };
+      // dV^T += dO^T P and dK^T += Q^T dS of global tile n (first = the segment's first tile)
+      auto issue_dvdk = [&](uint32_t n, bool first) {
+        const uint32_t x = n % kBtPBufs;
+        const uint32_t pb = pb0 + 2u * x * kBtPBytes, db = pb + kBtPBytes;
+        const uint32_t qa = smem_u32(tiles + static_cast<int>(n & 1u) * kBtStageBytes), da = qa + kBtTileBytes;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // 16 rows per step
+          umma_bf16(tmem + kBtColDV, desc_mn_sw128(da + k * 2048, kBtHalfBytes, 1024),
+                    desc_mn_sw128(pb + k * 2048, kBtPBytes, 1024), id_dk, (!first || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_bf16(tmem + kBtColDK, desc_mn_sw128(qa + k * 2048, kBtHalfBytes, 1024),
+                    desc_mn_sw128(db + k * 2048, kBtPBytes, 1024), id_dk, (!first || k > 0) ? 1u : 0u);
+        umma_commit(&S.pds_empty[x]);                       // P / dS of buffer x may be rewritten
+        umma_commit(&S.t_empty[static_cast<int>(n & 1u)]);  // the Q / dO tile is no longer read
+      };
+      // Within a segment the two kinds of products are issued as soon as their inputs are
+      // ready, neither waiting behind the other: a tile's dV / dK never waits for the next
+      // tile's Q / dO rows to land (which would chain the gather latency onto every tile).
+      // Each barrier is tested only after its previous phase was seen, so a parity test
+      // cannot alias.
       for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
         const int e = bwd_find_entry(p.segoff, n_entries, item);
         const int seg = item - p.segoff[e];
         const int r0 = seg * kBwdSeg, nrows = min(kBwdSeg, p.cnt[e] - r0);
-        const int ntiles = (nrows + kBtTok - 1) / kBtTok;
-        mbar_wait(&S.kv_full, static_cast<uint32_t>(it) & 1u, &S.abort);
+        const uint32_t ntiles = static_cast<uint32_t>((nrows + kBtTok - 1) / kBtTok);
+        if (!mbar_wait(&S.kv_full, static_cast<uint32_t>(it) & 1u, &S.abort)) break;
         tc_fence_after();
         const uint32_t g0 = gt;
-        issue_sdp(gt++);
-        for (int ti = 0; ti < ntiles; ++ti) {
-          if (ti + 1 < ntiles) {
-            issue_sdp(gt++);
-          } else {
-            umma_commit(&S.kv_empty);  // every read of the block's K / V has been issued
+        uint32_t ns = 0, nd = 0;  // tiles of the segment whose S / dP, dV / dK were issued
+        bool acc_free = it == 0;  // the epilogue has read the previous segment's dV^T / dK^T
+        uint32_t idle = 0;
+        uint64_t t_idle = 0;
+        while (nd < ntiles) {
+          bool progress = false;
+          if (ns < ntiles) {
+            const uint32_t n = g0 + ns, st = n & 1u;
+            if (mbar_test(&S.t_full[st], (n >> 1) & 1u) &&
+                (n < 2 || mbar_test(&S.sdp_empty[st], ((n >> 1) - 1u) & 1u))) {
+              tc_fence_after();
+              issue_sdp(n);
+              if (++ns == ntiles) umma_commit(&S.kv_empty);  // every read of the block's K / V was issued
+              progress = true;
+            }
           }
-          const uint32_t n = g0 + static_cast<uint32_t>(ti);
-          if (ti == 0 && it > 0) mbar_wait(&S.acc_empty, static_cast<uint32_t>(it - 1) & 1u, &S.abort);
-          mbar_wait(&S.pds_full, n & 1u, &S.abort);  // P and dS of tile n are in shared memory
-          tc_fence_after();
-          const uint32_t qa = smem_u32(tiles + static_cast<int>(n & 1u) * kBtStageBytes), da = qa + kBtTileBytes;
-#pragma unroll
-          for (int k = 0; k < 8; ++k)  // 16 rows per step
-            umma_bf16(tmem + kBtColDV, desc_mn_sw128(da + k * 2048, kBtHalfBytes, 1024),
-                      desc_mn_sw128(pb + k * 2048, kBtPBytes, 1024), id_dk, (ti > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_bf16(tmem + kBtColDK, desc_mn_sw128(qa + k * 2048, kBtHalfBytes, 1024),
-                      desc_mn_sw128(db + k * 2048, kBtPBytes, 1024), id_dk, (ti > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&S.pds_empty);                    // P / dS may be rewritten
-          umma_commit(&S.t_empty[static_cast<int>(n & 1u)]);  // the Q / dO tile is no longer read
+          if (nd < ns) {
+            const uint32_t n = g0 + nd;
+            if (!acc_free) acc_free = mbar_test(&S.acc_empty, static_cast<uint32_t>(it - 1) & 1u);
+            if (acc_free && mbar_test(&S.pds_full[n % kBtPBufs], (n / kBtPBufs) & 1u)) {
+              tc_fence_after();
+              issue_dvdk(n, nd == 0);
+              ++nd;
+              progress = true;
+            }
+          }
+          if (progress) {
+            idle = 0;
+            t_idle = 0;
+          } else if (++idle == 64u) {  // bounded: give up like mbar_wait
+            idle = 0;
+            if (S.abort || (*reinterpret_cast<volatile unsigned int*>(&g_device_error) & kDevErrWaitTimeout) != 0u) {
+              S.abort = 1;
+              break;
+            }
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) {
+              t_idle = now;
+            } else if (now - t_idle > kWaitLimitNs) {
+              S.abort = 1;
+              atomicOr(&g_device_error, kDevErrWaitTimeout);
+              break;
+            }
+          }
         }
+        gt = g0 + ns;
+        if (S.abort) break;
         umma_commit(&S.acc_full);  // dV^T and dK^T of the segment are complete
       }
       umma_commit(&S.mma_done);
@@ -273,8 +322,12 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       const int t = t_n;
       const float lse2 = lse2_n, dl = dl_n;
       if (ti + 1 < ntiles) load_row(ti + 1, t_n, lse2_n, dl_n);
+      const uint32_t x = gt % kBtPBufs;
+      unsigned char* pbx = pbuf + 2 * x * kBtPBytes;
+      unsigned char* dsx = pbx + kBtPBytes;
       mbar_wait(&S.sdp_full[sb], (gt >> 1) & 1u, &S.abort);
-      if (gt > 0) mbar_wait(&S.pds_empty, (gt - 1u) & 1u, &S.abort);  // dV / dK of the previous tile done
+      if (gt >= kBtPBufs)  // dV / dK of the tile that last used buffer x are done
+        mbar_wait(&S.pds_empty[x], (gt / kBtPBufs - 1u) & 1u, &S.abort);
       tc_fence_after();
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
@@ -298,9 +351,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // four 16-byte chunks of this row's 32 keys
           const int chunk = 4 * half + q;
-          *reinterpret_cast<uint4*>(pbuf + sw128(row, chunk)) =
+          *reinterpret_cast<uint4*>(pbx + sw128(row, chunk)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-          *reinterpret_cast<uint4*>(dsbuf + sw128(row, chunk)) =
+          *reinterpret_cast<uint4*>(dsx + sw128(row, chunk)) =
               make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
         }
       }
@@ -309,7 +362,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&S.sdp_empty[sb]);
-        mbar_arrive(&S.pds_full);
+        mbar_arrive(&S.pds_full[x]);
       }
     }
     // the segment's dV^T and dK^T: thread = dimension d, columns = the block's 64 keys
