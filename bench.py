@@ -574,8 +574,8 @@ def run_extras(args, device, pk, peak_src):
     out["backward_32k"] = {"workload": "prefill_32k (B=1, L=32768, 32/2 heads, top-96)", "ms": ms_bwd,
                            "tflops": bwd_flops / ms_bwd / 1e9, "frac": bwd_flops / ms_bwd / 1e9 / tc_peak,
                            "algorithmic_flops": bwd_flops,
-                           "note": "kernels run 7 products (S and dP are recomputed in both passes), "
-                                   "on m16n8k16 tensor-core MMAs"}
+                           "note": "kernels run 7 products (S and dP are recomputed in both passes): "
+                                   "dq on m16n8k16 MMAs, dK / dV on tcgen05 (TMEM accumulators)"}
     del q, k, v, d_o, o, lse, idx, kc, ws
     torch.cuda.empty_cache()
     return out
@@ -641,15 +641,28 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def profile_run(name, device):
+def profile_run(name, device, backward=False):
     """The hot path of one workload, twice (a warm-up and one more run), for single-kernel
     profiler captures: prefill (compress, select, attend) or a decode step (compress the
     caches, then the fused step, then the separate selection and attention calls on the
-    same inputs).  Prints nothing."""
+    same inputs); with `backward` (prefill workloads), the forward once and then the
+    backward twice, with the upstream gradient of the bench's backward line.  Prints
+    nothing."""
     wl = WORKLOADS[name]
     p = ops.Params.from_workload(wl)
     x = make_inputs(wl, seed=0)
     q, k, v = x.q.to(device), x.k.to(device), x.v.to(device)
+    if backward:
+        assert wl.mode == "prefill", "the backward runs on prefill workloads"
+        g = torch.Generator().manual_seed(7)
+        d_o = torch.randn(x.q.shape, generator=g).to(torch.bfloat16).to(device)
+        o, lse, idx, _ = ops.prefill(p, q, k, v)
+        ws = torch.empty(ops.workspace_size(p, 5, wl.seq_len), dtype=torch.uint8, device=device)
+        for _ in range(2):
+            ops.sparse_attn_backward(p, q, k, v, o, lse, d_o, idx, ws=ws)
+        torch.cuda.synchronize()
+        assert ops.device_error(clear=True) == 0
+        return
     for _ in range(2):
         if wl.mode == "prefill":
             ops.prefill(p, q, k, v)
@@ -682,11 +695,13 @@ def main():
     ap.add_argument("--reference-rows", type=int, default=96)
     ap.add_argument("--profile-run", default=None, metavar="WORKLOAD",
                     help="run WORKLOAD's hot path twice and exit (for profiler captures)")
+    ap.add_argument("--profile-backward", action="store_true",
+                    help="with --profile-run: the forward once, then the backward twice")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.profile_run:
         lib_build.build()
-        profile_run(args.profile_run, torch.device("cuda", 0))
+        profile_run(args.profile_run, torch.device("cuda", 0), backward=args.profile_backward)
         return
 
     ri = dist.rank_info()
