@@ -63,6 +63,7 @@ KERNEL_SOURCES = {
     "attn_decode_cluster_kernel": ["attn_dec.cuh", "attn.cuh", "common.cuh", "infllmv2.cu"],
     "decode_step_kernel": ["decode_step.cuh", "select_decode.cuh", "attn_dec.cuh", "select_prefill.cuh", "topk.cuh",
                            "attn.cuh", "common.cuh", "infllmv2.cu"],
+    "bwd_dkdv_tc_kernel": ["attn_bwd_tc.cuh", "attn_bwd.cuh", "attn.cuh", "tcgen05.cuh", "common.cuh", "infllmv2.cu"],
 }
 
 
@@ -574,6 +575,7 @@ def run_extras(args, device, pk, peak_src):
     out["backward_32k"] = {"workload": "prefill_32k (B=1, L=32768, 32/2 heads, top-96)", "ms": ms_bwd,
                            "tflops": bwd_flops / ms_bwd / 1e9, "frac": bwd_flops / ms_bwd / 1e9 / tc_peak,
                            "algorithmic_flops": bwd_flops,
+                           "dkdv_kernel_traffic": dram_traffic("bwd_dkdv_tc_kernel", "prefill_32k backward"),
                            "note": "kernels run 7 products (S and dP are recomputed in both passes): "
                                    "dq on m16n8k16 MMAs, dK / dV on tcgen05 (TMEM accumulators)"}
     del q, k, v, d_o, o, lse, idx, kc, ws
