@@ -14,12 +14,13 @@
 //      the previous CTA's carry into its first block (both read through distributed
 //      shared memory, all loads in parallel), computes S(j) = sum_h exp(m_h(j) - lse_h)
 //      (or, with logit-sum scoring, sum_h m_h(j)) for its blocks and stores the keys into
-//      CTA 0 (with inside pooling block j pools kernels 4j .. 4j+2 only, and no carry);
-//   3. CTA 0 finds the k-th largest key: the candidates' common leading bits come from
-//      one AND / OR reduction, the bits below them from shared-memory histograms of
-//      11-bit digits (a suffix scan picks the digit that holds the k-th key; once its
-//      bucket holds at most 32 keys they are ranked directly), and all its threads
-//      write the ascending list (prefix sums place ties and outputs).
+//      CTA 0 -- in the fused decode step into every CTA of the cluster -- (with inside
+//      pooling block j pools kernels 4j .. 4j+2 only, and no carry);
+//   3. a CTA that holds every key finds the k-th largest: the candidates' common leading
+//      bits come from one AND / OR reduction, the bits below them from shared-memory
+//      histograms of 11-bit digits (a suffix scan picks the digit that holds the k-th key;
+//      once its bucket holds at most 32 keys they are ranked directly), and all its
+//      threads write the ascending list (one scan places ties and outputs).
 // The phases are device functions: select_decode_kernel runs them alone, the fused decode
 // step (decode_step.cuh) runs them before the attention in the same cluster.
 // No workspace, one launch; reading Kc once bounds it (HBM).
@@ -40,14 +41,12 @@ constexpr int kSdMaxChunk = 2048;  // kernels per CTA at most
 constexpr int kSdMaxQuads = kSdMaxChunk / 4;
 constexpr int kSdBStride = kSdMaxQuads + 4;  // per-head block-max rows (quads + 1 carry), padded
 constexpr int kSdMaxCluster = 16;
-// CTA 0's top-k visits the keys slot-major: thread i takes keys i + kSdThreads s.
 constexpr int kSdMaxKeys = INFLLMV2_MAX_SEQ_LEN / kBlock;
-constexpr int kSdMaxR = (kSdMaxKeys + kSdThreads - 1) / kSdThreads;
 constexpr int kSdHistBits = 11;  // digit width of the threshold search
 constexpr int kSdHistBins = 1 << kSdHistBits;
 constexpr int kSdBinsPerThread = (kSdHistBins + kSdThreads - 1) / kSdThreads;
-// CTA 0's selection scratch, in its drained tile ring: block keys, the digit histogram
-// and the take flags of a tie-ranked emission
+// The selection scratch of a CTA that selects, in its drained tile ring: block keys and
+// the digit histogram
 constexpr int kSdKeysOff = 0;
 constexpr int kSdHistOff = kSdKeysOff + 4 * kSdMaxKeys;
 constexpr int kSdScratchBytes = kSdHistOff + 4 * kSdHistBins;
@@ -71,19 +70,17 @@ struct SdSmem {
   float pm[kSdMaxCluster][kGroupRows], pl[kSdMaxCluster][kGroupRows];  // every CTA's, gathered
   float lse2[kGroupRows];  // log2-sum-exp2 per head over the whole sequence
   float carry[kGroupRows];  // previous CTA's last kernel, for this CTA's first block
-  int kcnt;                            // CTA 0: candidates among the keys, and the AND / OR of
-  unsigned int kand, kor;              // their keys (every CTA adds its blocks' through DSMEM)
-  int wsum[kSdWarps];                  // per-warp histogram totals of the digit search
-  int dig, dig_above, dig_in;          // the digit found, keys above its bin, keys in it
-  int wc[kSdMaxR][kSdWarps];          // per (slot, warp) counts of the emission
-  int sbase[kSdMaxR];                 // flagged keys in earlier slots
-  int total;
+  int kcnt;                    // a selecting CTA: candidates among the keys, and the AND / OR of
+  unsigned int kand, kor;      // their keys (every CTA adds its blocks' through DSMEM)
+  int wsum[kSdWarps];          // per-warp histogram totals of the digit search
+  int dig, dig_above, dig_in;  // the digit found, keys above its bin, keys in it
+  int wc[2][kSdWarps];         // per-warp counts of the emission (strict takes, ties)
   int nlist;
   uint32_t list[32];
   volatile int abort;
 };
 
-// Tile ring (reused by CTA 0 as the selection scratch) and per-head block maxima.
+// Tile ring (reused as the selection scratch) and per-head block maxima.
 constexpr size_t kSdRegionBytes =
     static_cast<size_t>(kSdStages) * kKcTileBytes + static_cast<size_t>(kGroupRows) * kSdBStride * 4;
 
@@ -322,7 +319,7 @@ __device__ __forceinline__ void sd_score_chunk(const CUtensorMap* tm_kc, const S
       mbar_init(&S.empty[s], kSdConsumers);
     }
     S.abort = 0;
-    S.kcnt = 0;  // CTA 0's are filled by every CTA of the cluster after the next cluster barrier
+    S.kcnt = 0;  // a selecting CTA's are filled by every CTA of the cluster after the next cluster barrier
     S.kand = 0xffffffffu;
     S.kor = 0u;
     fence_mbar_init();
